@@ -1,0 +1,292 @@
+"""IsoQuant fp64 CPU oracle: ctypes shim over ``isoq_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference arm may import this package.  It shares no code
+with the CUDA library and never imports the product package.
+
+Every function follows the method page "RotaryQuant: Fitting 120B MoE Models on Consumer
+Hardware via Fused Compressed-Space Attention", Abstract (WHT, block-diagonal SO(4)
+rotations, 3-bit scalar quantisation, attention on the packed tensors); the readings the
+pages leave open are listed at the top of ``isoq_oracle.c``.  All arithmetic is fp64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "isoq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libisoq_oracle.so")
+
+_GCC_FLAGS = ["-O2", "-std=gnu11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+              "-fno-fast-math"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain -O2, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _declare(_lib)
+    return _lib
+
+
+_d = ctypes.c_double
+_i = ctypes.c_int
+_p = ctypes.c_void_p
+
+
+def _declare(L):
+    L.ref_level.restype = _d
+    L.ref_level.argtypes = [_i]
+    L.ref_threshold.restype = _d
+    L.ref_threshold.argtypes = [_i]
+    L.ref_num_threads.restype = _i
+    L.ref_splitmix64_next.restype = ctypes.c_uint64
+    L.ref_splitmix64_next.argtypes = [_p]
+    L.ref_normal.restype = _d
+    L.ref_normal.argtypes = [_p]
+    L.ref_make_params.restype = None
+    L.ref_make_params.argtypes = [ctypes.c_uint64, _i, _i, _p, _p]
+    L.ref_wht.restype = None
+    L.ref_wht.argtypes = [_p, _i]
+    L.ref_quat_mul.restype = None
+    L.ref_quat_mul.argtypes = [_p, _p, _p]
+    L.ref_so4_forward.restype = None
+    L.ref_so4_forward.argtypes = [_p, _p, _p, _p]
+    L.ref_so4_inverse.restype = None
+    L.ref_so4_inverse.argtypes = [_p, _p, _p, _p]
+    L.ref_rotate.restype = None
+    L.ref_rotate.argtypes = [_p, _p, _p, _i]
+    L.ref_unrotate.restype = None
+    L.ref_unrotate.argtypes = [_p, _p, _p, _i]
+    L.ref_fp16_bits.restype = ctypes.c_uint16
+    L.ref_fp16_bits.argtypes = [_d]
+    L.ref_fp16_value.restype = _d
+    L.ref_fp16_value.argtypes = [ctypes.c_uint16]
+    L.ref_quantize_vector.restype = _i
+    L.ref_quantize_vector.argtypes = [_p, _p, _i, _p, _p, _p]
+    L.ref_pack_codes.restype = None
+    L.ref_pack_codes.argtypes = [_p, _i, _p]
+    L.ref_unpack_codes.restype = None
+    L.ref_unpack_codes.argtypes = [_p, _i, _p]
+    L.ref_block_bytes.restype = ctypes.c_size_t
+    L.ref_block_bytes.argtypes = [_i, _i]
+    L.ref_quantize_append.restype = _i
+    L.ref_quantize_append.argtypes = [_p, _i, _i, _i, _p, _p, _i, _p, _p, _i, _p, _p]
+    L.ref_dequantize_slot.restype = None
+    L.ref_dequantize_slot.argtypes = [_p, _i, _i, _i, _p, _i, _i, _i, _i, _p]
+    L.ref_decode_attention.restype = None
+    L.ref_decode_attention.argtypes = [_p, _i, _i, _i, _p, _p, _i, _i, _i, _p, _p, _d, _p,
+                                       _p, _i]
+    L.ref_attention_full.restype = None
+    L.ref_attention_full.argtypes = [_i, _i, _i, _i, _p, _p, _p, _d, _p]
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+# ------------------------------------------------------------------------------------
+# Constants
+# ------------------------------------------------------------------------------------
+def levels() -> np.ndarray:
+    """The 8 codebook levels in N(0,1) units, ascending (Lloyd-Max, Max 1960)."""
+    return np.array([lib().ref_level(c) for c in range(8)])
+
+
+def thresholds() -> np.ndarray:
+    """The 7 decision thresholds: midpoints of adjacent levels."""
+    return np.array([lib().ref_threshold(j) for j in range(7)])
+
+
+def num_threads() -> int:
+    return int(lib().ref_num_threads())
+
+
+# ------------------------------------------------------------------------------------
+# Parameters and rotations
+# ------------------------------------------------------------------------------------
+def splitmix64_stream(seed: int, n: int) -> np.ndarray:
+    st = ctypes.c_uint64(seed)
+    return np.array([lib().ref_splitmix64_next(ctypes.byref(st)) for _ in range(n)],
+                    dtype=np.uint64)
+
+
+def normals(seed: int, n: int) -> np.ndarray:
+    st = ctypes.c_uint64(seed)
+    return np.array([lib().ref_normal(ctypes.byref(st)) for _ in range(n)])
+
+
+def make_params(seed: int, d: int, n_kv_heads: int):
+    """(params64, params32), each [n_kv_heads][d/4][2][4]: per block p then q (w,x,y,z)."""
+    p64 = np.zeros((n_kv_heads, d // 4, 2, 4), dtype=np.float64)
+    p32 = np.zeros((n_kv_heads, d // 4, 2, 4), dtype=np.float32)
+    lib().ref_make_params(ctypes.c_uint64(seed), d, n_kv_heads, _ptr(p64), _ptr(p32))
+    return p64, p32
+
+
+def wht(x) -> np.ndarray:
+    """Orthonormal natural-order WHT of each row of x (last axis = d)."""
+    x = _f64(x).copy()
+    flat = x.reshape(-1, x.shape[-1])
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        lib().ref_wht(_ptr(row), row.shape[0])
+        flat[r] = row
+    return flat.reshape(x.shape)
+
+
+def quat_mul(a, b) -> np.ndarray:
+    a, b = _f64(a), _f64(b)
+    out = np.zeros(4)
+    lib().ref_quat_mul(_ptr(a), _ptr(b), _ptr(out))
+    return out
+
+
+def so4_forward(p, q, y) -> np.ndarray:
+    p, q, y = _f64(p), _f64(q), _f64(y)
+    z = np.zeros(4)
+    lib().ref_so4_forward(_ptr(p), _ptr(q), _ptr(y), _ptr(z))
+    return z
+
+
+def so4_inverse(p, q, z) -> np.ndarray:
+    p, q, z = _f64(p), _f64(q), _f64(z)
+    y = np.zeros(4)
+    lib().ref_so4_inverse(_ptr(p), _ptr(q), _ptr(z), _ptr(y))
+    return y
+
+
+def rotate(params_head, x) -> np.ndarray:
+    """z = R x for one head: WHT then the SO(4) blocks.  params_head: [d/4][2][4]."""
+    ph, x = _f64(params_head), _f64(x)
+    z = np.zeros_like(x)
+    lib().ref_rotate(_ptr(ph), _ptr(x), _ptr(z), x.shape[-1])
+    return z
+
+
+def unrotate(params_head, z) -> np.ndarray:
+    ph, z = _f64(params_head), _f64(z)
+    x = np.zeros_like(z)
+    lib().ref_unrotate(_ptr(ph), _ptr(z), _ptr(x), z.shape[-1])
+    return x
+
+
+# ------------------------------------------------------------------------------------
+# binary16
+# ------------------------------------------------------------------------------------
+def fp16_bits(v: float) -> int:
+    return int(lib().ref_fp16_bits(float(v)))
+
+
+def fp16_value(h: int) -> float:
+    return float(lib().ref_fp16_value(int(h)))
+
+
+# ------------------------------------------------------------------------------------
+# Quantisation and packing
+# ------------------------------------------------------------------------------------
+def quantize_vector(params_head, x):
+    """-> (codes uint8[d], norm16 bits, overflow flag, z fp64[d])."""
+    ph, x = _f64(params_head), _f64(x)
+    d = x.shape[0]
+    codes = np.zeros(d, dtype=np.uint8)
+    n16 = ctypes.c_uint16(0)
+    z = np.zeros(d)
+    ov = lib().ref_quantize_vector(_ptr(ph), _ptr(x), d, _ptr(codes), ctypes.byref(n16), _ptr(z))
+    return codes, int(n16.value), int(ov), z
+
+
+def pack_codes(codes) -> np.ndarray:
+    codes = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    d = codes.shape[0]
+    out = np.zeros(3 * d // 8, dtype=np.uint8)
+    lib().ref_pack_codes(_ptr(codes), d, _ptr(out))
+    return out
+
+
+def unpack_codes(packed, d: int) -> np.ndarray:
+    packed = np.ascontiguousarray(np.asarray(packed, dtype=np.uint8))
+    codes = np.zeros(d, dtype=np.uint8)
+    lib().ref_unpack_codes(_ptr(packed), d, _ptr(codes))
+    return codes
+
+
+def block_bytes(d: int, page: int = 64) -> int:
+    return int(lib().ref_block_bytes(d, page))
+
+
+def quantize_append(params64, d, n_kv_heads, page, blocks, page_table, K, V, seq_ids,
+                    positions) -> int:
+    """Quantise K, V ([n_tokens][n_kv_heads][d]) into ``blocks`` (uint8, modified in place).
+    Returns the number of saturated norms."""
+    assert blocks.dtype == np.uint8 and blocks.flags.c_contiguous
+    pt = _i32(page_table)
+    K, V = _f64(K), _f64(V)
+    sid, pos = _i32(seq_ids), _i32(positions)
+    return int(lib().ref_quantize_append(_ptr(_f64(params64)), d, n_kv_heads, page,
+                                         _ptr(blocks), _ptr(pt), pt.shape[-1], _ptr(K),
+                                         _ptr(V), K.shape[0], _ptr(sid), _ptr(pos)))
+
+
+def dequantize_slot(params64, d, n_kv_heads, page, blocks, phys_page, kv_head, slot,
+                    kind) -> np.ndarray:
+    out = np.zeros(d)
+    lib().ref_dequantize_slot(_ptr(_f64(params64)), d, n_kv_heads, page,
+                              _ptr(np.ascontiguousarray(blocks)), phys_page, kv_head, slot,
+                              kind, _ptr(out))
+    return out
+
+
+def decode_attention(params64, d, n_kv_heads, page, blocks, page_table, seq_lens, Q, scale,
+                     sel=None) -> np.ndarray:
+    """Decode attention on the packed cache.  Q: [n_seqs][n_q_heads][d].  ``sel``: optional
+    list of (seq, q_head) pairs to compute (others stay NaN)."""
+    Q = _f64(Q)
+    n_seqs, n_q_heads = Q.shape[0], Q.shape[1]
+    pt = _i32(page_table)
+    sl = _i32(seq_lens)
+    out = np.full(Q.shape, np.nan)
+    selp, nsel = None, 0
+    if sel is not None:
+        sa = _i32(np.asarray(sel).reshape(-1, 2))
+        selp, nsel = _ptr(sa), sa.shape[0]
+    lib().ref_decode_attention(_ptr(_f64(params64)), d, n_kv_heads, page,
+                               _ptr(np.ascontiguousarray(blocks)), _ptr(pt), pt.shape[-1],
+                               n_seqs, n_q_heads, _ptr(sl), _ptr(Q), float(scale), _ptr(out),
+                               selp, nsel)
+    return out
+
+
+def attention_full(K, V, Q, scale) -> np.ndarray:
+    """Full-precision attention for one sequence: K, V [n_tok][n_kv][d], Q [n_q][d]."""
+    K, V, Q = _f64(K), _f64(V), _f64(Q)
+    n_tok, n_kv, d = K.shape
+    out = np.zeros((Q.shape[0], d))
+    lib().ref_attention_full(d, n_kv, Q.shape[0], n_tok, _ptr(K), _ptr(V), _ptr(Q),
+                             float(scale), _ptr(out))
+    return out

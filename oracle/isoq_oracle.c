@@ -1,0 +1,472 @@
+/*
+ * IsoQuant fp64 CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only the test suite, the package smoke check and the benchmark's CPU-baseline /
+ * reference arm may load this library.  The product path (the CUDA library and its
+ * Python binding) never calls it, and the two share no code, header, table or helper.
+ *
+ * What it computes follows the method page
+ *   "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
+ *    Compressed-Space Attention" (arXiv 2608.08081v1), Abstract:
+ * each per-token, per-head K/V vector is (1) normalised by a Walsh-Hadamard transform,
+ * (2) rotated by block-diagonal SO(4) rotations, (3) scalar-quantised to 3 bits; and
+ * attention runs directly on the packed 3-bit tensors, never materialising full
+ * precision K/V.  Page 1 ("FreeToken issue #141, unified KV cache backend", Proposed
+ * Solution, Quantization layer) says the rotations are quaternion rotations.
+ *
+ * The pages leave these steps open; this oracle takes the plainest reading of each:
+ *   - rotation parameters: one unit-quaternion pair (p, q) per 4-element block,
+ *     z = p * y * conj(q) (Hamilton product, components ordered w, x, y, z), drawn
+ *     Haar-uniformly from a SplitMix64 stream via Box-Muller; one set per KV head,
+ *     shared by K and V (the only reading that keeps 256 parameters per head at d=128);
+ *   - WHT: Sylvester (natural) order, scaled by 1/sqrt(d), no random sign diagonal;
+ *   - codebook: the 8-level Lloyd-Max quantiser for N(0,1) (J. Max, "Quantizing for
+ *     minimum distortion", IRE Trans. Inf. Theory IT-6, 1960) applied to
+ *     u = sqrt(d) * z / ||x||; thresholds are midpoints of adjacent levels; a value
+ *     exactly on a threshold takes the upper code; a zero vector has u = 0 (code 4);
+ *   - norm: the L2 norm of the input vector, stored as IEEE binary16 (round to
+ *     nearest even), saturating at 65504;
+ *   - dequantised coordinate: (stored fp16 norm / sqrt(d)) * level, no renormalisation;
+ *   - decode: softmax(scale * q.k) over positions 0..len-1 of each sequence, query head
+ *     h reading KV head h / G.
+ *
+ * Everything is plain fp64 scalar code in the order the method states it.  The only
+ * parallelism is an OpenMP loop over independent vectors / (sequence, head) pairs.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------------ */
+/* Codebook: Lloyd-Max 8-level quantiser for N(0,1) (Max, 1960), ascending.         */
+/* ------------------------------------------------------------------------------ */
+static const double REF_LEVELS[8] = {-2.1520, -1.3440, -0.7560, -0.2451,
+                                     0.2451,  0.7560,  1.3440,  2.1520};
+
+double ref_level(int code) { return REF_LEVELS[code]; }
+
+/* Threshold j (0..6) is the midpoint between levels j and j+1. */
+double ref_threshold(int j) { return 0.5 * (REF_LEVELS[j] + REF_LEVELS[j + 1]); }
+
+int ref_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Random rotation parameters.                                                      */
+/* SplitMix64: G. Steele, D. Lea, C. Flood, "Fast splittable pseudorandom number   */
+/* generators", OOPSLA 2014.  Box-Muller: G. Box, M. Muller, Ann. Math. Stat. 1958.  */
+/* ------------------------------------------------------------------------------ */
+uint64_t ref_splitmix64_next(uint64_t *state) {
+  *state += 0x9E3779B97F4A7C15ULL;
+  uint64_t z = *state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+/* One standard normal from two successive 64-bit draws: the top 53 bits of each give
+ * u1 in (0, 1] and u2 in [0, 1); the cosine branch of Box-Muller is used. */
+double ref_normal(uint64_t *state) {
+  const double two_m53 = 1.0 / 9007199254740992.0; /* 2^-53 */
+  uint64_t k1 = ref_splitmix64_next(state) >> 11;
+  uint64_t k2 = ref_splitmix64_next(state) >> 11;
+  double u1 = ((double)k1 + 1.0) * two_m53;
+  double u2 = (double)k2 * two_m53;
+  return sqrt(-2.0 * log(u1)) * cos(2.0 * M_PI * u2);
+}
+
+/* params: [n_kv_heads][d/4][2][4] = per block the unit quaternion p then q, each
+ * (w, x, y, z).  Each quaternion is four normals divided by their Euclidean length,
+ * which is uniform on the unit 3-sphere, so (p, q) -> (x -> p x conj(q)) is Haar on
+ * SO(4).  params32 (optional) receives the same values rounded to binary32. */
+void ref_make_params(uint64_t seed, int d, int n_kv_heads, double *params, float *params32) {
+  uint64_t state = seed;
+  int nblk = d / 4;
+  for (int h = 0; h < n_kv_heads; h++)
+    for (int b = 0; b < nblk; b++)
+      for (int which = 0; which < 2; which++) {
+        double g[4], s = 0.0;
+        for (int c = 0; c < 4; c++) {
+          g[c] = ref_normal(&state);
+          s += g[c] * g[c];
+        }
+        double len = sqrt(s);
+        for (int c = 0; c < 4; c++) {
+          size_t idx = (((size_t)h * nblk + b) * 2 + which) * 4 + c;
+          params[idx] = g[c] / len;
+          if (params32) params32[idx] = (float)(g[c] / len);
+        }
+      }
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Walsh-Hadamard transform, natural (Sylvester) order, orthonormal (1/sqrt(d)).    */
+/* The O(d log d) butterfly: at stride h, pairs (j, j+h) become (a+b, a-b).         */
+/* ------------------------------------------------------------------------------ */
+void ref_wht(double *x, int d) {
+  for (int h = 1; h < d; h *= 2)
+    for (int i = 0; i < d; i += 2 * h)
+      for (int j = i; j < i + h; j++) {
+        double a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+  double s = 1.0 / sqrt((double)d);
+  for (int i = 0; i < d; i++) x[i] *= s;
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Quaternions (w, x, y, z), Hamilton convention i^2 = j^2 = k^2 = ijk = -1.        */
+/* ------------------------------------------------------------------------------ */
+void ref_quat_mul(const double *a, const double *b, double *out) {
+  double w = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
+  double x = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
+  double y = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
+  double z = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
+  out[0] = w;
+  out[1] = x;
+  out[2] = y;
+  out[3] = z;
+}
+
+static void quat_conj(const double *a, double *out) {
+  out[0] = a[0];
+  out[1] = -a[1];
+  out[2] = -a[2];
+  out[3] = -a[3];
+}
+
+/* z = p * y * conj(q): the SO(4) rotation of one 4-element block. */
+void ref_so4_forward(const double *p, const double *q, const double *y, double *z) {
+  double qc[4], t[4];
+  quat_conj(q, qc);
+  ref_quat_mul(p, y, t);
+  ref_quat_mul(t, qc, z);
+}
+
+/* y = conj(p) * z * q: the inverse (transpose) of ref_so4_forward. */
+void ref_so4_inverse(const double *p, const double *q, const double *z, double *y) {
+  double pc[4], t[4];
+  quat_conj(p, pc);
+  ref_quat_mul(pc, z, t);
+  ref_quat_mul(t, q, y);
+}
+
+/* Forward rotation of one d-vector with one head's params: WHT, then the d/4 blocks. */
+void ref_rotate(const double *params_head, const double *x, double *z, int d) {
+  double *y = (double *)malloc(sizeof(double) * d);
+  memcpy(y, x, sizeof(double) * d);
+  ref_wht(y, d);
+  for (int b = 0; b < d / 4; b++)
+    ref_so4_forward(params_head + b * 8, params_head + b * 8 + 4, y + 4 * b, z + 4 * b);
+  free(y);
+}
+
+/* Inverse rotation: inverse blocks, then the WHT (orthonormal and symmetric, so it is
+ * its own inverse). */
+void ref_unrotate(const double *params_head, const double *z, double *x, int d) {
+  for (int b = 0; b < d / 4; b++)
+    ref_so4_inverse(params_head + b * 8, params_head + b * 8 + 4, z + 4 * b, x + 4 * b);
+  ref_wht(x, d);
+}
+
+/* ------------------------------------------------------------------------------ */
+/* IEEE 754 binary16, round to nearest, ties to even (from the format definition).   */
+/* ------------------------------------------------------------------------------ */
+uint16_t ref_fp16_bits(double v) {
+  uint16_t sign = signbit(v) ? 0x8000 : 0;
+  double a = fabs(v);
+  if (isnan(v)) return 0x7e00;
+  if (a >= 65520.0) return sign | 0x7c00; /* rounds past the largest finite, 65504 */
+  int e;
+  frexp(a, &e); /* a = f * 2^e, f in [0.5, 1): the leading bit has weight 2^(e-1) */
+  if (a == 0.0 || e - 1 < -14) {
+    /* subnormal range: quantum 2^-24; nearbyint rounds ties to even */
+    double m = nearbyint(ldexp(a, 24));
+    return sign | (uint16_t)m; /* m == 1024 is the smallest normal, same bits */
+  }
+  double m = nearbyint(ldexp(a, 10 - (e - 1))); /* in [1024, 2048] */
+  int ex = e - 1;
+  if (m == 2048.0) {
+    m = 1024.0;
+    ex += 1;
+  }
+  if (ex > 15) return sign | 0x7c00;
+  return sign | (uint16_t)((ex + 15) << 10) | (uint16_t)((int)m - 1024);
+}
+
+double ref_fp16_value(uint16_t h) {
+  int ex = (h >> 10) & 31, man = h & 1023;
+  double s = (h & 0x8000) ? -1.0 : 1.0;
+  if (ex == 0) return s * ldexp((double)man, -24);
+  if (ex == 31) return man ? NAN : s * INFINITY;
+  return s * ldexp(1024.0 + man, ex - 25);
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Quantise one vector: norm, WHT, SO(4) blocks, scalar quantisation.               */
+/* ------------------------------------------------------------------------------ */
+/* codes[i] in 0..7 (ascending level index); *norm16 = binary16 bits of the norm.
+ * Returns 1 if the norm overflowed binary16 (stored as 65504), else 0.
+ * z_out (optional) receives the rotated coordinates z. */
+int ref_quantize_vector(const double *params_head, const double *x, int d, uint8_t *codes,
+                        uint16_t *norm16, double *z_out) {
+  double ss = 0.0;
+  for (int i = 0; i < d; i++) ss += x[i] * x[i];
+  double n = sqrt(ss);
+
+  double *z = (double *)malloc(sizeof(double) * d);
+  ref_rotate(params_head, x, z, d);
+
+  /* code_i = #{j : u_i >= t_j} with u_i = sqrt(d) z_i / n, compared as
+   * sqrt(d) z_i >= n t_j.  A zero vector has no direction: u is taken as 0, which the
+   * tie rule sends to code 4 (the level just above 0). */
+  double sqd = sqrt((double)d);
+  for (int i = 0; i < d; i++) {
+    int c = 0;
+    if (n == 0.0) {
+      c = 4;
+    } else {
+      for (int j = 0; j < 7; j++)
+        if (sqd * z[i] >= n * ref_threshold(j)) c++;
+    }
+    codes[i] = (uint8_t)c;
+  }
+  if (z_out) memcpy(z_out, z, sizeof(double) * d);
+  free(z);
+
+  uint16_t h = ref_fp16_bits(n);
+  int overflow = 0;
+  if (h == 0x7c00) {
+    h = 0x7bff;
+    overflow = 1;
+  }
+  *norm16 = h;
+  return overflow;
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Packed code layout (3 bits per code, d/32 groups of 12 bytes per vector).        */
+/* Group g covers dims 32g..32g+31 and is three little-endian 32-bit words w0..w2:  */
+/*   dim 32g + 8j + k  (j = 0,1,2; k = 0..7): the code is bits 4k..4k+2 of w_j;       */
+/*   dim 32g + 24 + k  (k = 0..7): code bit (2 - b) is bit 4k+3 of w_b.              */
+/* ------------------------------------------------------------------------------ */
+void ref_pack_codes(const uint8_t *codes, int d, uint8_t *out) {
+  for (int g = 0; g < d / 32; g++) {
+    uint32_t w[3] = {0, 0, 0};
+    for (int e = 0; e < 32; e++) {
+      uint32_t c = codes[32 * g + e] & 7u;
+      if (e < 24) {
+        int j = e / 8, k = e % 8;
+        w[j] |= c << (4 * k);
+      } else {
+        int k = e - 24;
+        for (int b = 0; b < 3; b++) w[b] |= ((c >> (2 - b)) & 1u) << (4 * k + 3);
+      }
+    }
+    for (int j = 0; j < 3; j++)
+      for (int byte = 0; byte < 4; byte++)
+        out[12 * g + 4 * j + byte] = (uint8_t)(w[j] >> (8 * byte));
+  }
+}
+
+void ref_unpack_codes(const uint8_t *in, int d, uint8_t *codes) {
+  for (int g = 0; g < d / 32; g++) {
+    uint32_t w[3];
+    for (int j = 0; j < 3; j++) {
+      w[j] = 0;
+      for (int byte = 0; byte < 4; byte++)
+        w[j] |= (uint32_t)in[12 * g + 4 * j + byte] << (8 * byte);
+    }
+    for (int e = 0; e < 32; e++) {
+      uint32_t c = 0;
+      if (e < 24) {
+        c = (w[e / 8] >> (4 * (e % 8))) & 7u;
+      } else {
+        int k = e - 24;
+        for (int b = 0; b < 3; b++) c |= ((w[b] >> (4 * k + 3)) & 1u) << (2 - b);
+      }
+      codes[32 * g + e] = (uint8_t)c;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Paged cache: blocks[page][kv_head] of block_bytes; a block holds, for 64 (page)  */
+/* token slots: K codes [P][3d/8] | K norms [P] binary16 | V codes | V norms.        */
+/* ------------------------------------------------------------------------------ */
+size_t ref_block_bytes(int d, int page) { return (size_t)2 * page * (3 * d / 8 + 2); }
+
+static size_t k_codes_off(int d, int page, int slot) { (void)page; return (size_t)slot * (3 * d / 8); }
+static size_t k_norm_off(int d, int page, int slot) {
+  return (size_t)page * (3 * d / 8) + 2 * (size_t)slot;
+}
+static size_t v_codes_off(int d, int page, int slot) {
+  return (size_t)page * (3 * d / 8 + 2) + (size_t)slot * (3 * d / 8);
+}
+static size_t v_norm_off(int d, int page, int slot) {
+  return (size_t)page * (3 * d / 8 + 2) + (size_t)page * (3 * d / 8) + 2 * (size_t)slot;
+}
+
+/* Quantise n_tokens tokens of K and V ([n_tokens][n_kv_heads][d], fp64) into the paged
+ * cache at (seq_ids[t], positions[t]).  params: fp64 [n_kv_heads][d/4][2][4].
+ * Returns the number of norms that saturated. */
+int ref_quantize_append(const double *params, int d, int n_kv_heads, int page,
+                        uint8_t *blocks, const int32_t *page_table, int max_pages_per_seq,
+                        const double *K, const double *V, int n_tokens,
+                        const int32_t *seq_ids, const int32_t *positions) {
+  size_t bb = ref_block_bytes(d, page);
+  int overflow = 0;
+#pragma omp parallel for schedule(static) reduction(+ : overflow)
+  for (int t = 0; t < n_tokens; t++) {
+    uint8_t codes[1024];
+    for (int h = 0; h < n_kv_heads; h++) {
+      int pos = positions[t];
+      int phys = page_table[(size_t)seq_ids[t] * max_pages_per_seq + pos / page];
+      int slot = pos % page;
+      uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + h) * bb;
+      const double *ph = params + (size_t)h * (d / 4) * 8;
+      for (int kv = 0; kv < 2; kv++) {
+        const double *x = (kv == 0 ? K : V) + ((size_t)t * n_kv_heads + h) * d;
+        uint16_t n16;
+        overflow += ref_quantize_vector(ph, x, d, codes, &n16, NULL);
+        uint8_t *dst = blk + (kv == 0 ? k_codes_off(d, page, slot) : v_codes_off(d, page, slot));
+        ref_pack_codes(codes, d, dst);
+        uint8_t *nd = blk + (kv == 0 ? k_norm_off(d, page, slot) : v_norm_off(d, page, slot));
+        nd[0] = (uint8_t)(n16 & 0xff);
+        nd[1] = (uint8_t)(n16 >> 8);
+      }
+    }
+  }
+  return overflow;
+}
+
+/* Dequantised vector in the rotated space: (stored norm / sqrt(d)) * level[code]. */
+static void dequant_rotated(const uint8_t *packed, const uint8_t *norm_bytes, int d, double *out) {
+  uint8_t codes[1024];
+  ref_unpack_codes(packed, d, codes);
+  uint16_t n16 = (uint16_t)(norm_bytes[0] | (norm_bytes[1] << 8));
+  double s = ref_fp16_value(n16) / sqrt((double)d);
+  for (int i = 0; i < d; i++) out[i] = s * REF_LEVELS[codes[i]];
+}
+
+/* Materialise one cached vector back in the input space (K-hat or V-hat): inverse
+ * rotation of the dequantised rotated vector.  kind 0 = K, 1 = V.  Used by tests to
+ * check that attention in the rotated space equals attention over K-hat, V-hat. */
+void ref_dequantize_slot(const double *params, int d, int n_kv_heads, int page,
+                         const uint8_t *blocks, int phys_page, int kv_head, int slot, int kind,
+                         double *out) {
+  size_t bb = ref_block_bytes(d, page);
+  const uint8_t *blk = blocks + ((size_t)phys_page * n_kv_heads + kv_head) * bb;
+  double zr[1024];
+  if (kind == 0)
+    dequant_rotated(blk + k_codes_off(d, page, slot), blk + k_norm_off(d, page, slot), d, zr);
+  else
+    dequant_rotated(blk + v_codes_off(d, page, slot), blk + v_norm_off(d, page, slot), d, zr);
+  ref_unrotate(params + (size_t)kv_head * (d / 4) * 8, zr, out, d);
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Decode attention on the packed cache, all in the rotated space.                  */
+/*   a6: q~ = R q (same WHT + SO(4) as the KV head's keys);                          */
+/*   a7: s_t = scale * q~ . k~_t,  k~_t = (n_t / sqrt d) L[c_t];                      */
+/*   a8: softmax over t = 0..len-1 and o~ = sum_t p_t v~_t;                          */
+/*   a9: out = R^T o~.                                                               */
+/* Q: [n_seqs][n_q_heads][d] fp64; out likewise.  A sequence of length 0 gives 0.    */
+/* The (sequence, head) pairs listed in sel (pairs of ints; n_sel of them; NULL =    */
+/* all) are the ones computed; others in out are left untouched.                     */
+/* ------------------------------------------------------------------------------ */
+void ref_decode_attention(const double *params, int d, int n_kv_heads, int page,
+                          const uint8_t *blocks, const int32_t *page_table,
+                          int max_pages_per_seq, int n_seqs, int n_q_heads,
+                          const int32_t *seq_lens, const double *Q, double scale, double *out,
+                          const int32_t *sel, int n_sel) {
+  int G = n_q_heads / n_kv_heads;
+  size_t bb = ref_block_bytes(d, page);
+  int total = sel ? n_sel : n_seqs * n_q_heads;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int w = 0; w < total; w++) {
+    int s = sel ? sel[2 * w] : w / n_q_heads;
+    int h = sel ? sel[2 * w + 1] : w % n_q_heads;
+    int kvh = h / G;
+    int len = seq_lens[s];
+    const double *ph = params + (size_t)kvh * (d / 4) * 8;
+    double *o = out + ((size_t)s * n_q_heads + h) * d;
+    if (len <= 0) {
+      for (int i = 0; i < d; i++) o[i] = 0.0;
+      continue;
+    }
+    double qt[1024], kt[1024], vt[1024], ot[1024];
+    ref_rotate(ph, Q + ((size_t)s * n_q_heads + h) * d, qt, d);
+
+    double *sc = (double *)malloc(sizeof(double) * len);
+    for (int t = 0; t < len; t++) {
+      int phys = page_table[(size_t)s * max_pages_per_seq + t / page];
+      const uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + kvh) * bb;
+      dequant_rotated(blk + k_codes_off(d, page, t % page), blk + k_norm_off(d, page, t % page),
+                      d, kt);
+      double dot = 0.0;
+      for (int i = 0; i < d; i++) dot += qt[i] * kt[i];
+      sc[t] = scale * dot;
+    }
+    double m = -INFINITY;
+    for (int t = 0; t < len; t++)
+      if (sc[t] > m) m = sc[t];
+    double l = 0.0;
+    for (int i = 0; i < d; i++) ot[i] = 0.0;
+    for (int t = 0; t < len; t++) {
+      double p = exp(sc[t] - m);
+      l += p;
+      int phys = page_table[(size_t)s * max_pages_per_seq + t / page];
+      const uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + kvh) * bb;
+      dequant_rotated(blk + v_codes_off(d, page, t % page), blk + v_norm_off(d, page, t % page),
+                      d, vt);
+      for (int i = 0; i < d; i++) ot[i] += p * vt[i];
+    }
+    for (int i = 0; i < d; i++) ot[i] /= l;
+    free(sc);
+    ref_unrotate(ph, ot, o, d);
+  }
+}
+
+/* Full-precision attention (no quantisation, no rotation) for the error-bound tests:
+ * K, V [n_tokens][n_kv_heads][d], one sequence of n_tokens, Q [n_q_heads][d]. */
+void ref_attention_full(int d, int n_kv_heads, int n_q_heads, int n_tokens, const double *K,
+                        const double *V, const double *Q, double scale, double *out) {
+  int G = n_q_heads / n_kv_heads;
+  for (int h = 0; h < n_q_heads; h++) {
+    int kvh = h / G;
+    const double *q = Q + (size_t)h * d;
+    double *sc = (double *)malloc(sizeof(double) * (n_tokens > 0 ? n_tokens : 1));
+    double m = -INFINITY;
+    for (int t = 0; t < n_tokens; t++) {
+      const double *k = K + ((size_t)t * n_kv_heads + kvh) * d;
+      double dot = 0.0;
+      for (int i = 0; i < d; i++) dot += q[i] * k[i];
+      sc[t] = scale * dot;
+      if (sc[t] > m) m = sc[t];
+    }
+    double *o = out + (size_t)h * d;
+    for (int i = 0; i < d; i++) o[i] = 0.0;
+    double l = 0.0;
+    for (int t = 0; t < n_tokens; t++) {
+      double p = exp(sc[t] - m);
+      l += p;
+      const double *v = V + ((size_t)t * n_kv_heads + kvh) * d;
+      for (int i = 0; i < d; i++) o[i] += p * v[i];
+    }
+    if (n_tokens > 0)
+      for (int i = 0; i < d; i++) o[i] /= l;
+    free(sc);
+  }
+}

@@ -1,0 +1,420 @@
+"""Benchmark of the IsoQuant packed-KV path on B200: quantize-append + decode attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 5] [--impl ours|reference]
+
+One step = the whole hot path over one batch of the workload: quantize-append of the full
+prefill (in the workload's chunked calls) followed by one decode step of every sequence
+on the packed cache.  Default workload: 8 sequences x 131072 tokens, 64 query / 8 KV
+heads, d = 128, bf16 K/V quantised in 16384-token chunks (the long-context configuration,
+on which both halves of the metric -- quantize Mvec/s and packed-KV decode GB/s -- are
+quoted).  Inputs are resident in HBM before the timed region and larger than L2; L2 is
+also flushed before each decode.  Timing: CUDA events on the launching stream, barrier +
+synchronize around the K timed steps, max over ranks.  Multi-GPU: every rank runs its own
+replica (the (sequence, KV head) units are independent), no collective on the data path.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on a bounded
+sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def _dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        if j.get("hbm_gbs"):
+            return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def _kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "rotated_bit_kv_isoquant_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/, if the kernel sources
+    have not changed since (else None)."""
+    sha = _kernel_sources_sha()
+    for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        txt = open(p).read()
+        m_k = re.search(r"^kernel_group:\s*(\S+)", txt, re.M)
+        m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
+        m_s = re.search(r"^source_sha:\s*(\S+)", txt, re.M)
+        m_t = re.search(r"^dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt, re.M)
+        if m_k and m_w and m_s and m_t and m_k.group(1) == kernel and m_w.group(1) == workload:
+            if m_s.group(1) == sha:
+                return float(m_t.group(1))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is None:
+            self.out = ""
+            return
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.strip()]
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = sorted(sm)[len(sm) // 4:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------
+# Oracle timing (CPU baseline and the reference arm)
+# ------------------------------------------------------------------------------------
+def oracle_sample(cfg, tokens: int = 4096, units: int = 1):
+    """Bounded sample of the workload for the fp64 oracle: the first `tokens` tokens of
+    sequence 0 for `units` KV heads (all their query heads), quantised by the oracle into
+    its own paged cache, then decoded.  Returns timings and the bytes/vectors processed."""
+    import numpy as np
+    import torch
+    import oracle
+    import workloads as wl
+
+    oracle.build()
+    K, V = wl.kv_tokens(cfg, 0, 0, tokens, device="cpu")
+    H = units
+    K = K[:, :H].float().numpy().astype(np.float64)
+    V = V[:, :H].float().numpy().astype(np.float64)
+    Q = wl.queries(cfg, device="cpu")[:1, :H * cfg.group].float().numpy().astype(np.float64)
+    _, p32 = oracle.make_params(wl.PARAM_SEED, cfg.d, H)
+    p64 = p32.astype(np.float64)
+    npg = -(-tokens // 64)
+    pt = np.arange(npg, dtype=np.int32)[None, :]
+    blocks = np.zeros(npg * H * oracle.block_bytes(cfg.d), np.uint8)
+    t0 = time.perf_counter()
+    oracle.quantize_append(p64, cfg.d, H, 64, blocks, pt, K, V, np.zeros(tokens, np.int32),
+                           np.arange(tokens, dtype=np.int32))
+    t1 = time.perf_counter()
+    oracle.decode_attention(p64, cfg.d, H, 64, blocks, pt, [tokens], Q, cfg.scale)
+    t2 = time.perf_counter()
+    packed = tokens * H * 2 * (3 * cfg.d // 8 + 2)
+    return {"quant_s": t1 - t0, "decode_s": t2 - t1, "vectors": tokens * H * 2,
+            "packed_bytes": packed, "threads": oracle.num_threads(),
+            "pairs": H * cfg.group, "tokens": tokens, "units": H}
+
+
+def cpu_baseline(cfg, budget_s: float = 12.0):
+    """Oracle decode GB/s (and quantize Mvec/s) on a bounded sample sized to ~budget_s."""
+    probe = oracle_sample(cfg, tokens=1024, units=1)
+    per_tok = (probe["quant_s"] + probe["decode_s"]) / 1024
+    tokens = int(max(1024, min(cfg.decode_lens()[0], budget_s / max(per_tok, 1e-9))))
+    tokens = (tokens // 64) * 64
+    r = oracle_sample(cfg, tokens=tokens, units=1)
+    return {
+        "value": r["packed_bytes"] / r["decode_s"] / 1e9, "unit": "GB/s",
+        "cores": min(r["threads"], r["pairs"]), "kind": "oracle",
+        "quantize_mvec_s": r["vectors"] / r["quant_s"] / 1e6,
+        "quantize_cores": r["threads"],
+        "sample": (f"sequence 0, first {r['tokens']} tokens, 1 KV head x {r['pairs']} query "
+                   f"heads: oracle quantize ({r['vectors']} vectors) then decode "
+                   f"({r['packed_bytes']} packed bytes)"),
+    }
+
+
+def run_reference(args, cfg):
+    rank, world, _ = _dist_env()
+    if rank != 0:
+        return 0
+    tokens = 2048
+    for _ in range(args.warmup):
+        oracle_sample(cfg, tokens=tokens)
+    dec, qt, rr = 0.0, 0.0, None
+    for _ in range(args.steps):
+        rr = oracle_sample(cfg, tokens=tokens)
+        dec += rr["decode_s"]
+        qt += rr["quant_s"]
+    value = rr["packed_bytes"] * args.steps / dec / 1e9
+    sample = (f"per step: sequence 0, first {tokens} tokens, 1 KV head x {rr['pairs']} query "
+              f"heads; oracle quantize then decode")
+    line = {
+        "impl": "reference", "metric": "packed-KV decode attention GB/s", "value": value,
+        "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": (dec + qt) / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(cfg),
+        "quantize": {"value": rr["vectors"] * args.steps / qt / 1e6, "unit": "Mvec/s"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle",
+                         "cores": min(rr["threads"], rr["pairs"]), "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(cfg):
+    return {"workload": cfg.name, "description": cfg.description, "n_seqs": cfg.n_seqs,
+            "context": cfg.decode_lens()[0] if cfg.fixed_len else "varied",
+            "n_q_heads": cfg.n_q_heads, "n_kv_heads": cfg.n_kv_heads, "head_dim": cfg.d,
+            "kv_dtype": str(cfg.in_dtype).replace("torch.", ""),
+            "quantize_chunk_tokens": cfg.quant_chunk or None,
+            "l2": "inputs larger than L2; L2 flushed before each decode"}
+
+
+# ------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import rotated_bit_kv_isoquant_b200 as iq
+    import workloads as wl
+
+    rank, world, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream(dev)
+    params = iq.isoq_make_params(wl.PARAM_SEED, cfg.d, cfg.n_kv_heads)
+    layout = wl.page_layout(cfg)
+    cache = iq.PagedCache(cfg.d, cfg.n_kv_heads, layout.n_pages, layout.page_table, device=dev)
+    calls = wl.prefill_calls(cfg)
+    inputs = []
+    for s, start, count in calls:
+        K, V = wl.kv_tokens(cfg, s, start, count, device=dev)
+        sid = torch.full((count,), s, dtype=torch.int32, device=dev)
+        pos = torch.arange(start, start + count, dtype=torch.int32, device=dev)
+        inputs.append((K, V, sid, pos))
+    app = wl.append_kv(cfg, device=dev)
+    Q = wl.queries(cfg, device=dev)
+    lens = cfg.decode_lens()
+    max_len = max(lens)
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    out = torch.empty((cfg.n_seqs, cfg.n_q_heads, cfg.d), dtype=torch.float32, device=dev)
+    wsb = iq.isoq_decode_workspace_bytes(cfg.n_seqs, cfg.n_q_heads, cfg.n_kv_heads, cfg.d, max_len)
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty((2 * l2 // 4,), dtype=torch.int32, device=dev)
+
+    n_vec = 2 * cfg.n_kv_heads * sum(c for _, _, c in calls)
+    n_vec += 2 * cfg.n_kv_heads * app[0].shape[0]
+    packed = sum(lens) * cfg.n_kv_heads * 2 * (3 * cfg.d // 8 + 2)
+    launches_per_step = len(calls) + (1 if app[0].shape[0] else 0) + 2
+
+    def quantize_all():
+        for K, V, sid, pos in inputs:
+            iq.isoq_quantize_append(params, cache, K, V, sid, pos, stream=stream)
+        if app[0].shape[0]:
+            iq.isoq_quantize_append(params, cache, app[0], app[1], app[2], app[3], stream=stream)
+
+    def decode():
+        iq.isoq_decode_attention(params, cache, Q, sl, max_len, out, cfg.scale, ws, stream=stream)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(e_q0, e_q1, e_d0, e_d1):
+        e_q0.record(stream)
+        quantize_all()
+        e_q1.record(stream)
+        flush.zero_()
+        e_d0.record(stream)
+        decode()
+        e_d1.record(stream)
+
+    for _ in range(args.warmup):
+        step(ev(), ev(), ev(), ev())
+    torch.cuda.synchronize()
+    assert iq.isoq_get_status(cache) == 0, "device status bits set during warm-up"
+
+    evs = [(ev(), ev(), ev(), ev()) for _ in range(args.steps)]
+    t_start, t_end = ev(), ev()
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for e in evs:
+            step(*e)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    q_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b, _, _ in evs))
+    d_ms = max_over_ranks(sum(c.elapsed_time(d) for _, _, c, d in evs))
+    dec_launch_ms = d_ms / args.steps
+
+    value = packed * args.steps * world / (d_ms / 1e3) / 1e9
+    qval = n_vec * args.steps * world / (q_ms / 1e3) / 1e6
+    peak, peak_kind = _peaks()
+    dec_gbs_1 = packed / (dec_launch_ms / 1e3) / 1e9
+    q_bytes = n_vec * (cfg.d * (4 if cfg.in_dtype == torch.float32 else 2) + 3 * cfg.d // 8 + 2)
+    q_gbs_1 = q_bytes / (q_ms / args.steps / 1e3) / 1e9
+    tr_dec = _ncu_traffic("decode", cfg.name)
+    tr_q = _ncu_traffic("quantize", cfg.name)
+
+    # ---- e2e: host inputs (pinned), H2D inside the timed region, D2H of the output ----
+    e2e = None
+    if not args.no_e2e:
+        host = [(K.cpu().pin_memory(), V.cpu().pin_memory()) for K, V, _, _ in inputs]
+        hq = Q.cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(k.numel() * k.element_size() * 2 for k, _ in host) + hq.numel() * hq.element_size()
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for (hk, hv), (K, V, sid, pos) in zip(host, inputs):
+                K.copy_(hk, non_blocking=True)
+                V.copy_(hv, non_blocking=True)
+                iq.isoq_quantize_append(params, cache, K, V, sid, pos, stream=stream)
+            if app[0].shape[0]:
+                iq.isoq_quantize_append(params, cache, app[0], app[1], app[2], app[3],
+                                        stream=stream)
+            Q.copy_(hq, non_blocking=True)
+            decode()
+            hout.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        barrier()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(a.elapsed_time(b))
+        e2e = {"value": packed * args.e2e_steps * world / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
+               "what": "packed-KV bytes decoded per step / step time with the step's K, V and "
+                       "Q copied from pinned host memory, quantize-append, decode and the "
+                       "output copied back"}
+
+    line = {
+        "metric": "packed-KV decode attention GB/s (% of B200 HBM peak); quantize Mvec/s",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": _config(cfg),
+        "quantize": {"value": qval, "unit": "Mvec/s", "ms_per_step": q_ms / args.steps,
+                     "roofline": {"bound": "hbm", "achieved": q_gbs_1, "peak": peak,
+                                  "unit": "GB/s", "frac": q_gbs_1 / peak, "traffic": tr_q,
+                                  "peak_kind": peak_kind}},
+        "decode_ms": dec_launch_ms,
+        "roofline": {"bound": "hbm", "achieved": dec_gbs_1, "peak": peak, "unit": "GB/s",
+                     "frac": dec_gbs_1 / peak, "traffic": tr_dec, "peak_kind": peak_kind,
+                     "kernel": "decode (split-K kernel + combine kernel, one call)",
+                     "algorithmic_bytes_per_launch": packed},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = _args()
+    import workloads as wl
+    cfg = wl.workload(args.config)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,214 @@
+/*
+ * isoq.h -- C ABI of libisoq: IsoQuant 3-bit KV-cache compression and decode attention
+ * computed directly on the packed cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method is the IsoQuant axis of "RotaryQuant: Fitting 120B MoE Models on Consumer
+ * Hardware via Fused Compressed-Space Attention" (arXiv 2608.08081v1), Abstract: every
+ * per-token, per-head K or V vector is passed through a Walsh-Hadamard transform, then
+ * block-diagonal SO(4) rotations (quaternion rotations: "FreeToken issue #141, unified KV
+ * cache backend", Proposed Solution, Quantization layer), then 3-bit scalar
+ * quantisation; attention runs on the packed 3-bit tensors without materialising
+ * full-precision K/V.  The pages fix none of the numeric details below; this library's
+ * choices are stated with each declaration.
+ *
+ * Conventions for every call:
+ *   - Return value: ISOQ_OK (0) or a negative ISOQ_E_* code.  No exception, abort or
+ *     device trap crosses this boundary.
+ *   - Pointers documented as "device" must point to memory of the CUDA device that is
+ *     current when the call is made; the caller owns all of them (the library keeps no
+ *     reference after the call returns, except inside an isoq_params handle).
+ *   - GPU work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = the legacy
+ *     default stream) and the call returns without waiting for it.  Only
+ *     isoq_make_params, isoq_params_copy and isoq_get_status synchronise.
+ *   - Errors the device detects (an out-of-range sequence id, position or page id; a norm
+ *     that overflows binary16) never fault: the offending write is skipped (or the value
+ *     saturated) and a bit is OR-ed into the caller's status word, read with
+ *     isoq_get_status.
+ *   - The library allocates device memory only inside isoq_make_params.
+ */
+#ifndef ISOQ_H
+#define ISOQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------------ */
+#define ISOQ_OK 0
+#define ISOQ_E_ARG (-1)       /* null pointer, negative count, unknown dtype, bad scale */
+#define ISOQ_E_DIM (-2)       /* head dimension or page size not supported */
+#define ISOQ_E_GQA (-3)       /* n_q_heads not a multiple of n_kv_heads, or group > 16 */
+#define ISOQ_E_WORKSPACE (-4) /* workspace smaller than isoq_decode_workspace_bytes() */
+#define ISOQ_E_CUDA (-5)      /* a CUDA runtime call failed; see isoq_last_cuda_error() */
+#define ISOQ_E_DEVICE (-6)    /* no CUDA device, or params made on another device */
+
+/* ---- device status bits (sticky; OR-ed into isoq_cache.status) ------------------------ */
+#define ISOQ_ST_SEQ_RANGE 0x1u  /* quantize: seq_id outside [0, n_seqs); token skipped */
+#define ISOQ_ST_POS_RANGE 0x2u  /* quantize: position < 0 or beyond the page table; skipped */
+#define ISOQ_ST_PAGE_RANGE 0x4u /* a page-table entry outside [0, n_pages); page skipped */
+#define ISOQ_ST_NORM_SAT 0x8u   /* a norm >= 65520 was stored as 65504 (binary16 max) */
+#define ISOQ_ST_LEN_RANGE 0x10u /* decode: seq_len beyond the page table; clamped */
+
+/* ---- element types of K, V and Q ---------------------------------------------------- */
+#define ISOQ_F32 0
+#define ISOQ_BF16 1
+#define ISOQ_F16 2
+
+/* ---- supported sizes ------------------------------------------------------------------ */
+#define ISOQ_PAGE_SIZE 64 /* tokens per cache page (the only page size supported) */
+/* Head dimensions d: 128 and 256.  The packed format needs d % 32 == 0. */
+
+/* =======================================================================================
+ * Rotation parameters.
+ *
+ * Per KV head, one unit-quaternion pair (p_b, q_b) per 4-element block b = 0..d/4-1,
+ * rotating the block y_b (read as the quaternion w + x i + y j + z k, Hamilton
+ * convention) to z_b = p_b * y_b * conj(q_b).  That is d/4 * 8 = 256 stored parameters
+ * per head at d = 128 (the paper's count, versus d^2 = 16,384 for a dense rotation).
+ * K and V of one KV head share the same parameters.
+ *
+ * Values are drawn from SplitMix64 (Steele, Lea & Flood, OOPSLA 2014) seeded with `seed`:
+ * for head h, block b, then p before q, four standard normals, each from two successive
+ * 64-bit draws k1, k2 as sqrt(-2 ln u1) cos(2 pi u2) with u1 = ((k1>>11)+1) 2^-53 and
+ * u2 = (k2>>11) 2^-53 (Box-Muller), computed in binary64; the 4-vector is divided by its
+ * Euclidean length (uniform on the 3-sphere, so the block rotation is Haar on SO(4)) and
+ * rounded to binary32.  Layout of the float array: [n_kv_heads][d/4][2][4], component
+ * order (w, x, y, z).
+ * ===================================================================================== */
+typedef struct isoq_params isoq_params; /* opaque: d, n_kv_heads, device copy, host copy */
+
+/* Host only, needs no GPU: writes the n_kv_heads * d * 2 floats described above into
+ * host_out.  Errors: ISOQ_E_ARG (null, n_kv_heads < 1), ISOQ_E_DIM (d not 128 or 256). */
+int isoq_params_generate(uint64_t seed, int d, int n_kv_heads, float* host_out);
+
+/* Generates the parameters and uploads them to the current device (cudaMalloc +
+ * synchronous copy).  *out receives a handle to free with isoq_params_destroy.
+ * Errors: as isoq_params_generate, plus ISOQ_E_DEVICE / ISOQ_E_CUDA. */
+int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out);
+
+/* Copies the binary32 parameters ([n_kv_heads][d/4][2][4]) to host_dst. */
+int isoq_params_copy(const isoq_params* params, float* host_dst);
+
+/* d and n_kv_heads of a handle (either pointer may be NULL). */
+int isoq_params_shape(const isoq_params* params, int* d, int* n_kv_heads);
+
+/* Frees the device copy and the handle.  NULL is ignored. */
+void isoq_params_destroy(isoq_params* params);
+
+/* =======================================================================================
+ * Paged cache.
+ *
+ * blocks: device uint8 [n_pages][n_kv_heads][isoq_block_bytes(d, 64)].  One block holds
+ * one KV head of one 64-token page:
+ *     K codes [64][3d/8] | K norms [64] binary16 | V codes [64][3d/8] | V norms [64] binary16
+ * (6400 bytes at d = 128, 12544 at d = 256; both multiples of 16).
+ *
+ * Codes of one vector (3 bits each, 3d/8 bytes): d/32 groups of 12 bytes; group g covers
+ * dims 32g..32g+31 and is three little-endian 32-bit words w0, w1, w2:
+ *     dim 32g + 8j + k (j = 0,1,2; k = 0..7): the code is bits 4k..4k+2 of w_j;
+ *     dim 32g + 24 + k (k = 0..7): bit (2 - b) of the code is bit 4k+3 of w_b.
+ * A code c in 0..7 indexes the ascending levels
+ *     L = {-2.1520, -1.3440, -0.7560, -0.2451, 0.2451, 0.7560, 1.3440, 2.1520}
+ * (the 8-level Lloyd-Max quantiser for N(0,1), J. Max 1960), and stands for the rotated
+ * coordinate (norm / sqrt(d)) * L[c].  The norm is the input vector's L2 norm rounded to
+ * binary16 (round to nearest even; >= 65520 saturates to 65504 with ISOQ_ST_NORM_SAT).
+ *
+ * page_table: device int32 [n_seqs][max_pages_per_seq]: token position t of sequence s
+ * lives in physical page page_table[s][t / 64], slot t % 64.  Pages may be in any order.
+ * status: device uint32, one word; the caller zeroes it (isoq_reset_status) and the
+ * kernels OR ISOQ_ST_* bits into it.  May be NULL (bits are then dropped).
+ * ===================================================================================== */
+typedef struct isoq_cache {
+  int d;                     /* head dimension: 128 or 256 */
+  int n_kv_heads;            /* KV heads held per page */
+  int page_size;             /* must be ISOQ_PAGE_SIZE */
+  int n_pages;               /* physical pages in `blocks` */
+  int max_pages_per_seq;     /* row length of page_table */
+  int n_seqs;                /* rows of page_table */
+  uint8_t* blocks;           /* device */
+  const int32_t* page_table; /* device */
+  uint32_t* status;          /* device, optional */
+} isoq_cache;
+
+/* Bytes of one (page, KV head) block: 2 * page_size * (3d/8 + 2); 0 if unsupported. */
+size_t isoq_block_bytes(int d, int page_size);
+
+/* =======================================================================================
+ * Quantize-append.
+ *
+ * For every token t < n_tokens and KV head h: x = K[t][h] (then V[t][h]), n = ||x||_2,
+ * y = H x / sqrt(d) (orthonormal Walsh-Hadamard, natural order), z_b = p_b * y_b *
+ * conj(q_b) with the KV head's parameters, u_i = sqrt(d) z_i / n, and
+ * code_i = #{j : u_i >= t_j} over the 7 midpoint thresholds t_j = (L[j] + L[j+1]) / 2
+ * (a zero vector gets code 4 everywhere).  The codes and the
+ * binary16 norm are written to slot positions[t] % 64 of page
+ * page_table[seq_ids[t]][positions[t] / 64].
+ *
+ * K, V: device [n_tokens][n_kv_heads][d] contiguous, element type `dtype` (ISOQ_F32,
+ * ISOQ_BF16 or ISOQ_F16).  seq_ids, positions: device int32 [n_tokens].
+ * n_tokens == 0 is a no-op.  Arithmetic is binary32; the code decision compares
+ * sqrt(d) z_i against n t_j with no division.
+ * Errors: ISOQ_E_ARG (null pointers, n_tokens < 0, unknown dtype), ISOQ_E_DIM (cache d or
+ * page size unsupported, or d / n_kv_heads differ from the params), ISOQ_E_CUDA (launch).
+ * ===================================================================================== */
+int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, const void* K,
+                         const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
+                         const int32_t* positions, void* stream);
+
+/* =======================================================================================
+ * Decode attention on the packed cache (one query token per sequence).
+ *
+ * For sequence s and query head h (KV head g = h / (n_q_heads / n_kv_heads)):
+ *   q~ = R_g q            (the same WHT + SO(4) rotation as the cached vectors)
+ *   s_t = scale * q~ . k~_t,   k~_t = (n_t / sqrt d) L[c_t]   for t = 0..seq_lens[s]-1
+ *   o~  = sum_t softmax(s)_t v~_t                               (in the rotated space)
+ *   out[s][h] = R_g^T o~                                        (inverse blocks, then WHT)
+ * Full-precision K/V are never formed.  The context is split into chunks processed in
+ * parallel (flash-decoding style, cf. "FreeToken releases", v0.2.0, Kernels: split
+ * decode attention by context length and SM count); per-chunk partial results (running
+ * max, sum, rotated accumulator) live in `workspace` and are merged, empty chunks
+ * contributing nothing (the -inf start of an empty chunk is never exponentiated: cf. the
+ * same release's note on a NaN from a softmax chunk that starts at -inf).
+ *
+ * Q: device [n_seqs][n_q_heads][d], element type q_dtype.  seq_lens: device int32
+ * [n_seqs], the number of cached tokens each query attends (0 gives an all-zero output;
+ * beyond the page table it is clamped and ISOQ_ST_LEN_RANGE set).  max_seq_len: a host
+ * upper bound of seq_lens used only to size the split; must equal the value passed to
+ * isoq_decode_workspace_bytes.  out: device fp32 [n_seqs][n_q_heads][d].
+ * workspace: device, at least isoq_decode_workspace_bytes(...) bytes, 16-byte aligned,
+ * contents need not be initialised.  Calls that share a workspace must not overlap.
+ * Errors: ISOQ_E_ARG, ISOQ_E_DIM, ISOQ_E_GQA, ISOQ_E_WORKSPACE, ISOQ_E_CUDA.
+ * ===================================================================================== */
+size_t isoq_decode_workspace_bytes(int n_seqs, int n_q_heads, int n_kv_heads, int d,
+                                   int max_seq_len);
+
+int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                          int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                          int max_seq_len, float* out, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Number of context chunks (splits) the decode uses for these sizes on the current
+ * device; >= 1, or a negative error code. */
+int isoq_decode_num_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len);
+
+/* ---- status and errors ------------------------------------------------------------------ */
+/* Synchronises the device and copies the status word to *host_bits (0 if status is NULL). */
+int isoq_get_status(const isoq_cache* cache, uint32_t* host_bits);
+
+/* Enqueues a zeroing of the status word on `stream`. */
+int isoq_reset_status(const isoq_cache* cache, void* stream);
+
+/* The cudaError_t of the last failing CUDA call in this thread (0 if none). */
+int isoq_last_cuda_error(void);
+
+/* A static string describing an ISOQ_* return code. */
+const char* isoq_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISOQ_H */

@@ -94,6 +94,10 @@ def _declare(L):
     L.ref_decode_attention.restype = None
     L.ref_decode_attention.argtypes = [_p, _i, _i, _i, _p, _p, _i, _i, _i, _p, _p, _d, _p,
                                        _p, _i]
+    L.ref_quantize_rows.restype = None
+    L.ref_quantize_rows.argtypes = [_p, _i, _i, _p, _i, _p, _p, _p]
+    L.ref_unpack_codes_batch.restype = None
+    L.ref_unpack_codes_batch.argtypes = [_p, _i, ctypes.c_long, _p]
     L.ref_attention_full.restype = None
     L.ref_attention_full.argtypes = [_i, _i, _i, _i, _p, _p, _p, _d, _p]
 
@@ -290,3 +294,27 @@ def attention_full(K, V, Q, scale) -> np.ndarray:
     lib().ref_attention_full(d, n_kv, Q.shape[0], n_tok, _ptr(K), _ptr(V), _ptr(Q),
                              float(scale), _ptr(out))
     return out
+
+
+def quantize_rows(params64, X, with_dist: bool = True):
+    """Quantise X [n_rows][n_kv_heads][d] (head h with params64[h]).
+    -> (codes uint8 [n][H][d], norms uint16 [n][H], dist fp64 [n][H][d] or None), where
+    dist is the distance of u to the nearest threshold."""
+    X = _f64(X)
+    n, H, d = X.shape
+    codes = np.zeros((n, H, d), np.uint8)
+    norms = np.zeros((n, H), np.uint16)
+    dist = np.zeros((n, H, d)) if with_dist else None
+    lib().ref_quantize_rows(_ptr(_f64(params64)), d, H, _ptr(X), n, _ptr(codes), _ptr(norms),
+                            _ptr(dist) if with_dist else None)
+    return codes, norms, dist
+
+
+def unpack_codes_batch(packed, d: int) -> np.ndarray:
+    """packed uint8 [..., 3d/8] -> codes uint8 [..., d]."""
+    packed = np.ascontiguousarray(np.asarray(packed, dtype=np.uint8))
+    lead = packed.shape[:-1]
+    n = int(np.prod(lead)) if lead else 1
+    codes = np.zeros(lead + (d,), np.uint8)
+    lib().ref_unpack_codes_batch(_ptr(packed), d, n, _ptr(codes))
+    return codes

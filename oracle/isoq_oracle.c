@@ -470,3 +470,44 @@ void ref_attention_full(int d, int n_kv_heads, int n_q_heads, int n_tokens, cons
     free(sc);
   }
 }
+
+/* ------------------------------------------------------------------------------ */
+/* Batch helpers for parity checks.                                                 */
+/* ------------------------------------------------------------------------------ */
+/* Quantise n_rows rows of X ([n_rows][n_kv_heads][d]; row r, head h uses head h's
+ * params) and report, per element, the distance of u = sqrt(d) z / n to the nearest
+ * threshold (N(0,1) units; +inf for a zero vector).  codes [n_rows][H][d],
+ * norms [n_rows][H] (binary16 bits), dist [n_rows][H][d] (may be NULL). */
+void ref_quantize_rows(const double *params, int d, int n_kv_heads, const double *X, int n_rows,
+                       uint8_t *codes, uint16_t *norms, double *dist) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < n_rows; r++) {
+    double z[1024];
+    for (int h = 0; h < n_kv_heads; h++) {
+      size_t v = (size_t)r * n_kv_heads + h;
+      const double *x = X + v * d;
+      ref_quantize_vector(params + (size_t)h * (d / 4) * 8, x, d, codes + v * d, norms + v, z);
+      if (!dist) continue;
+      double ss = 0.0;
+      for (int i = 0; i < d; i++) ss += x[i] * x[i];
+      double n = sqrt(ss);
+      for (int i = 0; i < d; i++) {
+        double best = INFINITY;
+        if (n > 0.0) {
+          double u = sqrt((double)d) * z[i] / n;
+          for (int j = 0; j < 7; j++) {
+            double e = fabs(u - ref_threshold(j));
+            if (e < best) best = e;
+          }
+        }
+        dist[v * d + i] = best;
+      }
+    }
+  }
+}
+
+/* Unpack n records of packed codes (3d/8 bytes each, contiguous) into codes [n][d]. */
+void ref_unpack_codes_batch(const uint8_t *in, int d, long n, uint8_t *codes) {
+#pragma omp parallel for schedule(static)
+  for (long i = 0; i < n; i++) ref_unpack_codes(in + i * (3 * d / 8), d, codes + i * d);
+}

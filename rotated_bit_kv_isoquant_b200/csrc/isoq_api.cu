@@ -1,0 +1,313 @@
+// C-ABI layer of libisoq: argument validation, rotation parameters, launch configuration.
+// See include/isoq.h for the contract of every entry point.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/isoq.h"
+#include "isoq_internal.h"
+
+struct isoq_params {
+  int d;
+  int n_kv_heads;
+  int device;
+  float* dev;               // [n_kv_heads][d/4][2][4]
+  std::vector<float> host;  // same values
+};
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return ISOQ_E_CUDA;
+}
+
+bool supported_d(int d) { return d == 128 || d == 256; }
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014).
+uint64_t splitmix64(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ULL;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
+
+// Box-Muller (cosine branch) from two 53-bit uniforms, binary64.
+double std_normal(uint64_t& state) {
+  const double two_m53 = 1.0 / 9007199254740992.0;
+  const uint64_t k1 = splitmix64(state) >> 11;
+  const uint64_t k2 = splitmix64(state) >> 11;
+  const double u1 = ((double)k1 + 1.0) * two_m53;
+  const double u2 = (double)k2 * two_m53;
+  const double two_pi = 2.0 * 3.14159265358979323846;
+  return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
+}
+
+// SM count of the current device (148 on B200 when no device can be queried, which keeps
+// the split arithmetic callable on a host without a GPU).
+int sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+struct SplitPlan {
+  int n_splits;
+  int pages_per_split;
+};
+
+// Context chunking: enough (split, KV head, sequence) CTAs to fill every SM several times
+// over, each chunk a whole number of pages.
+SplitPlan plan_splits(int n_seqs, int n_kv_heads, int max_seq_len) {
+  const int n_sm = sm_count();
+  const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
+  const long long units = (long long)n_seqs * n_kv_heads;
+  const long long target = (long long)n_sm * 16;
+  long long want = units > 0 ? (target + units - 1) / units : 1;
+  if (want < 1) want = 1;
+  if (want > max_pages) want = max_pages;
+  int pps = (int)((max_pages + want - 1) / want);
+  if (pps < 1) pps = 1;
+  int n_splits = (max_pages + pps - 1) / pps;
+  return SplitPlan{n_splits, pps};
+}
+
+int check_cache(const isoq_cache* c, const isoq_params* p) {
+  if (!c || !p) return ISOQ_E_ARG;
+  if (!c->blocks || !c->page_table) return ISOQ_E_ARG;
+  if (c->page_size != ISOQ_PAGE_SIZE || !supported_d(c->d)) return ISOQ_E_DIM;
+  if (c->d != p->d || c->n_kv_heads != p->n_kv_heads) return ISOQ_E_DIM;
+  if (c->n_pages < 0 || c->max_pages_per_seq < 1 || c->n_seqs < 1 || c->n_kv_heads < 1)
+    return ISOQ_E_ARG;
+  return ISOQ_OK;
+}
+
+int check_device(const isoq_params* p) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    g_last_cuda_error = (int)e;
+    cudaGetLastError();
+    return ISOQ_E_DEVICE;
+  }
+  return dev == p->device ? ISOQ_OK : ISOQ_E_DEVICE;
+}
+
+bool valid_dtype(int t) { return t == ISOQ_F32 || t == ISOQ_BF16 || t == ISOQ_F16; }
+
+}  // namespace
+
+extern "C" {
+
+int isoq_params_generate(uint64_t seed, int d, int n_kv_heads, float* host_out) {
+  if (!host_out || n_kv_heads < 1) return ISOQ_E_ARG;
+  if (!supported_d(d)) return ISOQ_E_DIM;
+  uint64_t state = seed;
+  const int nblk = d / 4;
+  for (int h = 0; h < n_kv_heads; ++h)
+    for (int b = 0; b < nblk; ++b)
+      for (int which = 0; which < 2; ++which) {
+        double g[4], s = 0.0;
+        for (int c = 0; c < 4; ++c) {
+          g[c] = std_normal(state);
+          s += g[c] * g[c];
+        }
+        const double len = sqrt(s);
+        for (int c = 0; c < 4; ++c)
+          host_out[(((size_t)h * nblk + b) * 2 + which) * 4 + c] = (float)(g[c] / len);
+      }
+  return ISOQ_OK;
+}
+
+int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
+  if (!out) return ISOQ_E_ARG;
+  *out = nullptr;
+  if (n_kv_heads < 1) return ISOQ_E_ARG;
+  if (!supported_d(d)) return ISOQ_E_DIM;
+  isoq_params* p = new isoq_params();
+  p->d = d;
+  p->n_kv_heads = n_kv_heads;
+  p->dev = nullptr;
+  p->host.resize((size_t)n_kv_heads * d * 2);
+  isoq_params_generate(seed, d, n_kv_heads, p->host.data());
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e != cudaSuccess) {
+    g_last_cuda_error = (int)e;
+    cudaGetLastError();
+    delete p;
+    return ISOQ_E_DEVICE;
+  }
+  const size_t bytes = p->host.size() * sizeof(float);
+  e = cudaMalloc(&p->dev, bytes);
+  if (e == cudaSuccess) e = cudaMemcpy(p->dev, p->host.data(), bytes, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    if (p->dev) cudaFree(p->dev);
+    delete p;
+    return cuda_fail(e);
+  }
+  *out = p;
+  return ISOQ_OK;
+}
+
+int isoq_params_copy(const isoq_params* p, float* host_dst) {
+  if (!p || !host_dst) return ISOQ_E_ARG;
+  memcpy(host_dst, p->host.data(), p->host.size() * sizeof(float));
+  return ISOQ_OK;
+}
+
+int isoq_params_shape(const isoq_params* p, int* d, int* n_kv_heads) {
+  if (!p) return ISOQ_E_ARG;
+  if (d) *d = p->d;
+  if (n_kv_heads) *n_kv_heads = p->n_kv_heads;
+  return ISOQ_OK;
+}
+
+void isoq_params_destroy(isoq_params* p) {
+  if (!p) return;
+  if (p->dev) cudaFree(p->dev);
+  delete p;
+}
+
+size_t isoq_block_bytes(int d, int page_size) {
+  if (!supported_d(d) || page_size != ISOQ_PAGE_SIZE) return 0;
+  return (size_t)2 * page_size * (3 * d / 8 + 2);
+}
+
+int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, const void* K,
+                         const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
+                         const int32_t* positions, void* stream) {
+  int rc = check_cache(cache, params);
+  if (rc) return rc;
+  if (n_tokens < 0 || !valid_dtype(dtype)) return ISOQ_E_ARG;
+  if (n_tokens == 0) return ISOQ_OK;
+  if (!K || !V || !seq_ids || !positions) return ISOQ_E_ARG;
+  if ((rc = check_device(params))) return rc;
+  isoq::QuantizeArgs a;
+  a.params = params->dev;
+  a.blocks = cache->blocks;
+  a.page_table = cache->page_table;
+  a.n_pages = cache->n_pages;
+  a.max_pages = cache->max_pages_per_seq;
+  a.n_seqs = cache->n_seqs;
+  a.n_kv_heads = cache->n_kv_heads;
+  a.d = cache->d;
+  a.K = K;
+  a.V = V;
+  a.dtype = dtype;
+  a.n_tokens = n_tokens;
+  a.seq_ids = seq_ids;
+  a.positions = positions;
+  a.status = cache->status;
+  cudaError_t e = isoq::launch_quantize_append(a, (cudaStream_t)stream, sm_count());
+  return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
+}
+
+int isoq_decode_num_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len) {
+  if (n_seqs < 0 || n_q_heads < 0 || n_kv_heads < 1 || max_seq_len < 0) return ISOQ_E_ARG;
+  if (!supported_d(d)) return ISOQ_E_DIM;
+  if (n_q_heads % n_kv_heads) return ISOQ_E_GQA;
+  return plan_splits(n_seqs, n_kv_heads, max_seq_len).n_splits;
+}
+
+size_t isoq_decode_workspace_bytes(int n_seqs, int n_q_heads, int n_kv_heads, int d,
+                                   int max_seq_len) {
+  const int ns = isoq_decode_num_splits(n_seqs, n_q_heads, n_kv_heads, d, max_seq_len);
+  if (ns < 1) return 0;
+  return (size_t)n_seqs * n_q_heads * ns * isoq::partial_stride(d) * sizeof(float);
+}
+
+int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                          int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                          int max_seq_len, float* out, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  int rc = check_cache(cache, params);
+  if (rc) return rc;
+  if (n_seqs < 0 || n_q_heads < 0 || max_seq_len < 0 || !valid_dtype(q_dtype)) return ISOQ_E_ARG;
+  if (!(scale == scale) || isinf(scale)) return ISOQ_E_ARG;
+  if (n_q_heads % cache->n_kv_heads || n_q_heads / cache->n_kv_heads > 16) return ISOQ_E_GQA;
+  if (n_seqs > cache->n_seqs) return ISOQ_E_ARG;
+  if (n_seqs == 0 || n_q_heads == 0) return ISOQ_OK;
+  if (!Q || !seq_lens || !out || !workspace) return ISOQ_E_ARG;
+  if (((uintptr_t)workspace & 15u) != 0) return ISOQ_E_WORKSPACE;
+  const size_t need =
+      isoq_decode_workspace_bytes(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
+  if (workspace_bytes < need) return ISOQ_E_WORKSPACE;
+  if ((rc = check_device(params))) return rc;
+  const SplitPlan plan = plan_splits(n_seqs, cache->n_kv_heads, max_seq_len);
+  isoq::DecodeArgs a;
+  a.params = params->dev;
+  a.blocks = cache->blocks;
+  a.page_table = cache->page_table;
+  a.n_pages = cache->n_pages;
+  a.max_pages = cache->max_pages_per_seq;
+  a.n_kv_heads = cache->n_kv_heads;
+  a.d = cache->d;
+  a.Q = Q;
+  a.q_dtype = q_dtype;
+  a.n_seqs = n_seqs;
+  a.n_q_heads = n_q_heads;
+  a.seq_lens = seq_lens;
+  a.scale = scale;
+  a.n_splits = plan.n_splits;
+  a.pages_per_split = plan.pages_per_split;
+  a.partials = static_cast<float*>(workspace);
+  a.out = out;
+  a.status = cache->status;
+  cudaError_t e = isoq::launch_decode(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
+}
+
+int isoq_get_status(const isoq_cache* cache, uint32_t* host_bits) {
+  if (!cache || !host_bits) return ISOQ_E_ARG;
+  *host_bits = 0;
+  if (!cache->status) return ISOQ_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(host_bits, cache->status, 4, cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
+}
+
+int isoq_reset_status(const isoq_cache* cache, void* stream) {
+  if (!cache) return ISOQ_E_ARG;
+  if (!cache->status) return ISOQ_OK;
+  cudaError_t e = cudaMemsetAsync(cache->status, 0, 4, (cudaStream_t)stream);
+  return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
+}
+
+int isoq_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* isoq_error_string(int code) {
+  switch (code) {
+    case ISOQ_OK: return "ok";
+    case ISOQ_E_ARG: return "invalid argument";
+    case ISOQ_E_DIM: return "unsupported head dimension or page size";
+    case ISOQ_E_GQA: return "n_q_heads is not a multiple (<= 16x) of n_kv_heads";
+    case ISOQ_E_WORKSPACE: return "workspace too small or misaligned";
+    case ISOQ_E_CUDA: return "CUDA runtime error";
+    case ISOQ_E_DEVICE: return "no CUDA device or parameters on another device";
+  }
+  return "unknown";
+}
+
+}  // extern "C"

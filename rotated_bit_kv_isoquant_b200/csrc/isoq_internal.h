@@ -1,0 +1,47 @@
+// Internal launch interface between the C-ABI layer (isoq_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace isoq {
+
+struct QuantizeArgs {
+  const float* params;  // device [H][d/4][2][4]
+  uint8_t* blocks;
+  const int32_t* page_table;
+  int n_pages, max_pages, n_seqs, n_kv_heads, d;
+  const void* K;
+  const void* V;
+  int dtype;
+  int n_tokens;
+  const int32_t* seq_ids;
+  const int32_t* positions;
+  uint32_t* status;
+};
+
+struct DecodeArgs {
+  const float* params;
+  const uint8_t* blocks;
+  const int32_t* page_table;
+  int n_pages, max_pages, n_kv_heads, d;
+  const void* Q;
+  int q_dtype;
+  int n_seqs, n_q_heads;
+  const int32_t* seq_lens;
+  float scale;
+  int n_splits;         // context chunks per (sequence, KV head)
+  int pages_per_split;  // pages in each chunk
+  float* partials;      // [n_seqs][n_q_heads][n_splits][d + 4]
+  float* out;
+  uint32_t* status;
+};
+
+cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Partial-result stride (floats) of one (sequence, head, split): acc[d], m, l, 2 pad.
+inline int partial_stride(int d) { return d + 4; }
+
+}  // namespace isoq

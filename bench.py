@@ -45,6 +45,8 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="use only this many sequences of the workload (small profiling case)")
     return ap.parse_args()
 
 
@@ -411,6 +413,9 @@ def main():
     args = _args()
     import workloads as wl
     cfg = wl.workload(args.config)
+    if args.seqs:
+        from dataclasses import replace
+        cfg = replace(cfg, n_seqs=args.seqs)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -190,6 +190,36 @@ int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, co
                           int max_seq_len, float* out, float scale, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* =======================================================================================
+ * Decode attention that allocates nothing and takes no workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory themselves -- for instance a plug-in that a host application
+ * hands only its input and output buffers, or a thread that must not call cudaMalloc
+ * because that call can synchronise the device.  It computes exactly what
+ * isoq_decode_attention computes, with the same kernels and the same arguments minus
+ * the workspace.  The split-K partial results go to a fixed device array inside the
+ * library instead, of ISOQ_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library keeps until the process exits.
+ *
+ * Limit: calls whose isoq_decode_workspace_bytes(n_seqs, n_q_heads, n_kv_heads, d,
+ * max_seq_len) exceeds ISOQ_NOALLOC_SCRATCH_BYTES are rejected with ISOQ_E_WORKSPACE
+ * (nothing is launched).  All calls share the one array: two calls that overlap on the
+ * GPU (different streams, or threads without ordering between them) race and give wrong
+ * results.  The array keeps the previous call's contents; nothing has to be cleared,
+ * since each call writes every partial result it reads.  The first call on a device looks
+ * up the array's device address there (cudaGetSymbolAddress), so make that first call
+ * before any stream capture.  No cudaMalloc, cudaFree or allocating library routine is
+ * called.
+ * Errors: as isoq_decode_attention (ISOQ_E_WORKSPACE meaning "too large for the array").
+ * ===================================================================================== */
+#define ISOQ_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per device */
+
+int isoq_decode_attention_noalloc(const isoq_params* params, const isoq_cache* cache,
+                                  const void* Q, int q_dtype, int n_seqs, int n_q_heads,
+                                  const int32_t* seq_lens, int max_seq_len, float* out,
+                                  float scale, void* stream);
+
 /* Number of context chunks (splits) the decode uses for these sizes on the current
  * device; >= 1, or a negative error code. */
 int isoq_decode_num_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len);

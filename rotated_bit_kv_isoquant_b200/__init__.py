@@ -41,6 +41,7 @@ ISOQ_ST_LEN_RANGE = 0x10
 
 ISOQ_F32, ISOQ_BF16, ISOQ_F16 = 0, 1, 2
 ISOQ_PAGE_SIZE = 64
+ISOQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class IsoqError(RuntimeError):
@@ -73,6 +74,7 @@ _SIGS = {
     "isoq_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "isoq_decode_num_splits": (_i, [_i, _i, _i, _i, _i]),
     "isoq_decode_attention": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
+    "isoq_decode_attention_noalloc": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p]),
     "isoq_get_status": (_i, [_cp, ctypes.POINTER(ctypes.c_uint32)]),
     "isoq_reset_status": (_i, [_cp, _p]),
     "isoq_last_cuda_error": (_i, []),
@@ -232,6 +234,19 @@ def isoq_decode_attention(params: Params, cache: PagedCache, Q, seq_lens, max_se
         _dev_ptr(out, "out", torch.float32), float(scale), _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
         "isoq_decode_attention")
+
+
+def isoq_decode_attention_noalloc(params: Params, cache: PagedCache, Q, seq_lens,
+                                  max_seq_len: int, out, scale: float, stream=None) -> None:
+    """isoq_decode_attention without a workspace, for callers that cannot allocate device
+    memory: the partial results use a fixed 16 MiB array inside the library (one per GPU,
+    shared by all calls, so calls must not overlap on the GPU)."""
+    import torch
+    _check(_lib.isoq_decode_attention_noalloc(
+        params.handle, ctypes.byref(cache.c), _dev_ptr(Q, "Q"), _dtype_code(Q), Q.shape[0],
+        Q.shape[1], _dev_ptr(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
+        _dev_ptr(out, "out", torch.float32), float(scale), _stream_ptr(stream)),
+        "isoq_decode_attention_noalloc")
 
 
 def isoq_get_status(cache: PagedCache) -> int:

@@ -311,3 +311,12 @@ const char* isoq_error_string(int code) {
 }
 
 }  // extern "C"
+
+// Internal accessors for other translation units of the library (not part of the C ABI).
+namespace isoq {
+const float* params_device_ptr(const isoq_params* p) { return p ? p->dev : nullptr; }
+int params_device(const isoq_params* p) { return p ? p->device : -1; }
+}  // namespace isoq
+namespace isoq {
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace isoq

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+struct isoq_params;
+
 namespace isoq {
 
 struct QuantizeArgs {
@@ -40,6 +42,12 @@ struct DecodeArgs {
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Accessors of the opaque parameter handle (defined in isoq_api.cu).
+const float* params_device_ptr(const struct ::isoq_params* p);
+int params_device(const struct ::isoq_params* p);
+// Records e as the thread's last CUDA error and returns ISOQ_E_CUDA.
+int record_cuda_error(cudaError_t e);
 
 // Partial-result stride (floats) of one (sequence, head, split): acc[d], m, l, 2 pad.
 inline int partial_stride(int d) { return d + 4; }

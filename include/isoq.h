@@ -7,7 +7,7 @@
  * per-token, per-head K or V vector is passed through a Walsh-Hadamard transform, then
  * block-diagonal SO(4) rotations (quaternion rotations: "FreeToken issue #141, unified KV
  * cache backend", Proposed Solution, Quantization layer), then 3-bit scalar
- * quantisation; attention runs on the packed 3-bit tensors without materialising
+ * quantisation; attention reads the packed 3-bit codes directly and never rebuilds
  * full-precision K/V.  The pages fix none of the numeric details below; this library's
  * choices are stated with each declaration.
  *

@@ -2,8 +2,8 @@
 // inverse rotation.
 //
 // Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
-// Compressed-Space Attention", Abstract ("performs attention directly on packed 3-bit
-// tensors without materializing full-precision KV state").  Because the rotation R is
+// Compressed-Space Attention", Abstract: attention is computed on the packed 3-bit codes
+// and full-precision K/V are never reconstructed.  Because the rotation R is
 // orthogonal, q.k_hat = (R q).(R k_hat): the query is rotated once, every score and the
 // value accumulation run on codebook levels in the rotated space, and only the final
 // output is rotated back.  The context is split into chunks that run in parallel and are

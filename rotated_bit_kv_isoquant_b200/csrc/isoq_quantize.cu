@@ -1,8 +1,9 @@
 // Quantize-append kernel: WHT -> SO(4) blocks -> 3-bit codes -> packed paged cache.
 //
 // Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
-// Compressed-Space Attention", Abstract ("a Walsh-Hadamard transform followed by
-// block-diagonal SO(4) rotations ... before 3-bit scalar quantization", O(d log d) work).
+// Compressed-Space Attention", Abstract: each K/V vector goes through a Walsh-Hadamard
+// transform, then block-diagonal SO(4) rotations, then a 3-bit scalar quantiser, at
+// O(d log d) cost per vector.
 //
 // One warp per (token, KV head); it quantises the K vector and then the V vector, which
 // share the head's rotation parameters.  Lane l holds elements E*l .. E*l+E-1 (E = d/32),

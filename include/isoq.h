@@ -51,6 +51,7 @@ extern "C" {
 #define ISOQ_ST_PAGE_RANGE 0x4u /* a page-table entry outside [0, n_pages); page skipped */
 #define ISOQ_ST_NORM_SAT 0x8u   /* a norm >= 65520 was stored as 65504 (binary16 max) */
 #define ISOQ_ST_LEN_RANGE 0x10u /* decode: seq_len beyond the page table; clamped */
+#define ISOQ_ST_TIMEOUT 0x20u   /* decode: a bounded wait for a page copy gave up (no hang) */
 
 /* ---- element types of K, V and Q ---------------------------------------------------- */
 #define ISOQ_F32 0

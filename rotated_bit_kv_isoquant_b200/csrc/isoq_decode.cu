@@ -269,13 +269,7 @@ static cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
 
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
-  cudaError_t e;
-  switch (a.q_dtype) {
-    case ISOQ_F32: e = launch_g<D, float>(a, stream); break;
-    case ISOQ_BF16: e = launch_g<D, __nv_bfloat16>(a, stream); break;
-    case ISOQ_F16: e = launch_g<D, __half>(a, stream); break;
-    default: return cudaErrorInvalidValue;
-  }
+  cudaError_t e = launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_q_heads, a.n_seqs);
   decode_combine_kernel<D><<<grid, 32, 0, stream>>>(a.params, a.n_kv_heads, a.n_q_heads,

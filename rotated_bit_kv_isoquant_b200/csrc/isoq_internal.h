@@ -42,6 +42,8 @@ struct DecodeArgs {
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// Tensor-core split kernel (partials only); the combine runs separately.
+cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
 
 // Accessors of the opaque parameter handle (defined in isoq_api.cu).
 const float* params_device_ptr(const struct ::isoq_params* p);

@@ -78,15 +78,19 @@ struct SplitPlan {
   int pages_per_split;
 };
 
-// Context chunking for the decode kernel (4 warps per CTA, 2 resident CTAs per SM): about
-// four waves of (chunk, KV head, query-head block, sequence) CTAs, each chunk a whole
+#ifndef ISOQ_DEC_WAVES
+#define ISOQ_DEC_WAVES 4
+#endif
+
+// Context chunking for the decode kernel: about ISOQ_DEC_WAVES waves of (chunk, KV head,
+// query-head block, sequence) CTAs at the kernel's resident CTAs per SM, each chunk a whole
 // number of pages and at least 16 pages (4 per warp) when the context allows.
-SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int max_seq_len) {
-  const int n_sm = sm_count();
+SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len) {
+  const int n_sm = sm_count() * isoq::decode_resident_ctas(d);
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const int group = n_kv_heads > 0 ? n_q_heads / n_kv_heads : 1;
   const long long units = (long long)n_seqs * n_kv_heads * ((group + 7) / 8);
-  const long long target = (long long)n_sm * 2 * 4;
+  const long long target = (long long)n_sm * ISOQ_DEC_WAVES;
   long long want = units > 0 ? (target + units - 1) / units : 1;
   const long long cap = (max_pages + 15) / 16;
   if (want > cap) want = cap;
@@ -231,7 +235,7 @@ int isoq_decode_num_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int
   if (n_seqs < 0 || n_q_heads < 0 || n_kv_heads < 1 || max_seq_len < 0) return ISOQ_E_ARG;
   if (!supported_d(d)) return ISOQ_E_DIM;
   if (n_q_heads % n_kv_heads) return ISOQ_E_GQA;
-  return plan_splits(n_seqs, n_q_heads, n_kv_heads, max_seq_len).n_splits;
+  return plan_splits(n_seqs, n_q_heads, n_kv_heads, d, max_seq_len).n_splits;
 }
 
 size_t isoq_decode_workspace_bytes(int n_seqs, int n_q_heads, int n_kv_heads, int d,
@@ -258,7 +262,7 @@ int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, co
       isoq_decode_workspace_bytes(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
   if (workspace_bytes < need) return ISOQ_E_WORKSPACE;
   if ((rc = check_device(params))) return rc;
-  const SplitPlan plan = plan_splits(n_seqs, n_q_heads, cache->n_kv_heads, max_seq_len);
+  const SplitPlan plan = plan_splits(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
   isoq::DecodeArgs a;
   a.params = params->dev;
   a.blocks = cache->blocks;

@@ -200,38 +200,92 @@ __global__ void __launch_bounds__(32)
 }
 
 // a9: merge the splits of one (sequence, query head), normalise, inverse SO(4) blocks and
-// inverse (orthonormal, self-inverse) WHT.  One warp per (sequence, head).
+// inverse (orthonormal, self-inverse) WHT.  One CTA of 128 threads per (sequence, head):
+// the splits are spread over 4 groups of 32 lanes (each lane 4 or 8 dims, 16-byte loads,
+// several splits in flight), so the merge costs a few memory round trips however many
+// splits there are; warp 0 then applies the inverse rotation.
 template <int D>
-__global__ void __launch_bounds__(32)
+__global__ void __launch_bounds__(128)
     decode_combine_kernel(const float* __restrict__ params, int H, int n_q_heads, int n_splits,
                           const float* __restrict__ partials, float* __restrict__ out) {
-  constexpr int E = D / 32;
+  constexpr int E = D / 32;   // dims per lane
   constexpr int NB = E / 4;
   constexpr int PS = D + 4;
-  const int lane = threadIdx.x;
+  constexpr int UNROLL = 4;
+  __shared__ float red_m[4];
+  __shared__ float red_acc[4][D];
+  __shared__ float red_l[4];
+  const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   const int s = blockIdx.y, h = blockIdx.x;
   const int G = n_q_heads / H;
   const float* base = partials + ((size_t)s * n_q_heads + h) * n_splits * PS;
 
-  float M = -CUDART_INF_F, Ls = 0.f, acc[E];
+  // global max of the splits' running maxima (empty splits report -inf)
+  float M = -CUDART_INF_F;
+  for (int j = tid; j < n_splits; j += 128) M = fmaxf(M, __ldg(base + (size_t)j * PS + D));
+  M = warp_max(M);
+  if (lane == 0) red_m[grp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+
+  float acc[E], L = 0.f;
 #pragma unroll
   for (int i = 0; i < E; ++i) acc[i] = 0.f;
-  for (int j = 0; j < n_splits; ++j) {
-    const float* p = base + (size_t)j * PS;
-    const float mj = p[D];
-    if (mj == -CUDART_INF_F) continue;  // empty split: contributes nothing
-    const float mn = fmaxf(M, mj);
-    const float a = __expf(M - mn), b = __expf(mj - mn);
-    Ls = Ls * a + p[D + 1] * b;
+  if (M != -CUDART_INF_F) {
+    int j = grp;
+    for (; j + 4 * (UNROLL - 1) < n_splits; j += 4 * UNROLL) {
+      float mj[UNROLL], lj[UNROLL];
+      float4 v[UNROLL][NB];
 #pragma unroll
-    for (int i = 0; i < E; ++i) acc[i] = acc[i] * a + p[lane * E + i] * b;
-    M = mn;
+      for (int u = 0; u < UNROLL; ++u) {
+        const float* p = base + (size_t)(j + 4 * u) * PS;
+        mj[u] = __ldg(p + D);
+        lj[u] = __ldg(p + D + 1);
+#pragma unroll
+        for (int k = 0; k < NB; ++k) v[u][k] = __ldg(reinterpret_cast<const float4*>(p + lane * E) + k);
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const float w = mj[u] == -CUDART_INF_F ? 0.f : __expf(mj[u] - M);
+        L = fmaf(w, lj[u], L);
+#pragma unroll
+        for (int k = 0; k < NB; ++k) {
+          acc[4 * k + 0] = fmaf(w, v[u][k].x, acc[4 * k + 0]);
+          acc[4 * k + 1] = fmaf(w, v[u][k].y, acc[4 * k + 1]);
+          acc[4 * k + 2] = fmaf(w, v[u][k].z, acc[4 * k + 2]);
+          acc[4 * k + 3] = fmaf(w, v[u][k].w, acc[4 * k + 3]);
+        }
+      }
+    }
+    for (; j < n_splits; j += 4) {
+      const float* p = base + (size_t)j * PS;
+      const float mj = __ldg(p + D);
+      const float w = mj == -CUDART_INF_F ? 0.f : __expf(mj - M);
+      L = fmaf(w, __ldg(p + D + 1), L);
+#pragma unroll
+      for (int k = 0; k < NB; ++k) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(p + lane * E) + k);
+        acc[4 * k + 0] = fmaf(w, x.x, acc[4 * k + 0]);
+        acc[4 * k + 1] = fmaf(w, x.y, acc[4 * k + 1]);
+        acc[4 * k + 2] = fmaf(w, x.z, acc[4 * k + 2]);
+        acc[4 * k + 3] = fmaf(w, x.w, acc[4 * k + 3]);
+      }
+    }
   }
-  float o[E];
-  const float inv = Ls > 0.f ? 1.f / (Ls * sqrtf((float)D)) : 0.f;
 #pragma unroll
-  for (int i = 0; i < E; ++i) o[i] = acc[i] * inv;
+  for (int i = 0; i < E; ++i) red_acc[grp][lane * E + i] = acc[i];
+  if (lane == 0) red_l[grp] = L;
+  __syncthreads();
+  if (grp != 0) return;
 
+  const float Ls = red_l[0] + red_l[1] + red_l[2] + red_l[3];
+  const float inv = Ls > 0.f ? 1.f / (Ls * sqrtf((float)D)) : 0.f;
+  float o[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const int dd = lane * E + i;
+    o[i] = (red_acc[0][dd] + red_acc[1][dd] + red_acc[2][dd] + red_acc[3][dd]) * inv;
+  }
   const float* hp = params + (size_t)(h / G) * D * 2;
   float y[E];
 #pragma unroll
@@ -272,7 +326,7 @@ static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_q_heads, a.n_seqs);
-  decode_combine_kernel<D><<<grid, 32, 0, stream>>>(a.params, a.n_kv_heads, a.n_q_heads,
+  decode_combine_kernel<D><<<grid, 128, 0, stream>>>(a.params, a.n_kv_heads, a.n_q_heads,
                                                     a.n_splits, a.partials, a.out);
   return cudaGetLastError();
 }

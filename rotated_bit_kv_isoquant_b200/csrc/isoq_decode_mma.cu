@@ -428,17 +428,18 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
       for (int gq = 0; gq < NG; ++gq) {
         const int q = (g >> 1) + 4 * gq;
-        const int j0 = 2 * (g & 1);
         const uint8_t* vbase = blk + v_codes_off(D);
+        const bool odd = (g & 1) != 0;  // odd g: words 2, 3 (w2 and the spare bits)
         uint32_t S[4][2];  // [token 2t, 2t+1, 2t+8, 2t+9][word j0, j0+1]
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int tk = tb + 2 * t + (r & 1) + 8 * (r >> 1);
           const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + 3 * q;
-          uint32_t Sx[4];
-          selectors(w[0], w[1], w[2], Sx);
-          S[r][0] = Sx[j0];
-          S[r][1] = Sx[j0 + 1];
+          const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
+          const uint32_t spare =
+              ((w0 & 0x88888888u) >> 1) | ((w1 & 0x88888888u) >> 2) | ((w2 & 0x88888888u) >> 3);
+          S[r][0] = (odd ? w2 : w0) & 0x77777777u;
+          S[r][1] = odd ? spare : (w1 & 0x77777777u);
         }
         uint32_t f[4][8];  // [pair/word combo][nibble = m-tile]
         deq8_pair(S[0][0], S[1][0], tl0, tl1, th0, th1, f[0]);  // tokens 2t,2t+1 word j0
@@ -563,10 +564,54 @@ cudaError_t launch_decode_mma_d(const DecodeArgs& a, cudaStream_t stream) {
   return cudaErrorInvalidValue;
 }
 
+#ifndef ISOQ_DEC_NST128
+#define ISOQ_DEC_NST128 2
+#endif
+#ifndef ISOQ_DEC_NST256
+#define ISOQ_DEC_NST256 2
+#endif
+
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.d == 128) return launch_decode_mma_d<128, 3>(a, stream);
-  if (a.d == 256) return launch_decode_mma_d<256, 2>(a, stream);
+  if (a.d == 128) return launch_decode_mma_d<128, ISOQ_DEC_NST128>(a, stream);
+  if (a.d == 256) return launch_decode_mma_d<256, ISOQ_DEC_NST256>(a, stream);
   return cudaErrorInvalidValue;
+}
+
+// Resident CTAs per SM of the decode kernel for head dimension d on the current device
+// (cached per device; 2 when it cannot be queried).
+int decode_resident_ctas(int d) {
+  static int cache[64][2] = {{0}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 2;
+  }
+  const int di = d == 256 ? 1 : 0;
+  if (!cache[dev][di]) {
+    int n = 0;
+    cudaError_t e;
+    if (d == 256) {
+      using SM = MmaSmem<256, ISOQ_DEC_NST256>;
+      e = cudaFuncSetAttribute(decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+      if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16>, kWarps * 32, SM::kBytes);
+    } else {
+      using SM = MmaSmem<128, ISOQ_DEC_NST128>;
+      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+      if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16>, kWarps * 32, SM::kBytes);
+    }
+    if (e != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 2;
+    }
+    cache[dev][di] = n;
+  }
+  return cache[dev][di];
 }
 
 }  // namespace isoq

@@ -44,6 +44,8 @@ cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, i
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Tensor-core split kernel (partials only); the combine runs separately.
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
+// Resident CTAs per SM of that kernel for head dimension d on the current device.
+int decode_resident_ctas(int d);
 
 // Accessors of the opaque parameter handle (defined in isoq_api.cu).
 const float* params_device_ptr(const struct ::isoq_params* p);

@@ -16,8 +16,9 @@ struct isoq_params {
   int d;
   int n_kv_heads;
   int device;
-  float* dev;               // [n_kv_heads][d/4][2][4]
-  std::vector<float> host;  // same values
+  float* dev;               // [n_kv_heads][d/4][2][4] quaternions (the 256 parameters/head)
+  float* dev_mat;           // [n_kv_heads][d/4][4][4] derived: matrix of y -> p y conj(q)
+  std::vector<float> host;  // quaternions, same values as dev
 };
 
 namespace {
@@ -49,6 +50,14 @@ double std_normal(uint64_t& state) {
   const double u2 = (double)k2 * two_m53;
   const double two_pi = 2.0 * 3.14159265358979323846;
   return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
+}
+
+// Hamilton product of quaternions (w, x, y, z), binary64.
+void hamilton(const double* a, const double* b, double* o) {
+  o[0] = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
+  o[1] = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
+  o[2] = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
+  o[3] = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
 }
 
 // SM count of the current device (148 on B200 when no device can be queried, which keeps
@@ -157,6 +166,7 @@ int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
   p->d = d;
   p->n_kv_heads = n_kv_heads;
   p->dev = nullptr;
+  p->dev_mat = nullptr;
   p->host.resize((size_t)n_kv_heads * d * 2);
   isoq_params_generate(seed, d, n_kv_heads, p->host.data());
   cudaError_t e = cudaGetDevice(&p->device);
@@ -166,9 +176,30 @@ int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
     delete p;
     return ISOQ_E_DEVICE;
   }
-  const size_t bytes = p->host.size() * sizeof(float);
+  // Derived copy for the quantiser: each block rotation as a 4x4 row-major matrix, column j
+  // = p * e_j * conj(q), computed in binary64 from the binary32 quaternions.
+  const size_t nq = p->host.size();
+  std::vector<float> mats((size_t)n_kv_heads * (d / 4) * 16);
+  for (size_t blk = 0; blk < (size_t)n_kv_heads * (d / 4); ++blk) {
+    const float* pq = p->host.data() + blk * 8;
+    const double P[4] = {pq[0], pq[1], pq[2], pq[3]};
+    const double Qc[4] = {pq[4], -(double)pq[5], -(double)pq[6], -(double)pq[7]};
+    for (int j = 0; j < 4; ++j) {
+      double e[4] = {0, 0, 0, 0}, tq[4], z[4];
+      e[j] = 1.0;
+      hamilton(P, e, tq);
+      hamilton(tq, Qc, z);
+      for (int i = 0; i < 4; ++i) mats[blk * 16 + i * 4 + j] = (float)z[i];
+    }
+  }
+  const size_t bytes = (nq + mats.size()) * sizeof(float);
   e = cudaMalloc(&p->dev, bytes);
-  if (e == cudaSuccess) e = cudaMemcpy(p->dev, p->host.data(), bytes, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) {
+    p->dev_mat = p->dev + nq;
+    e = cudaMemcpy(p->dev, p->host.data(), nq * sizeof(float), cudaMemcpyHostToDevice);
+  }
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->dev_mat, mats.data(), mats.size() * sizeof(float), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     if (p->dev) cudaFree(p->dev);
     delete p;
@@ -213,6 +244,7 @@ int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, con
   if ((rc = check_device(params))) return rc;
   isoq::QuantizeArgs a;
   a.params = params->dev;
+  a.mats = params->dev_mat;
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;
   a.n_pages = cache->n_pages;

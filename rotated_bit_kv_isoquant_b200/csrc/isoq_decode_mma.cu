@@ -117,24 +117,46 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Right shifts done as the high half of a multiplication by 2^(32-k).  `mul` comes from a
+// kernel argument (2^16), so the compiler cannot fold it back into a shift: the product
+// runs on the FMA pipe and leaves the ALU pipe, which the byte permutes saturate, free.
+struct Shifter {
+  uint32_t m16, m29, m30, m31;
+  __device__ __forceinline__ explicit Shifter(uint32_t mul16)
+      : m16(mul16), m29(mul16 << 13), m30(mul16 << 14), m31(mul16 << 15) {}
+  __device__ __forceinline__ uint32_t shr16(uint32_t x) const { return __umulhi(x, m16); }
+  // spare codes: bit (2-b) of code 24+k is bit 4k+3 of w_b -> nibble k
+  __device__ __forceinline__ uint32_t spare(uint32_t w0, uint32_t w1, uint32_t w2) const {
+    uint32_t r;
+    asm("{\n .reg .u32 t;\n"
+        " mul.hi.u32 t, %1, %4;\n"
+        " mad.hi.u32 t, %2, %5, t;\n"
+        " mad.hi.u32 %0, %3, %6, t;\n}"
+        : "=r"(r)
+        : "r"(w2 & 0x88888888u), "r"(w1 & 0x88888888u), "r"(w0 & 0x88888888u), "r"(m29),
+          "r"(m30), "r"(m31));
+    return r;
+  }
+};
+
 // The three words of group q of a packed vector -> four 8-nibble selector words:
 // S[j] nibble n = code of dim 32q + 8j + n (bit 3 of every nibble clear).
-__device__ __forceinline__ void selectors(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&S)[4]) {
+__device__ __forceinline__ void selectors(uint32_t w0, uint32_t w1, uint32_t w2, const Shifter& sh,
+                                          uint32_t (&S)[4]) {
   S[0] = w0 & 0x77777777u;
   S[1] = w1 & 0x77777777u;
   S[2] = w2 & 0x77777777u;
-  // spare bits: bit (2-b) of code 24+k is bit 4k+3 of w_b
-  S[3] = ((w0 & 0x88888888u) >> 1) | ((w1 & 0x88888888u) >> 2) | ((w2 & 0x88888888u) >> 3);
+  S[3] = sh.spare(w0, w1, w2);
 }
 
 // Eight f16 values of the nibbles of S: o[i] = (level(nibble 2i), level(nibble 2i+1)).
 __device__ __forceinline__ void deq8(uint32_t S, uint32_t tl0, uint32_t tl1, uint32_t th0,
-                                     uint32_t th1, uint32_t (&o)[4]) {
+                                     uint32_t th1, const Shifter& sh, uint32_t (&o)[4]) {
   uint32_t lo = prmt(tl0, tl1, S);
   uint32_t hi = prmt(th0, th1, S);
   o[0] = prmt(lo, hi, 0x5140);
   o[1] = prmt(lo, hi, 0x7362);
-  const uint32_t S2 = S >> 16;
+  const uint32_t S2 = sh.shr16(S);
   lo = prmt(tl0, tl1, S2);
   hi = prmt(th0, th1, S2);
   o[2] = prmt(lo, hi, 0x5140);
@@ -144,14 +166,15 @@ __device__ __forceinline__ void deq8(uint32_t S, uint32_t tl0, uint32_t tl1, uin
 // Token pair (a, b), selector words Sa, Sb of the same dims: o[n] = (level a, level b) of
 // nibble n (n = 0..7), i.e. an f16x2 of two tokens for one dim.
 __device__ __forceinline__ void deq8_pair(uint32_t Sa, uint32_t Sb, uint32_t tl0, uint32_t tl1,
-                                          uint32_t th0, uint32_t th1, uint32_t (&o)[8]) {
+                                          uint32_t th0, uint32_t th1, const Shifter& sh,
+                                          uint32_t (&o)[8]) {
 #pragma unroll
   for (int part = 0; part < 2; ++part) {
     // nibbles (a n, a n+1, b n, b n+1, a n+2, a n+3, b n+2, b n+3) with n = 4 part
     const uint32_t X = prmt(Sa, Sb, part == 0 ? 0x5140u : 0x7362u);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t sel = hh == 0 ? X : (X >> 16);
+      const uint32_t sel = hh == 0 ? X : sh.shr16(X);
       const uint32_t lo = prmt(tl0, tl1, sel);
       const uint32_t hi = prmt(th0, th1, sel);
       o[4 * part + 2 * hh + 0] = prmt(lo, hi, 0x6240);
@@ -174,7 +197,10 @@ struct MmaSmem {
   static constexpr int kRing = kWarps * NST * kStageBytes;
   static constexpr int kBarOff = kRing;
   static constexpr int kQOff = kBarOff + kWarps * NST * 8;
-  static constexpr int kBytes = kQOff + 8 * D * 4;
+  // rotated queries, row stride kQS floats: dim d of head h at h*kQS + 40*(d/32) + d%32, so
+  // the 16-byte fragment loads of a quarter warp hit distinct banks
+  static constexpr int kQS = 40 * (D / 32) + 4;
+  static constexpr int kBytes = kQOff + 8 * kQS * 4;
   static constexpr int kMergeBytes = kWarps * 8 * (D + 4) * 4;
   static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
 };
@@ -185,7 +211,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                       const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                       const TQ* __restrict__ Q, int n_q_heads, const int32_t* __restrict__ seq_lens,
                       float scale, int pages_per_split, int n_splits, float* __restrict__ partials,
-                      uint32_t* status) {
+                      uint32_t* status, uint32_t mul16) {
   using SM = MmaSmem<D, NST>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
@@ -272,7 +298,10 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
       for (int k = 0; k < NB; ++k) so4_fwd(pq[k], v + 4 * k, z + 4 * k);
 #pragma unroll
-      for (int i = 0; i < E; ++i) qs[h * D + lane * E + i] = z[i];
+      for (int i = 0; i < E; ++i) {
+        const int dd = lane * E + i;
+        qs[h * SM::kQS + 40 * (dd >> 5) + (dd & 31)] = z[i];
+      }
     }
   }
   __syncthreads();
@@ -285,8 +314,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   uint32_t qb0[KS], qb1[KS], ql0[KS], ql1[KS];
 #pragma unroll
   for (int kk = 0; kk < KS; ++kk) {
-    const int base = 32 * (t + 4 * (kk / 8)) + 4 * (kk % 8);
-    const float* q = qs + g * D + base;
+    const float* q = qs + g * SM::kQS + 40 * (t + 4 * (kk / 8)) + 4 * (kk % 8);
     float hi[4], lo[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -323,6 +351,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   const float kf = scale * kLog2e / (kAlpha * (float)D);  // log2 score per (dot * nK)
 
+  const Shifter sh(mul16);
   bool timed_out = false;
   int k = 0;
   for (; k < n_my; ++k) {
@@ -337,56 +366,67 @@ __global__ void __launch_bounds__(kWarps * 32)
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
 
-#pragma unroll 1
-    for (int tb = 0; tb < kPage; tb += 16) {
-      // ---- a7: scores, A = K_hat rows (tokens tb+g, tb+g+8), 32 dims of group t ------
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int gq = 0; gq < NG; ++gq) {
-        const int q = t + 4 * gq;
-        const uint32_t* ra = reinterpret_cast<const uint32_t*>(blk + (tb + g) * CB) + 3 * q;
-        const uint32_t* rb = reinterpret_cast<const uint32_t*>(blk + (tb + g + 8) * CB) + 3 * q;
-        uint32_t Sa[4], Sb[4];
-        selectors(ra[0], ra[1], ra[2], Sa);
-        selectors(rb[0], rb[1], rb[2], Sb);
+    for (int tb = 0; tb < kPage; tb += 32) {
+      // ---- a7: scores for two 16-token sub-tiles; A = K_hat rows (tokens r+g, r+g+8) ----
+      // four independent accumulator chains per sub-tile (k-step parity x hi/lo part of
+      // the query) so consecutive mma instructions do not wait on each other's results
+      float sc[2][4], part[2][4][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t fa[4], fb[4];
-          deq8(Sa[j], tl0, tl1, th0, th1, fa);
-          deq8(Sb[j], tl0, tl1, th0, th1, fb);
-          const int kk0 = 8 * gq + 2 * j;
-          mma16816(sc, fa[0], fb[0], fa[1], fb[1], qb0[kk0], qb1[kk0]);
-          mma16816(sc, fa[2], fb[2], fa[3], fb[3], qb0[kk0 + 1], qb1[kk0 + 1]);
-          mma16816(sc, fa[0], fb[0], fa[1], fb[1], ql0[kk0], ql1[kk0]);
-          mma16816(sc, fa[2], fb[2], fa[3], fb[3], ql0[kk0 + 1], ql1[kk0 + 1]);
+      for (int sub = 0; sub < 2; ++sub) {
+        const int r = tb + 16 * sub;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) part[sub][c][0] = part[sub][c][1] = part[sub][c][2] = part[sub][c][3] = 0.f;
+#pragma unroll
+        for (int gq = 0; gq < NG; ++gq) {
+          const int q = t + 4 * gq;
+          const uint32_t* ra = reinterpret_cast<const uint32_t*>(blk + (r + g) * CB) + 3 * q;
+          const uint32_t* rb = reinterpret_cast<const uint32_t*>(blk + (r + g + 8) * CB) + 3 * q;
+          uint32_t Sa[4], Sb[4];
+          selectors(ra[0], ra[1], ra[2], sh, Sa);
+          selectors(rb[0], rb[1], rb[2], sh, Sb);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t fa[4], fb[4];
+            deq8(Sa[j], tl0, tl1, th0, th1, sh, fa);
+            deq8(Sb[j], tl0, tl1, th0, th1, sh, fb);
+            const int kk0 = 8 * gq + 2 * j;
+            mma16816(part[sub][0], fa[0], fb[0], fa[1], fb[1], qb0[kk0], qb1[kk0]);
+            mma16816(part[sub][1], fa[2], fb[2], fa[3], fb[3], qb0[kk0 + 1], qb1[kk0 + 1]);
+            mma16816(part[sub][2], fa[0], fb[0], fa[1], fb[1], ql0[kk0], ql1[kk0]);
+            mma16816(part[sub][3], fa[2], fb[2], fa[3], fb[3], ql0[kk0 + 1], ql1[kk0 + 1]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sc[sub][i] = (part[sub][0][i] + part[sub][1][i]) + (part[sub][2][i] + part[sub][3][i]);
+      }
+      // token validity and norms of this thread's C rows: tokens tb+16sub+g (+8)
+      float s2[2][4], nv[2][2];
+      bool vd[2][2];
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int tk = tb + 16 * sub + g + 8 * rr;
+          vd[sub][rr] = page_ok && (tok0 + tk) < len;
+          const float nk = half_at(blk + k_norm_off(D) + 2 * tk);
+          nv[sub][rr] = vd[sub][rr] ? half_at(blk + v_norm_off(D) + 2 * tk) : 0.f;
+          s2[sub][2 * rr + 0] = vd[sub][rr] ? sc[sub][2 * rr + 0] * nk * kf : -CUDART_INF_F;
+          s2[sub][2 * rr + 1] = vd[sub][rr] ? sc[sub][2 * rr + 1] * nk * kf : -CUDART_INF_F;
         }
       }
-      // token validity and norms for this thread's C rows (tokens tb+g, tb+g+8)
-      const int ta = tb + g, tbb = tb + g + 8;
-      const bool va = page_ok && (tok0 + ta) < len;
-      const bool vb = page_ok && (tok0 + tbb) < len;
-      const float nka = half_at(blk + k_norm_off(D) + 2 * ta);
-      const float nkb = half_at(blk + k_norm_off(D) + 2 * tbb);
-      const float nva = va ? half_at(blk + v_norm_off(D) + 2 * ta) : 0.f;
-      const float nvb = vb ? half_at(blk + v_norm_off(D) + 2 * tbb) : 0.f;
-      // log2-domain scores; invalid tokens -> -inf
-      float s2[4];
-      s2[0] = va ? sc[0] * nka * kf : -CUDART_INF_F;
-      s2[1] = va ? sc[1] * nka * kf : -CUDART_INF_F;
-      s2[2] = vb ? sc[2] * nkb * kf : -CUDART_INF_F;
-      s2[3] = vb ? sc[3] * nkb * kf : -CUDART_INF_F;
 
-      // ---- a8: online softmax (per head: max over the tile's 16 tokens) ---------------
-      float tmax[2] = {fmaxf(s2[0], s2[2]), fmaxf(s2[1], s2[3])};
+      // ---- a8: online softmax over the 32 tokens (per head: 4 values here, 3 shuffles) --
+      float tmax[2] = {fmaxf(fmaxf(s2[0][0], s2[0][2]), fmaxf(s2[1][0], s2[1][2])),
+                       fmaxf(fmaxf(s2[0][1], s2[0][3]), fmaxf(s2[1][1], s2[1][3]))};
+      float vmax = fmaxf(fmaxf(nv[0][0], nv[0][1]), fmaxf(nv[1][0], nv[1][1]));
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) tmax[e] = fmaxf(tmax[e], __shfl_xor_sync(kFull, tmax[e], o));
+      for (int o = 4; o < 32; o <<= 1) {
+        tmax[0] = fmaxf(tmax[0], __shfl_xor_sync(kFull, tmax[0], o));
+        tmax[1] = fmaxf(tmax[1], __shfl_xor_sync(kFull, tmax[1], o));
+        vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
       }
-      float vmax = fmaxf(nva, nvb);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
-
       float resc[2] = {1.f, 1.f};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -397,9 +437,9 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
       }
       if (vmax > sigma * kSigmaSlack) {
-        const float r = sigma / vmax;  // 0 on the first valid tile
-        resc[0] *= r;
-        resc[1] *= r;
+        const float rr = sigma / vmax;  // 0 on the first valid tile
+        resc[0] *= rr;
+        resc[1] *= rr;
         sigma = vmax;
       }
       if (resc[0] != 1.f || resc[1] != 1.f) {
@@ -412,43 +452,53 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
       }
       const float inv_sigma = sigma > 0.f ? 1.f / sigma : 0.f;
-      float p[4];
-      p[0] = va ? ex2(s2[0] - m2[0]) : 0.f;
-      p[1] = va ? ex2(s2[1] - m2[1]) : 0.f;
-      p[2] = vb ? ex2(s2[2] - m2[0]) : 0.f;
-      p[3] = vb ? ex2(s2[3] - m2[1]) : 0.f;
-      lsum[0] += p[0] + p[2];
-      lsum[1] += p[1] + p[3];
-      const float wa = nva * inv_sigma, wb = nvb * inv_sigma;
-      // P'^T fragments: transpose the two 8x8 blocks (tokens 0-7, 8-15) of P'
-      const uint32_t pb0 = movmatrix_t(pack_f16x2(p[0] * wa, p[1] * wa));
-      const uint32_t pb1 = movmatrix_t(pack_f16x2(p[2] * wb, p[3] * wb));
+      uint32_t pb[2][2];
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        float pw[4];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const float p0 = vd[sub][rr] ? ex2(s2[sub][2 * rr] - m2[0]) : 0.f;
+          const float p1 = vd[sub][rr] ? ex2(s2[sub][2 * rr + 1] - m2[1]) : 0.f;
+          lsum[0] += p0;
+          lsum[1] += p1;
+          const float w = nv[sub][rr] * inv_sigma;
+          pw[2 * rr] = p0 * w;
+          pw[2 * rr + 1] = p1 * w;
+        }
+        // P'^T fragments: transpose the two 8x8 blocks (tokens 0-7, 8-15 of the sub-tile)
+        pb[sub][0] = movmatrix_t(pack_f16x2(pw[0], pw[1]));
+        pb[sub][1] = movmatrix_t(pack_f16x2(pw[2], pw[3]));
+      }
 
       // ---- a8: V accumulation, A = V_hat^T (rows = dims, k = tokens 2t,2t+1,2t+8,2t+9) --
 #pragma unroll
-      for (int gq = 0; gq < NG; ++gq) {
-        const int q = (g >> 1) + 4 * gq;
-        const uint8_t* vbase = blk + v_codes_off(D);
-        const bool odd = (g & 1) != 0;  // odd g: words 2, 3 (w2 and the spare bits)
-        uint32_t S[4][2];  // [token 2t, 2t+1, 2t+8, 2t+9][word j0, j0+1]
+      for (int sub = 0; sub < 2; ++sub) {
+        const int r = tb + 16 * sub;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int tk = tb + 2 * t + (r & 1) + 8 * (r >> 1);
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + 3 * q;
-          const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
-          const uint32_t spare =
-              ((w0 & 0x88888888u) >> 1) | ((w1 & 0x88888888u) >> 2) | ((w2 & 0x88888888u) >> 3);
-          S[r][0] = (odd ? w2 : w0) & 0x77777777u;
-          S[r][1] = odd ? spare : (w1 & 0x77777777u);
+        for (int gq = 0; gq < NG; ++gq) {
+          const int q = (g >> 1) + 4 * gq;
+          const uint8_t* vbase = blk + v_codes_off(D);
+          const bool odd = (g & 1) != 0;  // odd g: words 2, 3 (w2 and the spare bits)
+          uint32_t S[4][2];  // [token 2t, 2t+1, 2t+8, 2t+9][word j0, j0+1]
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const int tk = r + 2 * t + (x & 1) + 8 * (x >> 1);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + 3 * q;
+            const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
+            S[x][0] = (odd ? w2 : w0) & 0x77777777u;
+            S[x][1] = odd ? sh.spare(w0, w1, w2) : (w1 & 0x77777777u);
+          }
+          uint32_t f[4][8];  // [pair/word combo][nibble = m-tile]
+          deq8_pair(S[0][0], S[1][0], tl0, tl1, th0, th1, sh, f[0]);
+          deq8_pair(S[0][1], S[1][1], tl0, tl1, th0, th1, sh, f[1]);
+          deq8_pair(S[2][0], S[3][0], tl0, tl1, th0, th1, sh, f[2]);
+          deq8_pair(S[2][1], S[3][1], tl0, tl1, th0, th1, sh, f[3]);
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+            mma16816(acc[8 * gq + mt], f[0][mt], f[1][mt], f[2][mt], f[3][mt], pb[sub][0],
+                     pb[sub][1]);
         }
-        uint32_t f[4][8];  // [pair/word combo][nibble = m-tile]
-        deq8_pair(S[0][0], S[1][0], tl0, tl1, th0, th1, f[0]);  // tokens 2t,2t+1 word j0
-        deq8_pair(S[0][1], S[1][1], tl0, tl1, th0, th1, f[1]);  // tokens 2t,2t+1 word j0+1
-        deq8_pair(S[2][0], S[3][0], tl0, tl1, th0, th1, f[2]);  // tokens 2t+8,2t+9 word j0
-        deq8_pair(S[2][1], S[3][1], tl0, tl1, th0, th1, f[3]);  // tokens 2t+8,2t+9 word j0+1
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-          mma16816(acc[8 * gq + mt], f[0][mt], f[1][mt], f[2][mt], f[3][mt], pb0, pb1);
       }
     }
     __syncwarp();
@@ -550,7 +600,7 @@ static cudaError_t launch_mma_t(const DecodeArgs& a, cudaStream_t stream) {
   decode_mma_kernel<D, NST, TQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.seq_lens, a.scale, a.pages_per_split,
-      a.n_splits, a.partials, a.status);
+      a.n_splits, a.partials, a.status, 65536u);
   return cudaGetLastError();
 }
 

@@ -11,6 +11,7 @@ namespace isoq {
 
 struct QuantizeArgs {
   const float* params;  // device [H][d/4][2][4]
+  const float* mats;    // device [H][d/4][4][4]: block rotations as matrices
   uint8_t* blocks;
   const int32_t* page_table;
   int n_pages, max_pages, n_seqs, n_kv_heads, d;

@@ -5,21 +5,38 @@
 // transform, then block-diagonal SO(4) rotations, then a 3-bit scalar quantiser, at
 // O(d log d) cost per vector.
 //
-// One warp per (token, KV head); it quantises the K vector and then the V vector, which
-// share the head's rotation parameters.  Lane l holds elements E*l .. E*l+E-1 (E = d/32),
-// which makes the WHT's first log2(E) butterfly stages lane-local and the remaining five
-// __shfl_xor_sync stages; the lane's E elements are exactly its E/4 quaternion blocks, so
-// the SO(4) step is lane-local too.  The norm is a warp sum of squares.  Codes are counted
-// against the 7 thresholds scaled by the norm (no division), packed with shuffles into the
-// 12-byte group layout of isoq.h and written as 16-byte stores.
+// One warp per token: for each KV head it quantises the K and the V vector together (they
+// share the head's rotation).  Lane l holds elements E*l .. E*l+E-1 (E = d/32), which makes
+// the WHT's first log2(E) butterfly stages lane-local and the remaining five
+// __shfl_xor_sync stages (one FFMA each); the lane's E elements are exactly its E/4 SO(4)
+// blocks, so the rotation is lane-local too (applied as the block's 4x4 matrix, derived
+// from the quaternion pair when the parameters are made).  The norm is a warp sum of
+// squares.  Codes are decided against the thresholds scaled by the norm (no division),
+// packed with shuffles into the 12-byte group layout of isoq.h and written as 16-byte
+// stores.
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 
 namespace isoq {
 
+// Code of one rotated coordinate z (scaled by sqrt(d)) against thresholds T[k] = n * tau_k
+// (tau = 0.50055, 1.05, 1.748, the positive midpoints; the codebook is symmetric).  The
+// definition code = #{j : z >= t_j} over t = (-T3, -T2, -T1, 0, T1, T2, T3) equals
+//   z >= 0: 4 + #{k : |z| >= T_k}         z < 0: 3 - #{k : |z| > T_k}
+// and for non-negative floats "a > T" is "bits(a) - 1 >= bits(T)", so one set of integer
+// compares on bits(|z|) - [z < 0] serves both signs exactly; 3 - m = (4 + m) ^ 7.
+__device__ __forceinline__ uint32_t code_of(float z, const uint32_t (&tb)[3]) {
+  const uint32_t neg = z < 0.f ? 1u : 0u;
+  const uint32_t ai = (__float_as_uint(z) & 0x7fffffffu) - neg;
+  const uint32_t m = (ai >= tb[0] ? 1u : 0u) + (ai >= tb[1] ? 1u : 0u) + (ai >= tb[2] ? 1u : 0u);
+  return (4u + m) ^ (neg * 7u);
+}
+
+// One warp per token; it walks the KV heads and, per head, quantises K and V together
+// (two independent chains for the scheduler).
 template <int D, typename T>
 __global__ void __launch_bounds__(256)
-    quantize_append_kernel(const float* __restrict__ params, uint8_t* __restrict__ blocks,
+    quantize_append_kernel(const float* __restrict__ mats, uint8_t* __restrict__ blocks,
                            const int32_t* __restrict__ page_table, int n_pages, int max_pages,
                            int n_seqs, int H, const T* __restrict__ K, const T* __restrict__ V,
                            int n_tokens, const int32_t* __restrict__ seq_ids,
@@ -30,12 +47,13 @@ __global__ void __launch_bounds__(256)
   constexpr int BB = block_bytes(D);
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  const long long total = (long long)n_tokens * H;
-  const long long stride = (long long)gridDim.x * wpb;
+  // butterfly sign of this lane in cross-lane stage s: the lower lane keeps a+b, the upper
+  // a-b, i.e. fma(sign, own, partner)
+  float bsign[5];
+#pragma unroll
+  for (int st = 0; st < 5; ++st) bsign[st] = ((lane >> st) & 1) ? -1.f : 1.f;
 
-  for (long long w = (long long)blockIdx.x * wpb + (threadIdx.x >> 5); w < total; w += stride) {
-    const int t = (int)(w / H);
-    const int h = (int)(w - (long long)t * H);
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < n_tokens; t += gridDim.x * wpb) {
     const int sid = __ldg(seq_ids + t);
     const int pos = __ldg(positions + t);
     uint32_t bad = 0;
@@ -52,83 +70,132 @@ __global__ void __launch_bounds__(256)
       if (lane == 0) set_status(status, bad);
       continue;
     }
-    uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
     const int slot = pos & (kPage - 1);
 
-    float pq[NB][8];
-#pragma unroll
-    for (int k = 0; k < NB; ++k) load_block_params(params + (size_t)h * D * 2, lane * NB + k, pq[k]);
+    for (int h = 0; h < H; ++h) {
+      uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
+      const size_t row = ((size_t)t * H + h) * D + lane * E;
+      float x[2][E];
+      load_vec<T, E>(K + row, x[0]);
+      load_vec<T, E>(V + row, x[1]);
 
-#pragma unroll
-    for (int kind = 0; kind < 2; ++kind) {
-      const T* src = (kind == 0 ? K : V) + ((size_t)t * H + h) * D + lane * E;
-      float v[E];
-      load_vec<T, E>(src, v);
-
-      float ss = 0.f;
-#pragma unroll
-      for (int i = 0; i < E; ++i) ss = fmaf(v[i], v[i], ss);
-      const float n = sqrtf(warp_sum(ss));
-
-      // y = H x (unnormalised), z = blocks(y) = sqrt(d) * (rotated unit-scale vector)
-      wht_warp<E>(v, lane);
-      float z[E];
-#pragma unroll
-      for (int k = 0; k < NB; ++k) so4_fwd(pq[k], v + 4 * k, z + 4 * k);
-
-      // code = #{j : sqrt(d) z_i >= n t_j}; zero vector -> 4
-      float nt[7];
-#pragma unroll
-      for (int j = 0; j < 7; ++j) nt[j] = n * threshold_f32(j);
-      uint32_t nib = 0;  // this lane's codes, one per nibble
+      // a1: norms (both vectors' reductions interleaved)
+      float ss[2] = {0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < E; ++i) {
-        uint32_t c = 0;
+        ss[0] = fmaf(x[0][i], x[0][i], ss[0]);
+        ss[1] = fmaf(x[1][i], x[1][i], ss[1]);
+      }
 #pragma unroll
-        for (int j = 0; j < 7; ++j) c += (z[i] >= nt[j]) ? 1u : 0u;
-        if (n == 0.f) c = 4;
-        nib |= c << (4 * i);
+      for (int o = 16; o > 0; o >>= 1) {
+        ss[0] += __shfl_xor_sync(kFull, ss[0], o);
+        ss[1] += __shfl_xor_sync(kFull, ss[1], o);
       }
+      const float n[2] = {sqrtf(ss[0]), sqrtf(ss[1])};
 
-      // Assemble the 12-byte groups.  val = direct part of word j of the lane's group for
-      // lanes that own one, N = the nibble word of the group's 8 trailing codes.
-      uint32_t val;
-      uint32_t word;
-      if constexpr (E == 4) {
-        const int r = lane & 7;
-        uint32_t half = nib << (16 * (r & 1));
-        val = half | __shfl_xor_sync(kFull, half, 1);         // lanes 2j,2j+1: w_j; 6,7: N
-        const uint32_t N = __shfl_sync(kFull, val, (lane & ~7) | 6);
-        const int j = r >> 1;                                   // valid for r in {0,2,4}
-        word = val | (((N >> (2 - (j < 3 ? j : 0))) & 0x11111111u) << 3);
-      } else {
-        const int r = lane & 3;
-        val = nib;                                              // lanes r<3: w_r; r=3: N
-        const uint32_t N = __shfl_sync(kFull, val, (lane & ~3) | 3);
-        const int j = r;
-        word = val | (((N >> (2 - (j < 3 ? j : 0))) & 0x11111111u) << 3);
-      }
-      // record word m lives on lane src(m); gather 4 words per storing lane
-      uint32_t q4[4];
+      // a2: unnormalised WHT, natural order; lane-local stages then 5 shuffle stages
 #pragma unroll
-      for (int r4 = 0; r4 < 4; ++r4) {
-        const int m = (4 * lane + r4) % (CB / 4);
-        const int src_lane = (E == 4) ? (8 * (m / 3) + 2 * (m % 3)) : (4 * (m / 3) + (m % 3));
-        q4[r4] = __shfl_sync(kFull, word, src_lane);
-      }
-      uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D)) + slot * CB;
-      if (lane < CB / 16)
-        *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
-
-      if (lane == 0) {
-        __half hn = __float2half_rn(n);
-        uint16_t nb = __half_as_ushort(hn);
-        if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
-          nb = 0x7bffu;
-          set_status(status, ISOQ_ST_NORM_SAT);
+      for (int hs = 1; hs < E; hs <<= 1) {
+#pragma unroll
+        for (int i = 0; i < E; i += 2 * hs) {
+#pragma unroll
+          for (int j = i; j < i + hs; ++j) {
+#pragma unroll
+            for (int kv = 0; kv < 2; ++kv) {
+              const float a = x[kv][j], b = x[kv][j + hs];
+              x[kv][j] = a + b;
+              x[kv][j + hs] = a - b;
+            }
+          }
         }
-        *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D) : v_norm_off(D)) +
-                                     2 * slot) = nb;
+      }
+#pragma unroll
+      for (int st = 0; st < 5; ++st) {
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv) {
+            const float pv = __shfl_xor_sync(kFull, x[kv][j], 1 << st);
+            x[kv][j] = fmaf(bsign[st], x[kv][j], pv);
+          }
+        }
+      }
+
+      // a3: SO(4) blocks as 4x4 matrices (z = M y), this lane's blocks of head h
+      float z[2][E];
+#pragma unroll
+      for (int k = 0; k < NB; ++k) {
+        const float4* mp = reinterpret_cast<const float4*>(mats + ((size_t)h * (D / 4) + lane * NB + k) * 16);
+        float M[16];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float4 v = __ldg(mp + r);
+          M[4 * r + 0] = v.x;
+          M[4 * r + 1] = v.y;
+          M[4 * r + 2] = v.z;
+          M[4 * r + 3] = v.w;
+        }
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          const float* y = x[kv] + 4 * k;
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            z[kv][4 * k + r] =
+                fmaf(M[4 * r + 3], y[3], fmaf(M[4 * r + 2], y[2], fmaf(M[4 * r + 1], y[1], M[4 * r] * y[0])));
+        }
+      }
+
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        // a4: codes against n * tau (a zero vector codes 4 everywhere)
+        uint32_t tb[3];
+#pragma unroll
+        for (int k = 0; k < 3; ++k) tb[k] = __float_as_uint(n[kv] * threshold_f32(4 + k));
+        uint32_t nib = 0;  // this lane's codes, one per nibble
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const uint32_t c = n[kv] == 0.f ? 4u : code_of(z[kv][i], tb);
+          nib |= c << (4 * i);
+        }
+
+        // a5: assemble the 12-byte groups.  val = direct part of word j of the lane's group
+        // for lanes that own one, N = the nibble word of the group's 8 trailing codes.
+        uint32_t val, word;
+        if constexpr (E == 4) {
+          const int r = lane & 7;
+          const uint32_t half = nib << (16 * (r & 1));
+          val = half | __shfl_xor_sync(kFull, half, 1);         // lanes 2j,2j+1: w_j; 6,7: N
+          const uint32_t N = __shfl_sync(kFull, val, (lane & ~7) | 6);
+          const int j = r >> 1;                                   // valid for r in {0,2,4}
+          word = val | (((N >> (2 - (j < 3 ? j : 0))) & 0x11111111u) << 3);
+        } else {
+          const int r = lane & 3;
+          val = nib;                                              // lanes r<3: w_r; r=3: N
+          const uint32_t N = __shfl_sync(kFull, val, (lane & ~3) | 3);
+          const int j = r;
+          word = val | (((N >> (2 - (j < 3 ? j : 0))) & 0x11111111u) << 3);
+        }
+        // record word m lives on lane src(m); gather 4 words per storing lane
+        uint32_t q4[4];
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const int m = (4 * lane + r4) % (CB / 4);
+          const int src_lane = (E == 4) ? (8 * (m / 3) + 2 * (m % 3)) : (4 * (m / 3) + (m % 3));
+          q4[r4] = __shfl_sync(kFull, word, src_lane);
+        }
+        uint8_t* dst = blk + (kv == 0 ? 0 : v_codes_off(D)) + slot * CB;
+        if (lane < CB / 16)
+          *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+
+        if (lane == 0) {
+          uint16_t nb = __half_as_ushort(__float2half_rn(n[kv]));
+          if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
+            nb = 0x7bffu;
+            set_status(status, ISOQ_ST_NORM_SAT);
+          }
+          *reinterpret_cast<uint16_t*>(blk + (kv == 0 ? k_norm_off(D) : v_norm_off(D)) +
+                                       2 * slot) = nb;
+        }
       }
     }
   }
@@ -136,14 +203,14 @@ __global__ void __launch_bounds__(256)
 
 template <int D, typename T>
 static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
-  const long long warps = (long long)a.n_tokens * a.n_kv_heads;
+  const long long warps = a.n_tokens;  // one warp per token
   const int wpb = 8;
   long long grid = (warps + wpb - 1) / wpb;
-  const long long cap = (long long)n_sm * 32;
+  const long long cap = (long long)n_sm * 16;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   quantize_append_kernel<D, T><<<(unsigned)grid, wpb * 32, 0, stream>>>(
-      a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_seqs, a.n_kv_heads,
+      a.mats, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_seqs, a.n_kv_heads,
       static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.n_tokens, a.seq_ids, a.positions,
       a.status);
   return cudaGetLastError();

@@ -57,6 +57,25 @@ def _dist_env():
     return rank, world, local
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (the slowest rank's time).  One all-reduce
+    of a single float after timing; nothing on the data path."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(units_per_step_per_rank: float, steps: int, world: int,
+                      max_ms: float) -> float:
+    """Whole-job rate: every rank processes the same work per step (weak scaling), so the
+    job's throughput is all ranks' units divided by the slowest rank's time."""
+    return units_per_step_per_rank * steps * world / (max_ms / 1e3)
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -256,12 +275,8 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     stream = torch.cuda.current_stream(dev)
     params = iq.isoq_make_params(wl.PARAM_SEED, cfg.d, cfg.n_kv_heads)
@@ -326,13 +341,13 @@ def run_ours(args, cfg):
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    q_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b, _, _ in evs))
-    d_ms = max_over_ranks(sum(c.elapsed_time(d) for _, _, c, d in evs))
+    total_ms = rank_max(t_start.elapsed_time(t_end))
+    q_ms = rank_max(sum(a.elapsed_time(b) for a, b, _, _ in evs))
+    d_ms = rank_max(sum(c.elapsed_time(d) for _, _, c, d in evs))
     dec_launch_ms = d_ms / args.steps
 
-    value = packed * args.steps * world / (d_ms / 1e3) / 1e9
-    qval = n_vec * args.steps * world / (q_ms / 1e3) / 1e6
+    value = weak_scaling_rate(packed, args.steps, world, d_ms) / 1e9
+    qval = weak_scaling_rate(n_vec, args.steps, world, q_ms) / 1e6
     peak, peak_kind = _peaks()
     dec_gbs_1 = packed / (dec_launch_ms / 1e3) / 1e9
     q_bytes = n_vec * (cfg.d * (4 if cfg.in_dtype == torch.float32 else 2) + 3 * cfg.d // 8 + 2)
@@ -372,8 +387,9 @@ def run_ours(args, cfg):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = max_over_ranks(a.elapsed_time(b))
-        e2e = {"value": packed * args.e2e_steps * world / (e_ms / 1e3) / 1e9, "unit": "GB/s",
+        e_ms = rank_max(a.elapsed_time(b))
+        e2e = {"value": weak_scaling_rate(packed, args.e2e_steps, world, e_ms) / 1e9,
+               "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
                "what": "packed-KV bytes decoded per step / step time with the step's K, V and "

@@ -93,15 +93,17 @@ struct SplitPlan {
 
 // Context chunking for the decode kernel: about ISOQ_DEC_WAVES waves of (chunk, KV head,
 // query-head block, sequence) CTAs at the kernel's resident CTAs per SM, each chunk a whole
-// number of pages and at least 16 pages (4 per warp) when the context allows.
+// number of pages and at least min_pages pages when the context allows.
 SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len) {
-  const int n_sm = sm_count() * isoq::decode_resident_ctas(d);
+  const bool tc = isoq::kUseTc128 && d == 128;
+  const int n_sm = sm_count() * (tc ? isoq::decode_tc_resident_ctas() : isoq::decode_resident_ctas(d));
+  const int min_pages = tc ? 8 : 16;  // per CTA: 4 tiles of 2 pages, or 4 pages per warp
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const int group = n_kv_heads > 0 ? n_q_heads / n_kv_heads : 1;
   const long long units = (long long)n_seqs * n_kv_heads * ((group + 7) / 8);
   const long long target = (long long)n_sm * ISOQ_DEC_WAVES;
   long long want = units > 0 ? (target + units - 1) / units : 1;
-  const long long cap = (max_pages + 15) / 16;
+  const long long cap = (max_pages + min_pages - 1) / min_pages;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   int pps = (int)((max_pages + want - 1) / want);

@@ -323,7 +323,8 @@ static cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
 
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
-  cudaError_t e = launch_decode_split_mma(a, stream);
+  cudaError_t e = (kUseTc128 && D == 128) ? launch_decode_split_tc(a, stream)
+                                           : launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_q_heads, a.n_seqs);
   decode_combine_kernel<D><<<grid, 128, 0, stream>>>(a.params, a.n_kv_heads, a.n_q_heads,

@@ -25,169 +25,11 @@
 
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
+#include "isoq_ptx.cuh"
 
 namespace isoq {
-namespace {
+using namespace ptx;
 
-constexpr float kAlpha = 3618.98939633f;  // level scale with near-exact binary16 levels
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLazy = 8.0f;          // rescale the running max only when it grows by 2^8
-constexpr float kSigmaSlack = 16.0f;   // ... and the V-norm reference when it grows 16x
-constexpr int kWarps = 4;
-constexpr unsigned kWaitLimit = 1u << 24;  // bounded mbarrier polls (~seconds)
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
-// 2^x with the hardware approximation (relative error ~2^-22; -inf -> 0).
-__device__ __forceinline__ float ex2(float x) {
-  float r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
-  uint32_t r;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
-  return r;
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Polls the phase with the given parity; false if it did not complete within the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
-  const uint32_t a = smem_u32(bar);
-  for (unsigned i = 0; i < kWaitLimit; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void bulk_copy(void* dst, const void* src, unsigned bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Right shifts done as the high half of a multiplication by 2^(32-k).  `mul` comes from a
-// kernel argument (2^16), so the compiler cannot fold it back into a shift: the product
-// runs on the FMA pipe and leaves the ALU pipe, which the byte permutes saturate, free.
-struct Shifter {
-  uint32_t m16, m29, m30, m31;
-  __device__ __forceinline__ explicit Shifter(uint32_t mul16)
-      : m16(mul16), m29(mul16 << 13), m30(mul16 << 14), m31(mul16 << 15) {}
-  __device__ __forceinline__ uint32_t shr16(uint32_t x) const { return __umulhi(x, m16); }
-  // spare codes: bit (2-b) of code 24+k is bit 4k+3 of w_b -> nibble k
-  __device__ __forceinline__ uint32_t spare(uint32_t w0, uint32_t w1, uint32_t w2) const {
-    uint32_t r;
-    asm("{\n .reg .u32 t;\n"
-        " mul.hi.u32 t, %1, %4;\n"
-        " mad.hi.u32 t, %2, %5, t;\n"
-        " mad.hi.u32 %0, %3, %6, t;\n}"
-        : "=r"(r)
-        : "r"(w2 & 0x88888888u), "r"(w1 & 0x88888888u), "r"(w0 & 0x88888888u), "r"(m29),
-          "r"(m30), "r"(m31));
-    return r;
-  }
-};
-
-// The three words of group q of a packed vector -> four 8-nibble selector words:
-// S[j] nibble n = code of dim 32q + 8j + n (bit 3 of every nibble clear).
-__device__ __forceinline__ void selectors(uint32_t w0, uint32_t w1, uint32_t w2, const Shifter& sh,
-                                          uint32_t (&S)[4]) {
-  S[0] = w0 & 0x77777777u;
-  S[1] = w1 & 0x77777777u;
-  S[2] = w2 & 0x77777777u;
-  S[3] = sh.spare(w0, w1, w2);
-}
-
-// Eight f16 values of the nibbles of S: o[i] = (level(nibble 2i), level(nibble 2i+1)).
-__device__ __forceinline__ void deq8(uint32_t S, uint32_t tl0, uint32_t tl1, uint32_t th0,
-                                     uint32_t th1, const Shifter& sh, uint32_t (&o)[4]) {
-  uint32_t lo = prmt(tl0, tl1, S);
-  uint32_t hi = prmt(th0, th1, S);
-  o[0] = prmt(lo, hi, 0x5140);
-  o[1] = prmt(lo, hi, 0x7362);
-  const uint32_t S2 = sh.shr16(S);
-  lo = prmt(tl0, tl1, S2);
-  hi = prmt(th0, th1, S2);
-  o[2] = prmt(lo, hi, 0x5140);
-  o[3] = prmt(lo, hi, 0x7362);
-}
-
-// Token pair (a, b), selector words Sa, Sb of the same dims: o[n] = (level a, level b) of
-// nibble n (n = 0..7), i.e. an f16x2 of two tokens for one dim.
-__device__ __forceinline__ void deq8_pair(uint32_t Sa, uint32_t Sb, uint32_t tl0, uint32_t tl1,
-                                          uint32_t th0, uint32_t th1, const Shifter& sh,
-                                          uint32_t (&o)[8]) {
-#pragma unroll
-  for (int part = 0; part < 2; ++part) {
-    // nibbles (a n, a n+1, b n, b n+1, a n+2, a n+3, b n+2, b n+3) with n = 4 part
-    const uint32_t X = prmt(Sa, Sb, part == 0 ? 0x5140u : 0x7362u);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t sel = hh == 0 ? X : sh.shr16(X);
-      const uint32_t lo = prmt(tl0, tl1, sel);
-      const uint32_t hi = prmt(th0, th1, sel);
-      o[4 * part + 2 * hh + 0] = prmt(lo, hi, 0x6240);
-      o[4 * part + 2 * hh + 1] = prmt(lo, hi, 0x7351);
-    }
-  }
-}
-
-__device__ __forceinline__ float half_at(const uint8_t* p) {
-  return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
-}
-
-}  // namespace
 
 // Dynamic shared memory: [kWarps][NST] page stages of block_bytes(D), then the mbarriers,
 // then the rotated queries (fp32 [8][D]).  The stage area is reused for the final merge.

@@ -47,6 +47,17 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
 // Resident CTAs per SM of that kernel for head dimension d on the current device.
 int decode_resident_ctas(int d);
+// Tensor-memory (tcgen05) split kernel, head dimension 128 (partials only).
+cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t stream);
+int decode_tc_resident_ctas();
+
+// The decode uses the mma.sync kernel; building with ISOQ_DECODE_TC selects the tcgen05
+// kernel for d = 128 instead (parity-equivalent, measured slower: see the design notes).
+#ifdef ISOQ_DECODE_TC
+constexpr bool kUseTc128 = true;
+#else
+constexpr bool kUseTc128 = false;
+#endif
 
 // Accessors of the opaque parameter handle (defined in isoq_api.cu).
 const float* params_device_ptr(const struct ::isoq_params* p);

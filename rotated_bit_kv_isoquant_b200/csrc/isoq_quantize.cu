@@ -201,6 +201,135 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Thread-per-vector variant for d = 128: thread i of a warp quantises token t0+i of one
+// (KV head, K|V) pair.  The whole vector lives in the thread's registers, so the WHT needs
+// no shuffles and every per-vector cost (addressing, validation, norm, packing) is paid
+// once per 128 elements instead of once per 4.  A warp's 32 vectors share the head, so the
+// 4x4 block matrices are read as warp-uniform (broadcast) 16-byte loads from shared memory.
+constexpr int kTpvThreads = 128;
+#ifndef ISOQ_TPV_MINB
+#define ISOQ_TPV_MINB 3
+#endif
+
+template <typename T>
+__global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
+    quantize_tpv_kernel(const float* __restrict__ mats, uint8_t* __restrict__ blocks,
+                        const int32_t* __restrict__ page_table, int n_pages, int max_pages,
+                        int n_seqs, int H, const T* __restrict__ K, const T* __restrict__ V,
+                        int n_tokens, const int32_t* __restrict__ seq_ids,
+                        const int32_t* __restrict__ positions, uint32_t* status) {
+  constexpr int D = 128, CB = code_bytes(D), BB = block_bytes(D);
+  extern __shared__ __align__(16) float smats[];  // [H][32 blocks][16]
+  for (int i = threadIdx.x; i < H * (D / 4) * 16 / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(smats)[i] = __ldg(reinterpret_cast<const float4*>(mats) + i);
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int chunks = (n_tokens + 31) >> 5;
+  const int n_tasks = H * 2 * chunks;  // task = (32-token chunk, head, kind), chunk-major
+  for (int task = blockIdx.x * wpb + (threadIdx.x >> 5); task < n_tasks;
+       task += gridDim.x * wpb) {
+    const int chunk = task / (2 * H);
+    const int r = task - chunk * 2 * H;
+    const int h = r >> 1, kind = r & 1;
+    const int t = chunk * 32 + lane;
+    if (t >= n_tokens) continue;
+    const int sid = __ldg(seq_ids + t);
+    const int pos = __ldg(positions + t);
+    uint32_t bad = 0;
+    int phys = -1;
+    if (sid < 0 || sid >= n_seqs) {
+      bad = ISOQ_ST_SEQ_RANGE;
+    } else if (pos < 0 || (pos >> 6) >= max_pages) {
+      bad = ISOQ_ST_POS_RANGE;
+    } else {
+      phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
+      if (phys < 0 || phys >= n_pages) bad = ISOQ_ST_PAGE_RANGE;
+    }
+    if (bad) {
+      set_status(status, bad);
+      continue;
+    }
+
+    // load the vector (contiguous D elements)
+    float x[D];
+    const T* src = (kind == 0 ? K : V) + ((size_t)t * H + h) * D;
+#pragma unroll
+    for (int i = 0; i < D; i += 8) load_vec<T, 8>(src + i, *reinterpret_cast<float(*)[8]>(x + i));
+
+    // a1: norm (four partial sums)
+    float ss0 = 0.f, ss1 = 0.f, ss2 = 0.f, ss3 = 0.f;
+#pragma unroll
+    for (int i = 0; i < D; i += 4) {
+      ss0 = fmaf(x[i], x[i], ss0);
+      ss1 = fmaf(x[i + 1], x[i + 1], ss1);
+      ss2 = fmaf(x[i + 2], x[i + 2], ss2);
+      ss3 = fmaf(x[i + 3], x[i + 3], ss3);
+    }
+    const float n = sqrtf((ss0 + ss1) + (ss2 + ss3));
+
+    // a2: unnormalised WHT, natural order, all 7 butterfly stages in registers
+#pragma unroll
+    for (int hs = 1; hs < D; hs <<= 1) {
+#pragma unroll
+      for (int i = 0; i < D; i += 2 * hs) {
+#pragma unroll
+        for (int j = i; j < i + hs; ++j) {
+          const float a = x[j], b = x[j + hs];
+          x[j] = a + b;
+          x[j + hs] = a - b;
+        }
+      }
+    }
+
+    // a3 + a4: SO(4) block (matrix from shared memory) and codes, block by block
+    uint32_t tb[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) tb[k] = __float_as_uint(n * threshold_f32(4 + k));
+    const float4* mh = reinterpret_cast<const float4*>(smats) + (size_t)h * (D / 4) * 4;
+    uint32_t nib[D / 8];  // nibble words: word j holds dims 8j..8j+7
+#pragma unroll
+    for (int b = 0; b < D / 4; ++b) {
+      float z[4];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const float4 m = mh[4 * b + rr];
+        z[rr] = fmaf(m.w, x[4 * b + 3], fmaf(m.z, x[4 * b + 2], fmaf(m.y, x[4 * b + 1], m.x * x[4 * b])));
+      }
+      uint32_t w = (b & 1) ? nib[b >> 1] : 0u;
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const uint32_t c = n == 0.f ? 4u : code_of(z[rr], tb);
+        w |= c << (4 * (4 * (b & 1) + rr));
+      }
+      nib[b >> 1] = w;
+    }
+
+    // a5: pack: per 32-dim group, words 0..2 = nibble words + bit 3 from the trailing 8 codes
+    uint32_t rec[CB / 4];
+#pragma unroll
+    for (int g = 0; g < D / 32; ++g) {
+      const uint32_t N3 = nib[4 * g + 3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j)
+        rec[3 * g + j] = nib[4 * g + j] | (((N3 >> (2 - j)) & 0x11111111u) << 3);
+    }
+    uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
+    const int slot = pos & (kPage - 1);
+    uint4* dst = reinterpret_cast<uint4*>(blk + (kind == 0 ? 0 : v_codes_off(D)) + slot * CB);
+#pragma unroll
+    for (int q = 0; q < CB / 16; ++q)
+      dst[q] = make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
+    uint16_t nb = __half_as_ushort(__float2half_rn(n));
+    if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
+      nb = 0x7bffu;
+      set_status(status, ISOQ_ST_NORM_SAT);
+    }
+    *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D) : v_norm_off(D)) + 2 * slot) = nb;
+  }
+}
+
 template <int D, typename T>
 static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   const long long warps = a.n_tokens;  // one warp per token
@@ -216,8 +345,37 @@ static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm
   return cudaGetLastError();
 }
 
+template <typename T>
+static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  const size_t smem = (size_t)a.n_kv_heads * 32 * 16 * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const long long tasks = (long long)a.n_kv_heads * 2 * ((a.n_tokens + 31) / 32);
+  const int wpb = kTpvThreads / 32;
+  long long grid = (tasks + wpb - 1) / wpb;
+  const long long cap = (long long)n_sm * 3 * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  quantize_tpv_kernel<T><<<(unsigned)grid, kTpvThreads, smem, stream>>>(
+      a.mats, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_seqs, a.n_kv_heads,
+      static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.n_tokens, a.seq_ids, a.positions,
+      a.status);
+  return cudaGetLastError();
+}
+
 template <int D>
 static cudaError_t launch_d(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  if constexpr (D == 128) {
+    switch (a.dtype) {
+      case ISOQ_F32: return launch_tpv<float>(a, stream, n_sm);
+      case ISOQ_BF16: return launch_tpv<__nv_bfloat16>(a, stream, n_sm);
+      case ISOQ_F16: return launch_tpv<__half>(a, stream, n_sm);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (a.dtype) {
     case ISOQ_F32: return launch_t<D, float>(a, stream, n_sm);
     case ISOQ_BF16: return launch_t<D, __nv_bfloat16>(a, stream, n_sm);

@@ -47,8 +47,12 @@ struct MmaSmem {
   static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
 };
 
+#ifndef ISOQ_DEC_MINB
+#define ISOQ_DEC_MINB 4  // <= 128 registers: 4 CTAs (16 warps) per SM
+#endif
+
 template <int D, int NST, typename TQ>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
     decode_mma_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
                       const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                       const TQ* __restrict__ Q, int n_q_heads, const int32_t* __restrict__ seq_lens,

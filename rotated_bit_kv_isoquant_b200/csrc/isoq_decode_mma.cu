@@ -8,13 +8,15 @@
 //
 // Work: one CTA of 4 warps per (context chunk, KV head, block of <= 8 query heads,
 // sequence).  Each warp streams its own pages of the chunk through a private ring of
-// shared-memory stages filled by 1-D bulk copies (cp.async.bulk, one 6400-byte page block
-// per copy, completion on an mbarrier; every wait is bounded).  Per 16-token tile:
-//   scores  S[16 tok x 8 heads] = K_hat[16 x d] . Q~^T   (mma.sync m16n8k16, f16 -> f32;
-//                                                          Q~ as f16 hi + lo parts)
-//   online softmax per head (max by 3 shuffles, lazily rescaled), P' = p * nV / sigma
-//   out^T[d x 8 heads] += V_hat^T[d x 16 tok] . P'^T     (mma.sync, P' transposed in
-//                                                          registers with movmatrix)
+// shared-memory stages filled by 1-D bulk copies (cp.async.bulk, one page block per copy,
+// completion on an mbarrier; every wait is bounded).  Per 32-token tile:
+//   scores  S[16 x 8 tok] = Q~2[16 x d] . K_hat^T[d x 8 tok]  (mma.sync m16n8k16, f16 ->
+//           f32, 4 tiles of 8 tokens; rows 0-7 of Q~2 are the heads' f16 high parts,
+//           rows 8-15 the low parts, so one mma carries both and their sum is the score)
+//   online softmax per head, P' = p * nV / sigma, rescaled only when a running maximum
+//           grows (lazy), so the common tile needs no shuffles
+//   out^T[d x 8 heads] += V_hat^T[d x 16 tok] . P'^T  (mma.sync; the score accumulator of
+//           two 8-token tiles is already the P'^T fragment, no transpose)
 // K_hat / V_hat are never stored: each thread turns its codes into f16 mma fragments in
 // registers with byte permutes (prmt) against 8-entry tables of the levels' low and high
 // bytes.  The packed layout puts 24 of every 32 codes in nibbles (bit 3 clear), which is
@@ -22,6 +24,8 @@
 // Levels are scaled by ALPHA, a constant for which all four magnitudes round to binary16
 // with relative error < 2e-5 (1/ALPHA is folded into the score and output scales).
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
@@ -32,43 +36,43 @@ using namespace ptx;
 
 
 // Dynamic shared memory: [kWarps][NST] page stages of block_bytes(D), then the mbarriers,
-// then the rotated queries (fp32 [8][D]).  The stage area is reused for the final merge.
+// then the score mma's A fragments of the rotated queries (one uint4 per k-step and lane,
+// shared by the four warps).  The stage area is reused for the final merge.
 template <int D, int NST>
 struct MmaSmem {
   static constexpr int kStageBytes = block_bytes(D);
   static constexpr int kRing = kWarps * NST * kStageBytes;
   static constexpr int kBarOff = kRing;
-  static constexpr int kQOff = kBarOff + kWarps * NST * 8;
-  // rotated queries, row stride kQS floats: dim d of head h at h*kQS + 40*(d/32) + d%32, so
-  // the 16-byte fragment loads of a quarter warp hit distinct banks
-  static constexpr int kQS = 40 * (D / 32) + 4;
-  static constexpr int kBytes = kQOff + 8 * kQS * 4;
+  static constexpr int kAOff = kBarOff + kWarps * NST * 8;
+  static constexpr int kBytes = kAOff + (D / 16) * 32 * 16;
   static constexpr int kMergeBytes = kWarps * 8 * (D + 4) * 4;
   static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
+  static_assert(kAOff % 16 == 0, "A fragments must be 16-byte aligned");
 };
 
-#ifndef ISOQ_DEC_MINB
-#define ISOQ_DEC_MINB 4  // <= 128 registers: 4 CTAs (16 warps) per SM
-#endif
+// d = 128: <= 128 registers, 4 CTAs (16 warps) per SM; d = 256: two CTAs fill the shared
+// memory, so registers are not the limit
+template <int D>
+constexpr int dec_min_blocks() { return D == 128 ? 4 : 2; }
 
 template <int D, int NST, typename TQ>
-__global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
+__global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     decode_mma_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
                       const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                       const TQ* __restrict__ Q, int n_q_heads, const int32_t* __restrict__ seq_lens,
                       float scale, int pages_per_split, int n_splits, float* __restrict__ partials,
-                      uint32_t* status, uint32_t mul16) {
+                      uint32_t* status) {
   using SM = MmaSmem<D, NST>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
   constexpr int CB = code_bytes(D);
   constexpr int BB = block_bytes(D);
-  constexpr int KS = D / 16;          // k-steps of the score mma, m-tiles of the PV mma
-  constexpr int NG = D / 128;         // groups per thread (score side: t, t+4; PV side)
+  constexpr int KS = D / 16;          // k-steps of the score mma = m-tiles of the PV mma
+  constexpr int NG = D / 128;         // 32-dim groups per thread and token (score: t, t+4)
   constexpr int PS = D + 4;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
-  float* qs = reinterpret_cast<float*>(smem + SM::kQOff);
+  uint4* qa = reinterpret_cast<uint4*>(smem + SM::kAOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -123,7 +127,14 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
     for (int k = 0; k < NST && k < n_my; ++k) issue(k);
   int issued = min(NST, max(n_my, 0));  // warp-uniform count of copies issued
 
-  // ---- a6: rotate the CTA's queries (unnormalised WHT + SO(4)) into shared memory ------
+  // ---- a6: rotate the CTA's queries (unnormalised WHT + SO(4)) into the A fragments ----
+  // Rows 0-7 of the score mma's A are the f16 high parts of the 8 heads' rotated queries,
+  // rows 8-15 the low parts (q = hi + lo to ~2^-22 relative; one f16 rounding of q alone
+  // costs up to ~5e-3 relative error in the output when a few large scores dominate the
+  // softmax), so one mma yields both products.  k-step kb of lane (g, t) covers dims
+  // base..base+3, base = 32 (t + 4 (kb / 8)) + 4 (kb % 8):
+  //   a0 = hi(g; base, base+1)  a1 = lo(g; base, base+1)
+  //   a2 = hi(g; base+2, +3)    a3 = lo(g; base+2, +3)
   {
     const float* hp = params + (size_t)hk * D * 2;
     float pq[NB][8];
@@ -144,34 +155,23 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
 #pragma unroll
       for (int k = 0; k < NB; ++k) so4_fwd(pq[k], v + 4 * k, z + 4 * k);
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const int dd = lane * E + i;
-        qs[h * SM::kQS + 40 * (dd >> 5) + (dd & 31)] = z[i];
+      for (int k = 0; k < NB; ++k) {
+        const int base = lane * E + 4 * k;  // dims base..base+3
+        const int q = base >> 5;
+        const int kb = 8 * (q >> 2) + ((base & 31) >> 2);
+        float hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = __half2float(__float2half_rn(z[4 * k + e]));
+          lo[e] = z[4 * k + e] - hi[e];
+        }
+        qa[kb * 32 + h * 4 + (q & 3)] =
+            make_uint4(pack_f16x2(hi[0], hi[1]), pack_f16x2(lo[0], lo[1]),
+                       pack_f16x2(hi[2], hi[3]), pack_f16x2(lo[2], lo[3]));
       }
     }
   }
   __syncthreads();
-
-  // B fragments of Q~^T for the score mma: k-step kk covers dims base..base+3 of group
-  // t + 4*(kk / 8), base = 32*(t + 4*(kk/8)) + 4*(kk%8); b0 = dims (0,1), b1 = (2,3).
-  // The query is split into f16 high and low parts (q = hi + lo to ~2^-22 relative) and
-  // both are multiplied: one f16 rounding of q alone costs up to ~5e-3 relative error
-  // in the output when a few large scores dominate the softmax.
-  uint32_t qb0[KS], qb1[KS], ql0[KS], ql1[KS];
-#pragma unroll
-  for (int kk = 0; kk < KS; ++kk) {
-    const float* q = qs + g * SM::kQS + 40 * (t + 4 * (kk / 8)) + 4 * (kk % 8);
-    float hi[4], lo[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      hi[i] = __half2float(__float2half_rn(q[i]));
-      lo[i] = q[i] - hi[i];
-    }
-    qb0[kk] = pack_f16x2(hi[0], hi[1]);
-    qb1[kk] = pack_f16x2(hi[2], hi[3]);
-    ql0[kk] = pack_f16x2(lo[0], lo[1]);
-    ql1[kk] = pack_f16x2(lo[2], lo[3]);
-  }
 
   // level byte tables: tl = low bytes, th = high bytes of f16(ALPHA * L[c]), c = 0..7
   uint32_t tl0 = 0, tl1 = 0, th0 = 0, th1 = 0;
@@ -188,16 +188,17 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
     }
   }
 
-  // running state (heads 2t, 2t+1 of this thread's C columns)
-  float m2[2] = {-CUDART_INF_F, -CUDART_INF_F};  // running max of the log2 scores
-  float lsum[2] = {0.f, 0.f};                    // this thread's share of sum p
-  float sigma = 0.f;                             // V-norm reference (warp-uniform)
+  // Softmax state of head g (the score rows of this lane); the PV accumulator columns of
+  // this lane are heads 2t, 2t+1, whose rescale factors come from lanes 8t and 8t + 4.
+  float m2 = -CUDART_INF_F;  // running max of the log2 scores of head g
+  float lsum = 0.f;          // this lane's share of sum p of head g
+  float sigma = 0.f;         // V-norm reference (warp-uniform)
+  float inv_sigma = 0.f;
   float acc[KS][4];
 #pragma unroll
   for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   const float kf = scale * kLog2e / (kAlpha * (float)D);  // log2 score per (dot * nK)
 
-  const Shifter sh(mul16);
   bool timed_out = false;
   int k = 0;
   for (; k < n_my; ++k) {
@@ -212,115 +213,123 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
 
+    // a page whose 64 tokens are all valid takes the tile body without masking
+    const bool full = page_ok && tok0 + kPage <= len;
+    auto tile = [&](const int tb, auto full_c) {
+      constexpr bool FULL = decltype(full_c)::value;
+      // ---- a7: scores of 4 tiles of 8 tokens; B = K_hat^T of token tb + 8n + g ------------
+      float C[4][4];
 #pragma unroll
-    for (int tb = 0; tb < kPage; tb += 32) {
-      // ---- a7: scores for two 16-token sub-tiles; A = K_hat rows (tokens r+g, r+g+8) ----
-      // four independent accumulator chains per sub-tile (k-step parity x hi/lo part of
-      // the query) so consecutive mma instructions do not wait on each other's results
-      float sc[2][4], part[2][4][4];
+      for (int n = 0; n < 4; ++n) C[n][0] = C[n][1] = C[n][2] = C[n][3] = 0.f;
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        const int r = tb + 16 * sub;
+      for (int gq = 0; gq < NG; ++gq) {
+        uint32_t w[4][3];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) part[sub][c][0] = part[sub][c][1] = part[sub][c][2] = part[sub][c][3] = 0.f;
-#pragma unroll
-        for (int gq = 0; gq < NG; ++gq) {
-          const int q = t + 4 * gq;
-          const uint32_t* ra = reinterpret_cast<const uint32_t*>(blk + (r + g) * CB) + 3 * q;
-          const uint32_t* rb = reinterpret_cast<const uint32_t*>(blk + (r + g + 8) * CB) + 3 * q;
-          uint32_t Sa[4], Sb[4];
-          selectors(ra[0], ra[1], ra[2], sh, Sa);
-          selectors(rb[0], rb[1], rb[2], sh, Sb);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t fa[4], fb[4];
-            deq8(Sa[j], tl0, tl1, th0, th1, sh, fa);
-            deq8(Sb[j], tl0, tl1, th0, th1, sh, fb);
-            const int kk0 = 8 * gq + 2 * j;
-            mma16816(part[sub][0], fa[0], fb[0], fa[1], fb[1], qb0[kk0], qb1[kk0]);
-            mma16816(part[sub][1], fa[2], fb[2], fa[3], fb[3], qb0[kk0 + 1], qb1[kk0 + 1]);
-            mma16816(part[sub][2], fa[0], fb[0], fa[1], fb[1], ql0[kk0], ql1[kk0]);
-            mma16816(part[sub][3], fa[2], fb[2], fa[3], fb[3], ql0[kk0 + 1], ql1[kk0 + 1]);
-          }
+        for (int n = 0; n < 4; ++n) {
+          const uint32_t* p =
+              reinterpret_cast<const uint32_t*>(blk + (tb + 8 * n + g) * CB) + 3 * (t + 4 * gq);
+          w[n][0] = p[0];
+          w[n][1] = p[1];
+          w[n][2] = p[2];
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          sc[sub][i] = (part[sub][0][i] + part[sub][1][i]) + (part[sub][2][i] + part[sub][3][i]);
-      }
-      // token validity and norms of this thread's C rows: tokens tb+16sub+g (+8)
-      float s2[2][4], nv[2][2];
-      bool vd[2][2];
+        for (int j = 0; j < 4; ++j) {
+          const uint4 A0 = qa[(8 * gq + 2 * j) * 32 + lane];
+          const uint4 A1 = qa[(8 * gq + 2 * j + 1) * 32 + lane];
+          uint32_t f[4][4];
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
+          for (int n = 0; n < 4; ++n) {
+            const uint32_t S = j < 3 ? (w[n][j] & 0x77777777u) : spare_codes(w[n][0], w[n][1], w[n][2]);
+            deq8(S, tl0, tl1, th0, th1, f[n]);
+          }
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int tk = tb + 16 * sub + g + 8 * rr;
-          vd[sub][rr] = page_ok && (tok0 + tk) < len;
-          const float nk = half_at(blk + k_norm_off(D) + 2 * tk);
-          nv[sub][rr] = vd[sub][rr] ? half_at(blk + v_norm_off(D) + 2 * tk) : 0.f;
-          s2[sub][2 * rr + 0] = vd[sub][rr] ? sc[sub][2 * rr + 0] * nk * kf : -CUDART_INF_F;
-          s2[sub][2 * rr + 1] = vd[sub][rr] ? sc[sub][2 * rr + 1] * nk * kf : -CUDART_INF_F;
+          for (int n = 0; n < 4; ++n) mma16816(C[n], A0.x, A0.y, A0.z, A0.w, f[n][0], f[n][1]);
+#pragma unroll
+          for (int n = 0; n < 4; ++n) mma16816(C[n], A1.x, A1.y, A1.z, A1.w, f[n][2], f[n][3]);
         }
       }
 
-      // ---- a8: online softmax over the 32 tokens (per head: 4 values here, 3 shuffles) --
-      float tmax[2] = {fmaxf(fmaxf(s2[0][0], s2[0][2]), fmaxf(s2[1][0], s2[1][2])),
-                       fmaxf(fmaxf(s2[0][1], s2[0][3]), fmaxf(s2[1][1], s2[1][3]))};
-      float vmax = fmaxf(fmaxf(nv[0][0], nv[0][1]), fmaxf(nv[1][0], nv[1][1]));
+      // tokens of this lane: tb + 8n + 2t + e (n = 0..3, e = 0, 1).  sv = log2-domain score
+      // (-inf when masked), nv = V norm (0 when masked)
+      float sv[4][2], nv[4][2];
+      bool grow = false;
+      const float sthr = m2 + kLazy, vthr = sigma * kSigmaSlack;
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        tmax[0] = fmaxf(tmax[0], __shfl_xor_sync(kFull, tmax[0], o));
-        tmax[1] = fmaxf(tmax[1], __shfl_xor_sync(kFull, tmax[1], o));
-        vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
-      }
-      float resc[2] = {1.f, 1.f};
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        if (tmax[e] > m2[e] + kLazy) {
-          resc[e] = ex2(m2[e] - tmax[e]);  // 0 when m2 was -inf
-          lsum[e] *= resc[e];
-          m2[e] = tmax[e];
+      for (int n = 0; n < 4; ++n) {
+        const int tk = tb + 8 * n + 2 * t;
+        const float2 nk2 = __half22float2(
+            *reinterpret_cast<const __half2*>(blk + k_norm_off(D) + 2 * tk));
+        const float2 nv2 = __half22float2(
+            *reinterpret_cast<const __half2*>(blk + v_norm_off(D) + 2 * tk));
+        sv[n][0] = (C[n][0] + C[n][2]) * (nk2.x * kf);
+        sv[n][1] = (C[n][1] + C[n][3]) * (nk2.y * kf);
+        nv[n][0] = nv2.x;
+        nv[n][1] = nv2.y;
+        if constexpr (!FULL) {
+          const bool v0 = page_ok && (tok0 + tk) < len;
+          const bool v1 = page_ok && (tok0 + tk + 1) < len;
+          sv[n][0] = v0 ? sv[n][0] : -CUDART_INF_F;
+          sv[n][1] = v1 ? sv[n][1] : -CUDART_INF_F;
+          nv[n][0] = v0 ? nv[n][0] : 0.f;
+          nv[n][1] = v1 ? nv[n][1] : 0.f;
         }
+        grow |= (fmaxf(sv[n][0], sv[n][1]) > sthr) | (fmaxf(nv[n][0], nv[n][1]) > vthr);
       }
-      if (vmax > sigma * kSigmaSlack) {
-        const float rr = sigma / vmax;  // 0 on the first valid tile
-        resc[0] *= rr;
-        resc[1] *= rr;
-        sigma = vmax;
-      }
-      if (resc[0] != 1.f || resc[1] != 1.f) {
+      // ---- a8: online softmax.  The running max m2 of head g (shared by the 4 lanes t)
+      // and the V-norm reference sigma move only when a score exceeds m2 + 8 or a norm
+      // exceeds 16 sigma (first tile included), so the common tile needs no shuffles.
+      if (__any_sync(kFull, grow)) {
+        float tmax = -CUDART_INF_F, vmax = 0.f;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          tmax = fmaxf(tmax, fmaxf(sv[n][0], sv[n][1]));
+          vmax = fmaxf(vmax, fmaxf(nv[n][0], nv[n][1]));
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, o));
+          vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
+        }
+        float resc = 1.f;
+        if (tmax > sthr) {
+          resc = ex2(m2 - tmax);  // 0 when m2 was -inf
+          lsum *= resc;
+          m2 = tmax;
+        }
+        float vr = 1.f;
+        if (vmax > vthr) {   // warp-uniform
+          vr = sigma / vmax;  // 0 on the first valid tile
+          sigma = vmax;
+          inv_sigma = 1.f / vmax;
+        }
+        const float r0 = __shfl_sync(kFull, resc, 8 * t) * vr;
+        const float r1 = __shfl_sync(kFull, resc, 8 * t + 4) * vr;
 #pragma unroll
         for (int i = 0; i < KS; ++i) {
-          acc[i][0] *= resc[0];
-          acc[i][1] *= resc[1];
-          acc[i][2] *= resc[0];
-          acc[i][3] *= resc[1];
+          acc[i][0] *= r0;
+          acc[i][1] *= r1;
+          acc[i][2] *= r0;
+          acc[i][3] *= r1;
         }
       }
-      const float inv_sigma = sigma > 0.f ? 1.f / sigma : 0.f;
+      // P'^T B fragments of the PV mma: k16 block jb = tiles 2jb, 2jb+1; b0 = tile 2jb's
+      // tokens 2t, 2t+1, b1 = tile 2jb+1's, column = head g
       uint32_t pb[2][2];
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        float pw[4];
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const float p0 = vd[sub][rr] ? ex2(s2[sub][2 * rr] - m2[0]) : 0.f;
-          const float p1 = vd[sub][rr] ? ex2(s2[sub][2 * rr + 1] - m2[1]) : 0.f;
-          lsum[0] += p0;
-          lsum[1] += p1;
-          const float w = nv[sub][rr] * inv_sigma;
-          pw[2 * rr] = p0 * w;
-          pw[2 * rr + 1] = p1 * w;
+      for (int n = 0; n < 4; ++n) {
+        float p0 = ex2(sv[n][0] - m2), p1 = ex2(sv[n][1] - m2);
+        if constexpr (!FULL) {  // a masked token while m2 is still -inf: -inf - -inf
+          p0 = sv[n][0] != -CUDART_INF_F ? p0 : 0.f;
+          p1 = sv[n][1] != -CUDART_INF_F ? p1 : 0.f;
         }
-        // P'^T fragments: transpose the two 8x8 blocks (tokens 0-7, 8-15 of the sub-tile)
-        pb[sub][0] = movmatrix_t(pack_f16x2(pw[0], pw[1]));
-        pb[sub][1] = movmatrix_t(pack_f16x2(pw[2], pw[3]));
+        lsum += p0 + p1;
+        pb[n >> 1][n & 1] = pack_f16x2(p0 * (nv[n][0] * inv_sigma), p1 * (nv[n][1] * inv_sigma));
       }
 
       // ---- a8: V accumulation, A = V_hat^T (rows = dims, k = tokens 2t,2t+1,2t+8,2t+9) --
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        const int r = tb + 16 * sub;
+      for (int jb = 0; jb < 2; ++jb) {
+        const int r = tb + 16 * jb;
 #pragma unroll
         for (int gq = 0; gq < NG; ++gq) {
           const int q = (g >> 1) + 4 * gq;
@@ -333,19 +342,30 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
             const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + 3 * q;
             const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
             S[x][0] = (odd ? w2 : w0) & 0x77777777u;
-            S[x][1] = odd ? sh.spare(w0, w1, w2) : (w1 & 0x77777777u);
+            S[x][1] = odd ? spare_codes(w0, w1, w2) : (w1 & 0x77777777u);
           }
-          uint32_t f[4][8];  // [pair/word combo][nibble = m-tile]
-          deq8_pair(S[0][0], S[1][0], tl0, tl1, th0, th1, sh, f[0]);
-          deq8_pair(S[0][1], S[1][1], tl0, tl1, th0, th1, sh, f[1]);
-          deq8_pair(S[2][0], S[3][0], tl0, tl1, th0, th1, sh, f[2]);
-          deq8_pair(S[2][1], S[3][1], tl0, tl1, th0, th1, sh, f[3]);
+          // m-tile 4 ww + 2 part + hh: row g = nibble 4 part + 2 hh of word j0 + ww, row g+8
+          // = the next nibble, so each A quad is two output pairs of two lookups
 #pragma unroll
-          for (int mt = 0; mt < 8; ++mt)
-            mma16816(acc[8 * gq + mt], f[0][mt], f[1][mt], f[2][mt], f[3][mt], pb[sub][0],
-                     pb[sub][1]);
+          for (int ww = 0; ww < 2; ++ww) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+              uint32_t fa[4], fb[4];  // tokens (2t, 2t+1) and (2t+8, 2t+9)
+              deq4_pair(S[0][ww], S[1][ww], part, tl0, tl1, th0, th1, fa);
+              deq4_pair(S[2][ww], S[3][ww], part, tl0, tl1, th0, th1, fb);
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh)
+                mma16816(acc[8 * gq + 4 * ww + 2 * part + hh], fa[2 * hh], fa[2 * hh + 1],
+                         fb[2 * hh], fb[2 * hh + 1], pb[jb][0], pb[jb][1]);
+            }
+          }
         }
       }
+    };
+#pragma unroll 1
+    for (int tb = 0; tb < kPage; tb += 32) {
+      if (full) tile(tb, std::true_type{});
+      else tile(tb, std::false_type{});
     }
     __syncwarp();
     // stage st is consumed: refill it with page k + NST
@@ -367,12 +387,9 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
   }
 
   // ---- merge the 4 warps' states in shared memory, write the chunk's partials ---------
-  // reduce this thread's lsum over the 8 rows g (lanes with the same t)
+  // head g's sum p over the lanes t
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) lsum[e] += __shfl_xor_sync(kFull, lsum[e], o);
-  }
+  for (int o = 1; o < 4; o <<= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
   __syncthreads();  // all warps done with their rings
   float* mb = reinterpret_cast<float*>(smem);  // [kWarps][8 heads][D + 4]
   {
@@ -384,22 +401,19 @@ __global__ void __launch_bounds__(kWarps * 32, ISOQ_DEC_MINB)
       for (int mt = 0; mt < 8; ++mt) {
         const int q = (g >> 1) + 4 * gq;
         const int j0 = 2 * (g & 1);
-        const int d0 = 32 * q + 8 * j0 + mt;  // row g of m-tile; row g+8 is d0 + 8
+        const int d0 = 32 * q + 8 * j0 + 2 * mt;  // row g of m-tile; row g+8 is d0 + 1
         float* r0 = mb + (warp * 8 + 2 * t) * PS;
         float* r1 = mb + (warp * 8 + 2 * t + 1) * PS;
         r0[d0] = acc[8 * gq + mt][0] * f;
         r1[d0] = acc[8 * gq + mt][1] * f;
-        r0[d0 + 8] = acc[8 * gq + mt][2] * f;
-        r1[d0 + 8] = acc[8 * gq + mt][3] * f;
+        r0[d0 + 1] = acc[8 * gq + mt][2] * f;
+        r1[d0 + 1] = acc[8 * gq + mt][3] * f;
       }
     }
-    if (g == 0) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float* r = mb + (warp * 8 + 2 * t + e) * PS;
-        r[D] = m2[e];
-        r[D + 1] = lsum[e];
-      }
+    if (t == 0) {
+      float* r = mb + (warp * 8 + g) * PS;
+      r[D] = m2;
+      r[D + 1] = lsum;
     }
   }
   __syncthreads();
@@ -446,7 +460,7 @@ static cudaError_t launch_mma_t(const DecodeArgs& a, cudaStream_t stream) {
   decode_mma_kernel<D, NST, TQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.seq_lens, a.scale, a.pages_per_split,
-      a.n_splits, a.partials, a.status, 65536u);
+      a.n_splits, a.partials, a.status);
   return cudaGetLastError();
 }
 

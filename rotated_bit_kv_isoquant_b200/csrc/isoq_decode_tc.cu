@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kTcTile)
                      const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                      const TQ* __restrict__ Q, int n_q_heads, const int32_t* __restrict__ seq_lens,
                      float scale, int pages_per_split, int n_splits, float* __restrict__ partials,
-                     uint32_t* status, uint32_t mul16) {
+                     uint32_t* status) {
   constexpr int D = kTcD, E = D / 32, NB = E / 4, CB = code_bytes(D), PS = D + 4;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* ring_bar = reinterpret_cast<uint64_t*>(smem + kOffBar);   // [kTcStages]
@@ -319,7 +319,6 @@ __global__ void __launch_bounds__(kTcTile)
       th1 |= hi << (8 * (c - 4));
     }
   }
-  const Shifter sh(mul16);
   const float kf = scale * kLog2e / (kAlpha * (float)D);
   const uint32_t sQh = smem_u32(smem + kOffQh), sQl = smem_u32(smem + kOffQl);
   const uint32_t sV = smem_u32(smem + kOffV), sP = smem_u32(smem + kOffP);
@@ -355,11 +354,11 @@ __global__ void __launch_bounds__(kTcTile)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t S[4];
-        selectors(w[3 * q], w[3 * q + 1], w[3 * q + 2], sh, S);
+        selectors(w[3 * q], w[3 * q + 1], w[3 * q + 2], S);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t o[4];
-          deq8(S[j], tl0, tl1, th0, th1, sh, o);
+          deq8(S[j], tl0, tl1, th0, th1, o);
 #pragma unroll
           for (int m = 0; m < 4; ++m) a[16 * q + 4 * j + m] = o[m];
         }
@@ -395,11 +394,11 @@ __global__ void __launch_bounds__(kTcTile)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t S[4];
-        selectors(w[3 * q], w[3 * q + 1], w[3 * q + 2], sh, S);
+        selectors(w[3 * q], w[3 * q + 1], w[3 * q + 2], S);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t o[4];
-          deq8(S[j], tl0, tl1, th0, th1, sh, o);
+          deq8(S[j], tl0, tl1, th0, th1, o);
           st_shared_v4(vrow + (4 * q + j) * 128, o[0], o[1], o[2], o[3]);
         }
       }
@@ -556,7 +555,7 @@ static cudaError_t launch_tc_t(const DecodeArgs& a, cudaStream_t stream) {
   decode_tc_kernel<TQ><<<grid, kTcTile, kTcSmem, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.seq_lens, a.scale, a.pages_per_split,
-      a.n_splits, a.partials, a.status, 65536u);
+      a.n_splits, a.partials, a.status);
   return cudaGetLastError();
 }
 

@@ -35,12 +35,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
-  uint32_t r;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
-  return r;
-}
-
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -97,69 +91,49 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Right shifts done as the high half of a multiplication by 2^(32-k).  `mul` comes from a
-// kernel argument (2^16), so the compiler cannot fold it back into a shift: the product
-// runs on the FMA pipe and leaves the ALU pipe, which the byte permutes saturate, free.
-struct Shifter {
-  uint32_t m16, m29, m30, m31;
-  __device__ __forceinline__ explicit Shifter(uint32_t mul16)
-      : m16(mul16), m29(mul16 << 13), m30(mul16 << 14), m31(mul16 << 15) {}
-  __device__ __forceinline__ uint32_t shr16(uint32_t x) const { return __umulhi(x, m16); }
-  // spare codes: bit (2-b) of code 24+k is bit 4k+3 of w_b -> nibble k
-  __device__ __forceinline__ uint32_t spare(uint32_t w0, uint32_t w1, uint32_t w2) const {
-    uint32_t r;
-    asm("{\n .reg .u32 t;\n"
-        " mul.hi.u32 t, %1, %4;\n"
-        " mad.hi.u32 t, %2, %5, t;\n"
-        " mad.hi.u32 %0, %3, %6, t;\n}"
-        : "=r"(r)
-        : "r"(w2 & 0x88888888u), "r"(w1 & 0x88888888u), "r"(w0 & 0x88888888u), "r"(m29),
-          "r"(m30), "r"(m31));
-    return r;
-  }
-};
+// Spare codes of a group: bit (2-b) of code 24+k is bit 4k+3 of w_b -> nibble k.
+__device__ __forceinline__ uint32_t spare_codes(uint32_t w0, uint32_t w1, uint32_t w2) {
+  return ((w2 & 0x88888888u) >> 3) | ((w1 & 0x88888888u) >> 2) | ((w0 & 0x88888888u) >> 1);
+}
 
 // The three words of group q of a packed vector -> four 8-nibble selector words:
 // S[j] nibble n = code of dim 32q + 8j + n (bit 3 of every nibble clear).
-__device__ __forceinline__ void selectors(uint32_t w0, uint32_t w1, uint32_t w2, const Shifter& sh,
+__device__ __forceinline__ void selectors(uint32_t w0, uint32_t w1, uint32_t w2,
                                           uint32_t (&S)[4]) {
   S[0] = w0 & 0x77777777u;
   S[1] = w1 & 0x77777777u;
   S[2] = w2 & 0x77777777u;
-  S[3] = sh.spare(w0, w1, w2);
+  S[3] = spare_codes(w0, w1, w2);
 }
 
 // Eight f16 values of the nibbles of S: o[i] = (level(nibble 2i), level(nibble 2i+1)).
 __device__ __forceinline__ void deq8(uint32_t S, uint32_t tl0, uint32_t tl1, uint32_t th0,
-                                     uint32_t th1, const Shifter& sh, uint32_t (&o)[4]) {
+                                     uint32_t th1, uint32_t (&o)[4]) {
   uint32_t lo = prmt(tl0, tl1, S);
   uint32_t hi = prmt(th0, th1, S);
   o[0] = prmt(lo, hi, 0x5140);
   o[1] = prmt(lo, hi, 0x7362);
-  const uint32_t S2 = sh.shr16(S);
+  const uint32_t S2 = S >> 16;
   lo = prmt(tl0, tl1, S2);
   hi = prmt(th0, th1, S2);
   o[2] = prmt(lo, hi, 0x5140);
   o[3] = prmt(lo, hi, 0x7362);
 }
 
-// Token pair (a, b), selector words Sa, Sb of the same dims: o[n] = (level a, level b) of
-// nibble n (n = 0..7), i.e. an f16x2 of two tokens for one dim.
-__device__ __forceinline__ void deq8_pair(uint32_t Sa, uint32_t Sb, uint32_t tl0, uint32_t tl1,
-                                          uint32_t th0, uint32_t th1, const Shifter& sh,
-                                          uint32_t (&o)[8]) {
+// Token pair (a, b), selector words Sa, Sb of the same dims: o[i] = (level a, level b) of
+// nibble 4 part + i (i = 0..3), i.e. an f16x2 of two tokens for one dim.
+__device__ __forceinline__ void deq4_pair(uint32_t Sa, uint32_t Sb, int part, uint32_t tl0,
+                                          uint32_t tl1, uint32_t th0, uint32_t th1,
+                                          uint32_t (&o)[4]) {
+  // nibbles (a n, a n+1, b n, b n+1, a n+2, a n+3, b n+2, b n+3) with n = 4 part
+  const uint32_t X = prmt(Sa, Sb, part == 0 ? 0x5140u : 0x7362u);
 #pragma unroll
-  for (int part = 0; part < 2; ++part) {
-    // nibbles (a n, a n+1, b n, b n+1, a n+2, a n+3, b n+2, b n+3) with n = 4 part
-    const uint32_t X = prmt(Sa, Sb, part == 0 ? 0x5140u : 0x7362u);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t sel = hh == 0 ? X : sh.shr16(X);
-      const uint32_t lo = prmt(tl0, tl1, sel);
-      const uint32_t hi = prmt(th0, th1, sel);
-      o[4 * part + 2 * hh + 0] = prmt(lo, hi, 0x6240);
-      o[4 * part + 2 * hh + 1] = prmt(lo, hi, 0x7351);
-    }
+  for (int hh = 0; hh < 2; ++hh) {
+    const uint32_t sel = hh == 0 ? X : X >> 16;
+    const uint32_t lo = prmt(tl0, tl1, sel);
+    const uint32_t hi = prmt(th0, th1, sel);
+    o[2 * hh + 0] = prmt(lo, hi, 0x6240);
+    o[2 * hh + 1] = prmt(lo, hi, 0x7351);
   }
 }
 

@@ -225,6 +225,42 @@ int isoq_decode_attention_noalloc(const isoq_params* params, const isoq_cache* c
  * device; >= 1, or a negative error code. */
 int isoq_decode_num_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len);
 
+/* =======================================================================================
+ * Context-parallel decode: one sequence's context spread over several ranks (GPUs).
+ *
+ * Softmax attention over a union of disjoint token sets is the log-sum-exp merge of the
+ * per-set states, exactly as the split chunks above are merged (the same split-K rule,
+ * "FreeToken releases", v0.2.0, Kernels), so a rank that holds a slice of every
+ * sequence's context computes the state of its slice, the ranks exchange the states
+ * (a few hundred bytes per (sequence, query head)), and each finishes the merge.  Which
+ * tokens a rank holds is the caller's choice; positions only matter to RoPE, which is
+ * part of the cached K, so each rank's cache stores its slice at local positions 0..n-1.
+ *
+ * State layout (fp32, per (sequence, query head), d + 4 floats): acc[d], m, l, 0, 0 with
+ *   m = max over the slice of the score in natural-log units (-inf for an empty slice),
+ *   l = sum_t exp(s_t - m),  acc = sqrt(d) * sum_t exp(s_t - m) v~_t  (rotated space).
+ *
+ * isoq_decode_partial_state: as isoq_decode_attention over this rank's cache (same
+ *   arguments and errors), writing the state of each (sequence, query head) to `state`:
+ *   device fp32 [n_seqs][n_q_heads][d + 4], 16-byte aligned, isoq_decode_state_bytes()
+ *   bytes.
+ * isoq_decode_merge_states: states = device fp32 [n_states][n_seqs][n_q_heads][d + 4]
+ *   (what an all-gather of the ranks' `state` buffers produces, in any rank order),
+ *   16-byte aligned; writes out = device fp32 [n_seqs][n_q_heads][d], the attention over
+ *   the union of the slices (zeros where every slice is empty).  params gives d, the KV
+ *   head count and the inverse rotation.  Errors: ISOQ_E_ARG, ISOQ_E_GQA, ISOQ_E_DEVICE,
+ *   ISOQ_E_CUDA.
+ * ===================================================================================== */
+size_t isoq_decode_state_bytes(int n_seqs, int n_q_heads, int d);
+
+int isoq_decode_partial_state(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                              int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                              int max_seq_len, float* state, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+int isoq_decode_merge_states(const isoq_params* params, const float* states, int n_states,
+                             int n_seqs, int n_q_heads, float* out, void* stream);
+
 /* ---- status and errors ------------------------------------------------------------------ */
 /* Synchronises the device and copies the status word to *host_bits (0 if status is NULL). */
 int isoq_get_status(const isoq_cache* cache, uint32_t* host_bits);

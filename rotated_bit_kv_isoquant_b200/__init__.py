@@ -75,6 +75,9 @@ _SIGS = {
     "isoq_decode_num_splits": (_i, [_i, _i, _i, _i, _i]),
     "isoq_decode_attention": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
     "isoq_decode_attention_noalloc": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p]),
+    "isoq_decode_state_bytes": (_sz, [_i, _i, _i]),
+    "isoq_decode_partial_state": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
+    "isoq_decode_merge_states": (_i, [_p, _p, _i, _i, _i, _p, _p]),
     "isoq_get_status": (_i, [_cp, ctypes.POINTER(ctypes.c_uint32)]),
     "isoq_reset_status": (_i, [_cp, _p]),
     "isoq_last_cuda_error": (_i, []),
@@ -247,6 +250,35 @@ def isoq_decode_attention_noalloc(params: Params, cache: PagedCache, Q, seq_lens
         Q.shape[1], _dev_ptr(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
         _dev_ptr(out, "out", torch.float32), float(scale), _stream_ptr(stream)),
         "isoq_decode_attention_noalloc")
+
+
+def isoq_decode_state_bytes(n_seqs, n_q_heads, d) -> int:
+    return int(_lib.isoq_decode_state_bytes(n_seqs, n_q_heads, d))
+
+
+def isoq_decode_partial_state(params: Params, cache: PagedCache, Q, seq_lens, max_seq_len: int,
+                              state, scale: float, workspace, stream=None) -> None:
+    """Softmax state of this cache's slice of every context: state fp32 CUDA
+    [n_seqs][n_q_heads][d + 4] = (acc[d], m, l, 0, 0); other arguments as
+    isoq_decode_attention."""
+    import torch
+    n_seqs, n_q_heads = Q.shape[0], Q.shape[1]
+    _check(_lib.isoq_decode_partial_state(
+        params.handle, ctypes.byref(cache.c), _dev_ptr(Q, "Q"), _dtype_code(Q), n_seqs, n_q_heads,
+        _dev_ptr(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
+        _dev_ptr(state, "state", torch.float32), float(scale), _dev_ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+        "isoq_decode_partial_state")
+
+
+def isoq_decode_merge_states(params: Params, states, out, stream=None) -> None:
+    """states: fp32 CUDA [n_states][n_seqs][n_q_heads][d + 4] (gathered slice states);
+    out: fp32 CUDA [n_seqs][n_q_heads][d], attention over the union of the slices."""
+    import torch
+    n_states, n_seqs, n_q_heads = states.shape[0], states.shape[1], states.shape[2]
+    _check(_lib.isoq_decode_merge_states(
+        params.handle, _dev_ptr(states, "states", torch.float32), n_states, n_seqs, n_q_heads,
+        _dev_ptr(out, "out", torch.float32), _stream_ptr(stream)), "isoq_decode_merge_states")
 
 
 def isoq_get_status(cache: PagedCache) -> int:

@@ -279,10 +279,16 @@ size_t isoq_decode_workspace_bytes(int n_seqs, int n_q_heads, int n_kv_heads, in
   return (size_t)n_seqs * n_q_heads * ns * isoq::partial_stride(d) * sizeof(float);
 }
 
-int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, const void* Q,
-                          int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
-                          int max_seq_len, float* out, float scale, void* workspace,
-                          size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by the decode entry points: validation, the split plan, then the split kernel and
+// the combine into either the output rows (out) or merged states (state).
+int decode_common(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                  int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                  int max_seq_len, float* out, float* state, float scale, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   int rc = check_cache(cache, params);
   if (rc) return rc;
   if (n_seqs < 0 || n_q_heads < 0 || max_seq_len < 0 || !valid_dtype(q_dtype)) return ISOQ_E_ARG;
@@ -290,14 +296,15 @@ int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, co
   if (n_q_heads % cache->n_kv_heads || n_q_heads / cache->n_kv_heads > 16) return ISOQ_E_GQA;
   if (n_seqs > cache->n_seqs) return ISOQ_E_ARG;
   if (n_seqs == 0 || n_q_heads == 0) return ISOQ_OK;
-  if (!Q || !seq_lens || !out || !workspace) return ISOQ_E_ARG;
+  if (!Q || !seq_lens || !(out || state) || !workspace) return ISOQ_E_ARG;
+  if (state && ((uintptr_t)state & 15u) != 0) return ISOQ_E_ARG;
   if (((uintptr_t)workspace & 15u) != 0) return ISOQ_E_WORKSPACE;
   const size_t need =
       isoq_decode_workspace_bytes(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
   if (workspace_bytes < need) return ISOQ_E_WORKSPACE;
   if ((rc = check_device(params))) return rc;
   const SplitPlan plan = plan_splits(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
-  isoq::DecodeArgs a;
+  isoq::DecodeArgs a{};
   a.params = params->dev;
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;
@@ -315,8 +322,49 @@ int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, co
   a.pages_per_split = plan.pages_per_split;
   a.partials = static_cast<float*>(workspace);
   a.out = out;
+  a.state = state;
   a.status = cache->status;
   cudaError_t e = isoq::launch_decode(a, (cudaStream_t)stream);
+  return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                          int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                          int max_seq_len, float* out, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  return decode_common(params, cache, Q, q_dtype, n_seqs, n_q_heads, seq_lens, max_seq_len,
+                       out, nullptr, scale, workspace, workspace_bytes, stream);
+}
+
+size_t isoq_decode_state_bytes(int n_seqs, int n_q_heads, int d) {
+  if (n_seqs < 0 || n_q_heads < 0 || !supported_d(d)) return 0;
+  return (size_t)n_seqs * n_q_heads * isoq::partial_stride(d) * sizeof(float);
+}
+
+int isoq_decode_partial_state(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                              int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                              int max_seq_len, float* state, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!state) return ISOQ_E_ARG;
+  return decode_common(params, cache, Q, q_dtype, n_seqs, n_q_heads, seq_lens, max_seq_len,
+                       nullptr, state, scale, workspace, workspace_bytes, stream);
+}
+
+int isoq_decode_merge_states(const isoq_params* params, const float* states, int n_states,
+                             int n_seqs, int n_q_heads, float* out, void* stream) {
+  if (!params || n_states < 1 || n_seqs < 0 || n_q_heads < 0) return ISOQ_E_ARG;
+  if (n_q_heads % params->n_kv_heads || n_q_heads / params->n_kv_heads > 16) return ISOQ_E_GQA;
+  if (n_seqs == 0 || n_q_heads == 0) return ISOQ_OK;
+  if (!states || !out || ((uintptr_t)states & 15u) != 0) return ISOQ_E_ARG;
+  int rc = check_device(params);
+  if (rc) return rc;
+  cudaError_t e = isoq::launch_merge_states(params->dev, params->n_kv_heads, params->d, n_seqs,
+                                            n_q_heads, n_states, states, out,
+                                            (cudaStream_t)stream);
   return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
 }
 

@@ -37,12 +37,17 @@ struct DecodeArgs {
   int n_splits;         // context chunks per (sequence, KV head)
   int pages_per_split;  // pages in each chunk
   float* partials;      // [n_seqs][n_q_heads][n_splits][d + 4]
-  float* out;
+  float* out;           // [n_seqs][n_q_heads][d] (when state is null)
+  float* state;         // if set: merged state [n_seqs][n_q_heads][d + 4] instead of out
   uint32_t* status;
 };
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// Merge of context-slice states [n_states][n_seqs][n_q_heads][d + 4] into the output.
+cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int n_seqs,
+                                int n_q_heads, int n_states, const float* states, float* out,
+                                cudaStream_t stream);
 // Tensor-core split kernel (partials only); the combine runs separately.
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
 // Resident CTAs per SM of that kernel for head dimension d on the current device.

@@ -101,7 +101,7 @@ extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const is
   float* scratch = scratch_address(dev, &e);
   if (!scratch) return isoq::record_cuda_error(e);
 
-  isoq::DecodeArgs a;
+  isoq::DecodeArgs a{};
   a.params = isoq::params_device_ptr(params);
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;

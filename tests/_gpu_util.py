@@ -2,7 +2,9 @@
 fp64 oracle (which only ever sees host copies of the same seeded inputs)."""
 from __future__ import annotations
 
+import json
 import math
+import os
 
 import numpy as np
 import torch
@@ -12,6 +14,15 @@ import workloads as wl
 
 BAND = 1e-6          # codes may differ only where u is this close to a threshold (N(0,1) units)
 ATTN_TOL = 2e-3      # relative L2 error per (sequence, query head) vs the oracle on the same codes
+
+
+def log_record(record: dict) -> None:
+    """Print a parity record and append it to $ISOQ_PARITY_LOG (JSON lines) when set."""
+    print(json.dumps(record))
+    path = os.environ.get("ISOQ_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(record) + "\n")
 
 
 class Run:

@@ -45,6 +45,10 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the multi-token and context-parallel measurements")
+    ap.add_argument("--chunk", type=int, default=16,
+                    help="query tokens per sequence of the multi-token measurement")
     ap.add_argument("--seqs", type=int, default=0,
                     help="use only this many sequences of the workload (small profiling case)")
     return ap.parse_args()
@@ -416,6 +420,12 @@ def run_ours(args, cfg):
     }
     if e2e:
         line["e2e"] = e2e
+    if not args.no_next:
+        line["multi_token"] = _bench_multi_token(args, cfg, params, cache, lens, flush, stream,
+                                                 rank_max, packed, peak, peak_kind)
+        line["context_parallel"] = _bench_context_parallel(
+            args, cfg, params, cache, layout, lens, Q, flush, stream, rank_max, world, rank,
+            packed, peak, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:
@@ -423,6 +433,73 @@ def run_ours(args, cfg):
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def _time_calls(fn, flush, stream, iters: int = 5, warmup: int = 2) -> float:
+    """Mean device time (ms) of fn() on `stream`, L2 flushed before every call."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(iters):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    return total / iters
+
+
+def _bench_multi_token(args, cfg, params, cache, lens, flush, stream, rank_max, packed, peak,
+                       peak_kind):
+    """Causal attention of a chunk of query tokens per sequence on the same packed cache."""
+    import torch
+
+    import rotated_bit_kv_isoquant_b200 as iq
+    import workloads as wl
+    n_q = args.chunk
+    dev = cache.blocks.device
+    Qc = wl.query_chunk(cfg, n_q, device=dev)
+    out = torch.empty((cfg.n_seqs, n_q, cfg.n_q_heads, cfg.d), dtype=torch.float32, device=dev)
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    nb = iq.isoq_multi_token_workspace_bytes(cfg.n_seqs, n_q, cfg.n_q_heads, cfg.n_kv_heads,
+                                             cfg.d, max(lens))
+    ws = torch.empty((nb,), dtype=torch.uint8, device=dev)
+    fn = lambda: iq.isoq_multi_token_attention(params, cache, Qc, sl, max(lens), out, cfg.scale,
+                                               ws, stream=stream)
+    ms = rank_max(_time_calls(fn, flush, stream))
+    gbs = packed / (ms / 1e3) / 1e9
+    return {"n_q": n_q, "ms_per_call": ms,
+            "query_tokens_per_s": cfg.n_seqs * n_q / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "peak_kind": peak_kind,
+                         "note": "packed KV counted once per call; this version streams it "
+                                 "once per 8 (query token, head) rows"}}
+
+
+def _bench_context_parallel(args, cfg, params, cache, layout, lens, Q, flush, stream, rank_max,
+                            world, rank, packed, peak, peak_kind):
+    """One decode step of the whole workload with every context split over the ranks:
+    each rank decodes its slice (a view of its replica's cache), one all-gather of the
+    states, then the merge (strong scaling over the context)."""
+    import torch
+
+    from rotated_bit_kv_isoquant_b200.context_parallel import ContextParallelDecoder, slice_of
+    view, local = slice_of(cache, layout.page_table, lens, world, rank)
+    dec = ContextParallelDecoder(params, view, cfg.n_seqs, cfg.n_q_heads, max(1, max(local)))
+    dev = cache.blocks.device
+    sl = torch.tensor(local, dtype=torch.int32, device=dev)
+    out = torch.empty((cfg.n_seqs, cfg.n_q_heads, cfg.d), dtype=torch.float32, device=dev)
+    fn = lambda: dec(Q, sl, out, cfg.scale, stream=stream)
+    ms = rank_max(_time_calls(fn, flush, stream))
+    gbs = packed / (ms / 1e3) / 1e9
+    return {"value": gbs, "unit": "GB/s", "scaling": "strong", "ms_per_call": ms,
+            "n_gpus": world, "state_bytes_per_rank": int(dec.state.numel() * 4),
+            "roofline_frac_per_gpu": gbs / world / peak, "peak_kind": peak_kind}
 
 
 def main():

@@ -221,6 +221,34 @@ int isoq_decode_attention_noalloc(const isoq_params* params, const isoq_cache* c
                                   const int32_t* seq_lens, int max_seq_len, float* out,
                                   float scale, void* stream);
 
+/* =======================================================================================
+ * Multi-token attention on the packed cache (a chunk of n_q query tokens per sequence:
+ * chunked prefill, speculative-decoding verification).
+ *
+ * The chunk's K/V must already be appended (isoq_quantize_append).  With L = seq_lens[s]
+ * cached tokens, query token i (0 <= i < n_q) of sequence s sits at position L - n_q + i
+ * and attends, causally, cache positions 0 .. L - n_q + i; for each (i, query head h) the
+ * result is what isoq_decode_attention returns for one query attending the first
+ * L - n_q + i + 1 tokens (the same rotation, codebook and merge), so the method is the
+ * one of the decode above ("RotaryQuant ...", Abstract: attention on the packed codes).
+ * A row whose position is negative (L < n_q - i) attends nothing and is all zeros.
+ *
+ * Q: device [n_seqs][n_q][n_q_heads][d], element type q_dtype.  out: device fp32
+ * [n_seqs][n_q][n_q_heads][d].  workspace: device, 16-byte aligned, at least
+ * isoq_multi_token_workspace_bytes(...) bytes for the same sizes.  Other arguments as
+ * isoq_decode_attention; n_q = 1 is exactly the decode.  Requires
+ * n_kv_heads * ceil(n_q * n_q_heads / n_kv_heads / 8) <= 65535, else ISOQ_E_ARG.
+ * Errors: ISOQ_E_ARG, ISOQ_E_DIM, ISOQ_E_GQA, ISOQ_E_WORKSPACE, ISOQ_E_DEVICE, ISOQ_E_CUDA.
+ * ===================================================================================== */
+size_t isoq_multi_token_workspace_bytes(int n_seqs, int n_q, int n_q_heads, int n_kv_heads,
+                                        int d, int max_seq_len);
+
+int isoq_multi_token_attention(const isoq_params* params, const isoq_cache* cache,
+                               const void* Q, int q_dtype, int n_seqs, int n_q, int n_q_heads,
+                               const int32_t* seq_lens, int max_seq_len, float* out,
+                               float scale, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* Number of context chunks (splits) the decode uses for these sizes on the current
  * device; >= 1, or a negative error code. */
 int isoq_decode_num_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len);

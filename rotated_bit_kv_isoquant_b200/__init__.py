@@ -76,6 +76,8 @@ _SIGS = {
     "isoq_decode_attention": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
     "isoq_decode_attention_noalloc": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p]),
     "isoq_decode_state_bytes": (_sz, [_i, _i, _i]),
+    "isoq_multi_token_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "isoq_multi_token_attention": (_i, [_p, _cp, _p, _i, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
     "isoq_decode_partial_state": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
     "isoq_decode_merge_states": (_i, [_p, _p, _i, _i, _i, _p, _p]),
     "isoq_get_status": (_i, [_cp, ctypes.POINTER(ctypes.c_uint32)]),
@@ -250,6 +252,26 @@ def isoq_decode_attention_noalloc(params: Params, cache: PagedCache, Q, seq_lens
         Q.shape[1], _dev_ptr(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
         _dev_ptr(out, "out", torch.float32), float(scale), _stream_ptr(stream)),
         "isoq_decode_attention_noalloc")
+
+
+def isoq_multi_token_workspace_bytes(n_seqs, n_q, n_q_heads, n_kv_heads, d, max_seq_len) -> int:
+    return int(_lib.isoq_multi_token_workspace_bytes(n_seqs, n_q, n_q_heads, n_kv_heads, d,
+                                                     max_seq_len))
+
+
+def isoq_multi_token_attention(params: Params, cache: PagedCache, Q, seq_lens, max_seq_len: int,
+                               out, scale: float, workspace, stream=None) -> None:
+    """Causal attention of a chunk of query tokens per sequence on the packed cache.
+    Q: CUDA [n_seqs][n_q][n_q_heads][d] (query i at position seq_len - n_q + i); out fp32
+    like Q; workspace >= isoq_multi_token_workspace_bytes(...) bytes."""
+    import torch
+    n_seqs, n_q, n_q_heads = Q.shape[0], Q.shape[1], Q.shape[2]
+    _check(_lib.isoq_multi_token_attention(
+        params.handle, ctypes.byref(cache.c), _dev_ptr(Q, "Q"), _dtype_code(Q), n_seqs, n_q,
+        n_q_heads, _dev_ptr(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
+        _dev_ptr(out, "out", torch.float32), float(scale), _dev_ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+        "isoq_multi_token_attention")
 
 
 def isoq_decode_state_bytes(n_seqs, n_q_heads, d) -> int:

@@ -38,10 +38,49 @@ def gather_states(state, group=None):
     """All-gather of the ranks' state tensors: returns [world, *state.shape], entry r =
     rank r's state.  Works on any torch.distributed backend (NCCL over NVLink on GPUs)."""
     import torch.distributed as dist
+    if not dist.is_initialized():   # a single-process job holds the whole context
+        return state.unsqueeze(0)
     world = dist.get_world_size(group)
     out = state.new_empty((world, *state.shape))
     dist.all_gather(list(out.unbind(0)), state.contiguous(), group=group)
     return out
+
+
+class CacheSlice:
+    """A view of an existing paged cache through another page table (same blocks, same
+    status word): e.g. the pages of one rank's slice of each sequence."""
+
+    def __init__(self, cache: PagedCache, page_table):
+        from . import isoq_cache
+        self.d, self.n_kv_heads, self.n_pages = cache.d, cache.n_kv_heads, cache.n_pages
+        self.blocks, self.status = cache.blocks, cache.status
+        self.page_table = page_table.to(device=cache.blocks.device,
+                                        dtype=page_table.dtype).int().contiguous()
+        self._c = isoq_cache(cache.d, cache.n_kv_heads, ISOQ_PAGE_SIZE, cache.n_pages,
+                             self.page_table.shape[1], self.page_table.shape[0],
+                             cache.blocks.data_ptr(), self.page_table.data_ptr(),
+                             cache.status.data_ptr())
+
+    @property
+    def c(self):
+        return self._c
+
+
+def slice_of(cache: PagedCache, page_table, lens, world: int, rank: int):
+    """This rank's slice of every sequence of a cache that holds whole contexts: a
+    CacheSlice over the slice's pages, and the slice lengths."""
+    import torch
+    pt = page_table.cpu()
+    rows, local = [], []
+    for s, n in enumerate(lens):
+        a, b = shard_tokens(int(n), world, rank)
+        rows.append(pt[s, a // ISOQ_PAGE_SIZE:-(-b // ISOQ_PAGE_SIZE)])
+        local.append(b - a)
+    width = max(1, max(len(r) for r in rows))
+    t = torch.zeros((len(rows), width), dtype=torch.int32)
+    for s, r in enumerate(rows):
+        t[s, :len(r)] = r
+    return CacheSlice(cache, t), local
 
 
 class ContextParallelDecoder:

@@ -94,13 +94,14 @@ struct SplitPlan {
 // Context chunking for the decode kernel: about ISOQ_DEC_WAVES waves of (chunk, KV head,
 // query-head block, sequence) CTAs at the kernel's resident CTAs per SM, each chunk a whole
 // number of pages and at least min_pages pages when the context allows.
-SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len) {
+SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len,
+                      int n_q = 1) {
   const bool tc = isoq::kUseTc128 && d == 128;
   const int n_sm = sm_count() * (tc ? isoq::decode_tc_resident_ctas() : isoq::decode_resident_ctas(d));
   const int min_pages = tc ? 8 : 16;  // per CTA: 4 tiles of 2 pages, or 4 pages per warp
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const int group = n_kv_heads > 0 ? n_q_heads / n_kv_heads : 1;
-  const long long units = (long long)n_seqs * n_kv_heads * ((group + 7) / 8);
+  const long long units = (long long)n_seqs * n_kv_heads * (((long long)n_q * group + 7) / 8);
   const long long target = (long long)n_sm * ISOQ_DEC_WAVES;
   long long want = units > 0 ? (target + units - 1) / units : 1;
   const long long cap = (max_pages + min_pages - 1) / min_pages;
@@ -283,10 +284,16 @@ size_t isoq_decode_workspace_bytes(int n_seqs, int n_q_heads, int n_kv_heads, in
 
 namespace {
 
+// The split kernel's grid.y = n_kv_heads * ceil(n_q * group / 8) must stay <= 65535.
+bool rows_fit(int n_q, int n_q_heads, int n_kv_heads) {
+  const long long group = n_kv_heads > 0 ? n_q_heads / n_kv_heads : 0;
+  return (long long)n_kv_heads * (((long long)n_q * group + 7) / 8) <= 65535;
+}
+
 // Shared by the decode entry points: validation, the split plan, then the split kernel and
 // the combine into either the output rows (out) or merged states (state).
 int decode_common(const isoq_params* params, const isoq_cache* cache, const void* Q,
-                  int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
+                  int q_dtype, int n_seqs, int n_q, int n_q_heads, const int32_t* seq_lens,
                   int max_seq_len, float* out, float* state, float scale, void* workspace,
                   size_t workspace_bytes, void* stream) {
   int rc = check_cache(cache, params);
@@ -295,16 +302,19 @@ int decode_common(const isoq_params* params, const isoq_cache* cache, const void
   if (!(scale == scale) || isinf(scale)) return ISOQ_E_ARG;
   if (n_q_heads % cache->n_kv_heads || n_q_heads / cache->n_kv_heads > 16) return ISOQ_E_GQA;
   if (n_seqs > cache->n_seqs) return ISOQ_E_ARG;
+  if (n_q < 1 || !rows_fit(n_q, n_q_heads, cache->n_kv_heads)) return ISOQ_E_ARG;
   if (n_seqs == 0 || n_q_heads == 0) return ISOQ_OK;
   if (!Q || !seq_lens || !(out || state) || !workspace) return ISOQ_E_ARG;
   if (state && ((uintptr_t)state & 15u) != 0) return ISOQ_E_ARG;
   if (((uintptr_t)workspace & 15u) != 0) return ISOQ_E_WORKSPACE;
-  const size_t need =
-      isoq_decode_workspace_bytes(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
+  const size_t need = isoq_multi_token_workspace_bytes(n_seqs, n_q, n_q_heads, cache->n_kv_heads,
+                                                       cache->d, max_seq_len);
   if (workspace_bytes < need) return ISOQ_E_WORKSPACE;
   if ((rc = check_device(params))) return rc;
-  const SplitPlan plan = plan_splits(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
+  const SplitPlan plan =
+      plan_splits(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len, n_q);
   isoq::DecodeArgs a{};
+  a.n_q = n_q;
   a.params = params->dev;
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;
@@ -336,7 +346,24 @@ int isoq_decode_attention(const isoq_params* params, const isoq_cache* cache, co
                           int q_dtype, int n_seqs, int n_q_heads, const int32_t* seq_lens,
                           int max_seq_len, float* out, float scale, void* workspace,
                           size_t workspace_bytes, void* stream) {
-  return decode_common(params, cache, Q, q_dtype, n_seqs, n_q_heads, seq_lens, max_seq_len,
+  return decode_common(params, cache, Q, q_dtype, n_seqs, 1, n_q_heads, seq_lens, max_seq_len,
+                       out, nullptr, scale, workspace, workspace_bytes, stream);
+}
+
+size_t isoq_multi_token_workspace_bytes(int n_seqs, int n_q, int n_q_heads, int n_kv_heads,
+                                        int d, int max_seq_len) {
+  if (n_seqs < 0 || n_q < 1 || n_q_heads < 0 || n_kv_heads < 1 || max_seq_len < 0) return 0;
+  if (!supported_d(d) || n_q_heads % n_kv_heads) return 0;
+  const int ns = plan_splits(n_seqs, n_q_heads, n_kv_heads, d, max_seq_len, n_q).n_splits;
+  return (size_t)n_seqs * n_q * n_q_heads * ns * isoq::partial_stride(d) * sizeof(float);
+}
+
+int isoq_multi_token_attention(const isoq_params* params, const isoq_cache* cache,
+                               const void* Q, int q_dtype, int n_seqs, int n_q, int n_q_heads,
+                               const int32_t* seq_lens, int max_seq_len, float* out,
+                               float scale, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return decode_common(params, cache, Q, q_dtype, n_seqs, n_q, n_q_heads, seq_lens, max_seq_len,
                        out, nullptr, scale, workspace, workspace_bytes, stream);
 }
 
@@ -350,7 +377,7 @@ int isoq_decode_partial_state(const isoq_params* params, const isoq_cache* cache
                               int max_seq_len, float* state, float scale, void* workspace,
                               size_t workspace_bytes, void* stream) {
   if (!state) return ISOQ_E_ARG;
-  return decode_common(params, cache, Q, q_dtype, n_seqs, n_q_heads, seq_lens, max_seq_len,
+  return decode_common(params, cache, Q, q_dtype, n_seqs, 1, n_q_heads, seq_lens, max_seq_len,
                        nullptr, state, scale, workspace, workspace_bytes, stream);
 }
 

@@ -28,9 +28,9 @@ namespace isoq {
 // round trips however many parts there are; warp 0 then finishes.
 template <int D, bool FINAL>
 __global__ void __launch_bounds__(128)
-    decode_combine_kernel(const float* __restrict__ params, int H, int n_q_heads, int n_splits,
-                          const float* __restrict__ partials, size_t sh_stride,
-                          size_t part_stride, float* __restrict__ out) {
+    decode_combine_kernel(const float* __restrict__ params, int H, int n_q_heads,
+                          int rows_per_seq, int n_splits, const float* __restrict__ partials,
+                          size_t sh_stride, size_t part_stride, float* __restrict__ out) {
   constexpr int E = D / 32;   // dims per lane
   constexpr int NB = E / 4;
   constexpr int PS = D + 4;
@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(128)
   const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   const int s = blockIdx.y, h = blockIdx.x;
   const int G = n_q_heads / H;
-  const float* base = partials + ((size_t)s * n_q_heads + h) * sh_stride;
+  const float* base = partials + ((size_t)s * rows_per_seq + h) * sh_stride;
 
   // global max of the splits' running maxima (empty splits report -inf)
   float M = -CUDART_INF_F;
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(128)
 
   const float Ls = red_l[0] + red_l[1] + red_l[2] + red_l[3];
   if constexpr (!FINAL) {
-    float* dst = out + ((size_t)s * n_q_heads + h) * PS;
+    float* dst = out + ((size_t)s * rows_per_seq + h) * PS;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
       const int dd = lane * E + i;
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(128)
     const int dd = lane * E + i;
     o[i] = (red_acc[0][dd] + red_acc[1][dd] + red_acc[2][dd] + red_acc[3][dd]) * inv;
   }
-  const float* hp = params + (size_t)(h / G) * D * 2;
+  const float* hp = params + (size_t)((h % n_q_heads) / G) * D * 2;
   float y[E];
 #pragma unroll
   for (int k = 0; k < NB; ++k) {
@@ -129,25 +129,26 @@ __global__ void __launch_bounds__(128)
   }
   wht_warp<E>(y, lane);
   const float r = rsqrtf((float)D);
-  float* dst = out + ((size_t)s * n_q_heads + h) * D + lane * E;
+  float* dst = out + ((size_t)s * rows_per_seq + h) * D + lane * E;
 #pragma unroll
   for (int i = 0; i < E; ++i) dst[i] = y[i] * r;
 }
 
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
-  cudaError_t e = (kUseTc128 && D == 128) ? launch_decode_split_tc(a, stream)
-                                           : launch_decode_split_mma(a, stream);
+  cudaError_t e = (kUseTc128 && D == 128 && a.n_q == 1) ? launch_decode_split_tc(a, stream)
+                                                         : launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_q_heads, a.n_seqs);
+  const int rows = a.n_q * a.n_q_heads;
+  dim3 grid(rows, a.n_seqs);
   const size_t PS = partial_stride(D);
   if (a.state)
     decode_combine_kernel<D, false><<<grid, 128, 0, stream>>>(
-        a.params, a.n_kv_heads, a.n_q_heads, a.n_splits, a.partials, a.n_splits * PS, PS,
+        a.params, a.n_kv_heads, a.n_q_heads, rows, a.n_splits, a.partials, a.n_splits * PS, PS,
         a.state);
   else
     decode_combine_kernel<D, true><<<grid, 128, 0, stream>>>(
-        a.params, a.n_kv_heads, a.n_q_heads, a.n_splits, a.partials, a.n_splits * PS, PS,
+        a.params, a.n_kv_heads, a.n_q_heads, rows, a.n_splits, a.partials, a.n_splits * PS, PS,
         a.out);
   return cudaGetLastError();
 }
@@ -168,11 +169,11 @@ cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int 
   const size_t PS = partial_stride(d);
   const size_t slice = (size_t)n_seqs * n_q_heads * PS;
   if (d == 128)
-    decode_combine_kernel<128, true><<<grid, 128, 0, stream>>>(params, n_kv_heads, n_q_heads,
-                                                               n_states, states, PS, slice, out);
+    decode_combine_kernel<128, true><<<grid, 128, 0, stream>>>(
+        params, n_kv_heads, n_q_heads, n_q_heads, n_states, states, PS, slice, out);
   else if (d == 256)
-    decode_combine_kernel<256, true><<<grid, 128, 0, stream>>>(params, n_kv_heads, n_q_heads,
-                                                               n_states, states, PS, slice, out);
+    decode_combine_kernel<256, true><<<grid, 128, 0, stream>>>(
+        params, n_kv_heads, n_q_heads, n_q_heads, n_states, states, PS, slice, out);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

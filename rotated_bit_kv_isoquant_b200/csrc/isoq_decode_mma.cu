@@ -44,7 +44,8 @@ struct MmaSmem {
   static constexpr int kRing = kWarps * NST * kStageBytes;
   static constexpr int kBarOff = kRing;
   static constexpr int kAOff = kBarOff + kWarps * NST * 8;
-  static constexpr int kBytes = kAOff + (D / 16) * 32 * 16;
+  static constexpr int kRowOff = kAOff + (D / 16) * 32 * 16;  // int [8]: output row per CTA row
+  static constexpr int kBytes = kRowOff + 8 * 4;
   static constexpr int kMergeBytes = kWarps * 8 * (D + 4) * 4;
   static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
   static_assert(kAOff % 16 == 0, "A fragments must be 16-byte aligned");
@@ -55,13 +56,15 @@ struct MmaSmem {
 template <int D>
 constexpr int dec_min_blocks() { return D == 128 ? 4 : 2; }
 
-template <int D, int NST, typename TQ>
+// MQ: chunks of several query tokens per sequence with causal limits; the decode (one
+// query token, every row attending the whole context) is compiled without them.
+template <int D, int NST, typename TQ, bool MQ>
 __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     decode_mma_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
                       const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
-                      const TQ* __restrict__ Q, int n_q_heads, const int32_t* __restrict__ seq_lens,
-                      float scale, int pages_per_split, int n_splits, float* __restrict__ partials,
-                      uint32_t* status) {
+                      const TQ* __restrict__ Q, int n_q_heads, int n_q,
+                      const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
+                      int n_splits, float* __restrict__ partials, uint32_t* status) {
   using SM = MmaSmem<D, NST>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
@@ -73,29 +76,47 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint4* qa = reinterpret_cast<uint4*>(smem + SM::kAOff);
+  int* row_off = reinterpret_cast<int*>(smem + SM::kRowOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int split = blockIdx.x, s = blockIdx.z;
+  // The CTA's 8 rows are (query token i, query head) pairs of KV head hk: row r is pair
+  // R = 8 rb + r of the group's n_q * G pairs, i = R / G, head hk * G + R % G.  Query token
+  // i of a sequence of len tokens sits at position len - n_q + i and attends the tokens
+  // before and at it (n_q = 1: the decode, every row attends the whole context).
+  if constexpr (!MQ) n_q = 1;
   const int G = n_q_heads / H;
-  const int nhb = (G + 7) >> 3;
-  const int hk = blockIdx.y / nhb, hb = blockIdx.y - hk * nhb;
-  const int h0 = hk * G + hb * 8;                // first query head of this CTA
-  const int nh = min(8, G - hb * 8);             // query heads handled here
+  const int n_rows = n_q * G;
+  const int nrb = (n_rows + 7) >> 3;
+  const int hk = blockIdx.y / nrb, rb = blockIdx.y - hk * nrb;
+  const int nh = min(8, n_rows - rb * 8);        // rows handled here
+  auto row_token = [&](int r) { return (rb * 8 + r) / G; };
+  auto row_index = [&](int r) {                  // row of the sequence's output / partials
+    const int R = rb * 8 + r;
+    return (R / G) * n_q_heads + hk * G + R % G;
+  };
 
   int len = __ldg(seq_lens + s);
   if (len > max_pages * kPage) {
     if (tid == 0 && split == 0 && blockIdx.y == 0) set_status(status, ISOQ_ST_LEN_RANGE);
     len = max_pages * kPage;
   }
+  // causal limits: lim(r) = len - n_q + 1 + i(r), clamped to [0, len]
+  const int lim_lo = MQ ? max(0, min(len, len - n_q + 1 + row_token(0))) : len;
+  const int lim_hi = MQ ? max(0, min(len, len - n_q + 1 + row_token(nh - 1))) : len;
+  const int lim_g =
+      MQ && g < nh ? max(0, min(len, len - n_q + 1 + row_token(g))) : lim_hi;
   const int p_begin = split * pages_per_split;
-  const int p_end = min((len + kPage - 1) / kPage, p_begin + pages_per_split);
+  const int p_end = min((lim_hi + kPage - 1) / kPage, p_begin + pages_per_split);
 
-  float* out_base = partials + ((size_t)s * n_q_heads + h0) * n_splits * PS + (size_t)split * PS;
+  float* out_base = partials + ((size_t)s * n_q * n_q_heads) * n_splits * PS + (size_t)split * PS;
+  if (tid < 8) row_off[tid] = tid < nh ? row_index(tid) : 0;
+  __syncthreads();
   if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
     for (int i = tid; i < nh * PS; i += blockDim.x) {
       const int h = i / PS, c = i - h * PS;
-      out_base[(size_t)h * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+      out_base[(size_t)row_off[h] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
     }
     return;
   }
@@ -143,7 +164,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     for (int h = warp; h < 8; h += kWarps) {
       float v[E];
       if (h < nh) {
-        const TQ* qp = Q + ((size_t)s * n_q_heads + h0 + h) * D + lane * E;
+        const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[h]) * D + lane * E;
 #pragma unroll
         for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
       } else {
@@ -214,7 +235,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     const int tok0 = pg * kPage;
 
     // a page whose 64 tokens are all valid takes the tile body without masking
-    const bool full = page_ok && tok0 + kPage <= len;
+    const bool full = page_ok && tok0 + kPage <= lim_lo;
     auto tile = [&](const int tb, auto full_c) {
       constexpr bool FULL = decltype(full_c)::value;
       // ---- a7: scores of 4 tiles of 8 tokens; B = K_hat^T of token tb + 8n + g ------------
@@ -266,10 +287,10 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
         nv[n][0] = nv2.x;
         nv[n][1] = nv2.y;
         if constexpr (!FULL) {
-          const bool v0 = page_ok && (tok0 + tk) < len;
-          const bool v1 = page_ok && (tok0 + tk + 1) < len;
-          sv[n][0] = v0 ? sv[n][0] : -CUDART_INF_F;
-          sv[n][1] = v1 ? sv[n][1] : -CUDART_INF_F;
+          const bool v0 = page_ok && (tok0 + tk) < lim_hi;
+          const bool v1 = page_ok && (tok0 + tk + 1) < lim_hi;
+          sv[n][0] = v0 && (!MQ || (tok0 + tk) < lim_g) ? sv[n][0] : -CUDART_INF_F;
+          sv[n][1] = v1 && (!MQ || (tok0 + tk + 1) < lim_g) ? sv[n][1] : -CUDART_INF_F;
           nv[n][0] = v0 ? nv[n][0] : 0.f;
           nv[n][1] = v1 ? nv[n][1] : 0.f;
         }
@@ -432,7 +453,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
         v += sc * mb[(w * 8 + h) * PS + (c == D ? D + 1 : c)];
       }
     }
-    float* o = out_base + (size_t)h * n_splits * PS;
+    float* o = out_base + (size_t)row_off[h] * n_splits * PS;
     if (c < D) o[c] = v;
     else {
       o[D] = M == -CUDART_INF_F ? -CUDART_INF_F : M / kLog2e;  // natural-log units
@@ -441,7 +462,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   }
 }
 
-template <int D, int NST, typename TQ>
+template <int D, int NST, typename TQ, bool MQ>
 static cudaError_t launch_mma_t(const DecodeArgs& a, cudaStream_t stream) {
   using SM = MmaSmem<D, NST>;
   // the dynamic shared-memory opt-in is per function and per device
@@ -450,26 +471,33 @@ static cudaError_t launch_mma_t(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !((attr_set >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(decode_mma_kernel<D, NST, TQ>,
+    e = cudaFuncSetAttribute(decode_mma_kernel<D, NST, TQ, MQ>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
     if (e != cudaSuccess) return e;
     attr_set |= 1ull << dev;
   }
   const int G = a.n_q_heads / a.n_kv_heads;
-  dim3 grid(a.n_splits, a.n_kv_heads * ((G + 7) / 8), a.n_seqs);
-  decode_mma_kernel<D, NST, TQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
+  dim3 grid(a.n_splits, a.n_kv_heads * ((a.n_q * G + 7) / 8), a.n_seqs);
+  decode_mma_kernel<D, NST, TQ, MQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
-      static_cast<const TQ*>(a.Q), a.n_q_heads, a.seq_lens, a.scale, a.pages_per_split,
+      static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
       a.n_splits, a.partials, a.status);
   return cudaGetLastError();
 }
 
 template <int D, int NST>
 cudaError_t launch_decode_mma_d(const DecodeArgs& a, cudaStream_t stream) {
+  const bool mq = a.n_q > 1;
   switch (a.q_dtype) {
-    case ISOQ_F32: return launch_mma_t<D, NST, float>(a, stream);
-    case ISOQ_BF16: return launch_mma_t<D, NST, __nv_bfloat16>(a, stream);
-    case ISOQ_F16: return launch_mma_t<D, NST, __half>(a, stream);
+    case ISOQ_F32:
+      return mq ? launch_mma_t<D, NST, float, true>(a, stream)
+                : launch_mma_t<D, NST, float, false>(a, stream);
+    case ISOQ_BF16:
+      return mq ? launch_mma_t<D, NST, __nv_bfloat16, true>(a, stream)
+                : launch_mma_t<D, NST, __nv_bfloat16, false>(a, stream);
+    case ISOQ_F16:
+      return mq ? launch_mma_t<D, NST, __half, true>(a, stream)
+                : launch_mma_t<D, NST, __half, false>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -502,18 +530,18 @@ int decode_resident_ctas(int d) {
     cudaError_t e;
     if (d == 256) {
       using SM = MmaSmem<256, ISOQ_DEC_NST256>;
-      e = cudaFuncSetAttribute(decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16>,
+      e = cudaFuncSetAttribute(decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16>, kWarps * 32, SM::kBytes);
+            &n, decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false>, kWarps * 32, SM::kBytes);
     } else {
       using SM = MmaSmem<128, ISOQ_DEC_NST128>;
-      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16>,
+      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16>, kWarps * 32, SM::kBytes);
+            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false>, kWarps * 32, SM::kBytes);
     }
     if (e != cudaSuccess || n < 1) {
       cudaGetLastError();

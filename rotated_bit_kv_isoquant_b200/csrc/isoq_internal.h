@@ -32,13 +32,14 @@ struct DecodeArgs {
   const void* Q;
   int q_dtype;
   int n_seqs, n_q_heads;
+  int n_q;              // query tokens per sequence (1 = decode)
   const int32_t* seq_lens;
   float scale;
   int n_splits;         // context chunks per (sequence, KV head)
   int pages_per_split;  // pages in each chunk
-  float* partials;      // [n_seqs][n_q_heads][n_splits][d + 4]
-  float* out;           // [n_seqs][n_q_heads][d] (when state is null)
-  float* state;         // if set: merged state [n_seqs][n_q_heads][d + 4] instead of out
+  float* partials;      // [n_seqs][n_q][n_q_heads][n_splits][d + 4]
+  float* out;           // [n_seqs][n_q][n_q_heads][d] (when state is null)
+  float* state;         // if set: merged state [n_seqs][n_q][n_q_heads][d + 4] instead of out
   uint32_t* status;
 };
 

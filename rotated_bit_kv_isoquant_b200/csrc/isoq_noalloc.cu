@@ -113,6 +113,7 @@ extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const is
   a.q_dtype = q_dtype;
   a.n_seqs = n_seqs;
   a.n_q_heads = n_q_heads;
+  a.n_q = 1;
   a.seq_lens = seq_lens;
   a.scale = scale;
   a.n_splits = n_splits;

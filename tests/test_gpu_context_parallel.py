@@ -11,8 +11,7 @@ import torch
 
 import rotated_bit_kv_isoquant_b200 as iq
 import workloads as wl
-from rotated_bit_kv_isoquant_b200.context_parallel import (ContextParallelDecoder,
-                                                          shard_tokens)
+from rotated_bit_kv_isoquant_b200.context_parallel import ContextParallelDecoder, slice_of
 from _gpu_util import Run, check_attention, log_record
 
 pytestmark = pytest.mark.gpu
@@ -24,41 +23,9 @@ def _cuda():
         pytest.skip("needs a CUDA device")
 
 
-class _View:
-    """The cache of one emulated rank: the shared blocks, a page table of its slice."""
-
-    def __init__(self, base: iq.PagedCache, page_table: torch.Tensor):
-        self.d, self.n_kv_heads, self.n_pages = base.d, base.n_kv_heads, base.n_pages
-        self.blocks = base.blocks
-        self.page_table = page_table.to(device=base.blocks.device, dtype=torch.int32).contiguous()
-        self.status = base.status
-        self._c = iq.isoq_cache(base.d, base.n_kv_heads, iq.ISOQ_PAGE_SIZE, base.n_pages,
-                                self.page_table.shape[1], self.page_table.shape[0],
-                                base.blocks.data_ptr(), self.page_table.data_ptr(),
-                                base.status.data_ptr())
-
-    @property
-    def c(self):
-        return self._c
-
-
 def _rank_views(run: Run, lens, R):
-    """Per emulated rank: its cache view and its local lengths."""
-    pt = run.layout.page_table
-    views = []
-    for r in range(R):
-        rows, local = [], []
-        for s, L in enumerate(lens):
-            a, b = shard_tokens(L, R, r)
-            p0, p1 = a // 64, -(-b // 64)
-            rows.append(pt[s, p0:p1].tolist())
-            local.append(b - a)
-        width = max(1, max(len(x) for x in rows))
-        t = torch.zeros((len(lens), width), dtype=torch.int32)
-        for s, x in enumerate(rows):
-            t[s, :len(x)] = torch.tensor(x, dtype=torch.int32)
-        views.append((_View(run.cache, t), local))
-    return views
+    """Per emulated rank: a view of its slice of the cache and its local lengths."""
+    return [slice_of(run.cache, run.layout.page_table, lens, R, r) for r in range(R)]
 
 
 def _cp_decode(run: Run, Q, lens, R, order=None):

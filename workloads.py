@@ -204,6 +204,16 @@ def queries(cfg: Workload, device="cpu") -> torch.Tensor:
     return q.to(cfg.in_dtype).contiguous()
 
 
+def query_chunk(cfg: Workload, n_q: int, device="cpu") -> torch.Tensor:
+    """A chunk of n_q query tokens per sequence (chunked prefill / speculative verify):
+    [n_seqs][n_q][n_q_heads][d] in cfg.in_dtype, drawn like queries()."""
+    g = _gen(device, _seed(cfg.idx, _Q, 1, n_q))
+    q = torch.randn((cfg.n_seqs, n_q, cfg.n_q_heads, cfg.d), generator=g, device=device)
+    if cfg.q_dist == "gauss_outlier8":
+        q *= _outlier_mult(cfg.n_q_heads, cfg.d, 4, 8.0, _seed(cfg.idx, _QOUT, 0, 0), device)
+    return q.to(cfg.in_dtype).contiguous()
+
+
 @dataclass
 class PageLayout:
     """Page table of a workload: per sequence, logical page -> physical page id."""

@@ -8,6 +8,10 @@ Every function follows the method page "RotaryQuant: Fitting 120B MoE Models on 
 Hardware via Fused Compressed-Space Attention", Abstract (WHT, block-diagonal SO(4)
 rotations, 3-bit scalar quantisation, attention on the packed tensors); the readings the
 pages leave open are listed at the top of ``isoq_oracle.c``.  All arithmetic is fp64.
+
+Variants of the same family take ``bits`` (2, 3 or 4: the Lloyd-Max codebook size) and
+``rot`` (0: SO(4) quaternion blocks, IsoQuant; 1: SO(2) blocks, the PlanarQuant variant the
+same abstract names); the defaults are the method's 3 bits and SO(4).
 """
 from __future__ import annotations
 
@@ -100,6 +104,41 @@ def _declare(L):
     L.ref_unpack_codes_batch.argtypes = [_p, _i, ctypes.c_long, _p]
     L.ref_attention_full.restype = None
     L.ref_attention_full.argtypes = [_i, _i, _i, _i, _p, _p, _p, _d, _p]
+    L.ref_level_v.restype = _d
+    L.ref_level_v.argtypes = [_i, _i]
+    L.ref_threshold_v.restype = _d
+    L.ref_threshold_v.argtypes = [_i, _i]
+    L.ref_make_params_so2.restype = None
+    L.ref_make_params_so2.argtypes = [ctypes.c_uint64, _i, _i, _p, _p]
+    L.ref_params_per_head.restype = _i
+    L.ref_params_per_head.argtypes = [_i, _i]
+    L.ref_so2_forward.restype = None
+    L.ref_so2_forward.argtypes = [_p, _p, _p]
+    L.ref_so2_inverse.restype = None
+    L.ref_so2_inverse.argtypes = [_p, _p, _p]
+    L.ref_rotate_v.restype = None
+    L.ref_rotate_v.argtypes = [_i, _p, _p, _p, _i]
+    L.ref_unrotate_v.restype = None
+    L.ref_unrotate_v.argtypes = [_i, _p, _p, _p, _i]
+    L.ref_quantize_vector_v.restype = _i
+    L.ref_quantize_vector_v.argtypes = [_i, _i, _p, _p, _i, _p, _p, _p]
+    L.ref_pack_codes_v.restype = None
+    L.ref_pack_codes_v.argtypes = [_i, _p, _i, _p]
+    L.ref_unpack_codes_v.restype = None
+    L.ref_unpack_codes_v.argtypes = [_i, _p, _i, _p]
+    L.ref_block_bytes_v.restype = ctypes.c_size_t
+    L.ref_block_bytes_v.argtypes = [_i, _i, _i]
+    L.ref_quantize_append_v.restype = _i
+    L.ref_quantize_append_v.argtypes = [_i, _i, _p, _i, _i, _i, _p, _p, _i, _p, _p, _i, _p, _p]
+    L.ref_dequantize_slot_v.restype = None
+    L.ref_dequantize_slot_v.argtypes = [_i, _i, _p, _i, _i, _i, _p, _i, _i, _i, _i, _p]
+    L.ref_decode_attention_v.restype = None
+    L.ref_decode_attention_v.argtypes = [_i, _i, _p, _i, _i, _i, _p, _p, _i, _i, _i, _p, _p, _d,
+                                         _p, _p, _i]
+    L.ref_quantize_rows_v.restype = None
+    L.ref_quantize_rows_v.argtypes = [_i, _i, _p, _i, _i, _p, _i, _p, _p, _p]
+    L.ref_unpack_codes_batch_v.restype = None
+    L.ref_unpack_codes_batch_v.argtypes = [_i, _p, _i, ctypes.c_long, _p]
 
 
 def _ptr(a: np.ndarray):
@@ -117,14 +156,14 @@ def _i32(a) -> np.ndarray:
 # ------------------------------------------------------------------------------------
 # Constants
 # ------------------------------------------------------------------------------------
-def levels() -> np.ndarray:
-    """The 8 codebook levels in N(0,1) units, ascending (Lloyd-Max, Max 1960)."""
-    return np.array([lib().ref_level(c) for c in range(8)])
+def levels(bits: int = 3) -> np.ndarray:
+    """The 2^bits codebook levels in N(0,1) units, ascending (Lloyd-Max, Max 1960)."""
+    return np.array([lib().ref_level_v(bits, c) for c in range(1 << bits)])
 
 
-def thresholds() -> np.ndarray:
-    """The 7 decision thresholds: midpoints of adjacent levels."""
-    return np.array([lib().ref_threshold(j) for j in range(7)])
+def thresholds(bits: int = 3) -> np.ndarray:
+    """The 2^bits - 1 decision thresholds: midpoints of adjacent levels."""
+    return np.array([lib().ref_threshold_v(bits, j) for j in range((1 << bits) - 1)])
 
 
 def num_threads() -> int:
@@ -151,6 +190,33 @@ def make_params(seed: int, d: int, n_kv_heads: int):
     p32 = np.zeros((n_kv_heads, d // 4, 2, 4), dtype=np.float32)
     lib().ref_make_params(ctypes.c_uint64(seed), d, n_kv_heads, _ptr(p64), _ptr(p32))
     return p64, p32
+
+
+def make_params_so2(seed: int, d: int, n_kv_heads: int):
+    """(params64, params32), each [n_kv_heads][d/2][2]: per 2x2 block (cos phi, sin phi)."""
+    p64 = np.zeros((n_kv_heads, d // 2, 2), dtype=np.float64)
+    p32 = np.zeros((n_kv_heads, d // 2, 2), dtype=np.float32)
+    lib().ref_make_params_so2(ctypes.c_uint64(seed), d, n_kv_heads, _ptr(p64), _ptr(p32))
+    return p64, p32
+
+
+def make_params_v(seed: int, d: int, n_kv_heads: int, rot: int = 0):
+    """make_params (rot 0, SO(4)) or make_params_so2 (rot 1)."""
+    return make_params_so2(seed, d, n_kv_heads) if rot == 1 else make_params(seed, d, n_kv_heads)
+
+
+def so2_forward(cs, y) -> np.ndarray:
+    cs, y = _f64(cs), _f64(y)
+    z = np.zeros(2)
+    lib().ref_so2_forward(_ptr(cs), _ptr(y), _ptr(z))
+    return z
+
+
+def so2_inverse(cs, z) -> np.ndarray:
+    cs, z = _f64(cs), _f64(z)
+    y = np.zeros(2)
+    lib().ref_so2_inverse(_ptr(cs), _ptr(z), _ptr(y))
+    return y
 
 
 def wht(x) -> np.ndarray:
@@ -185,18 +251,19 @@ def so4_inverse(p, q, z) -> np.ndarray:
     return y
 
 
-def rotate(params_head, x) -> np.ndarray:
-    """z = R x for one head: WHT then the SO(4) blocks.  params_head: [d/4][2][4]."""
+def rotate(params_head, x, rot: int = 0) -> np.ndarray:
+    """z = R x for one head: WHT then the blocks (rot 0: SO(4), params_head [d/4][2][4];
+    rot 1: SO(2), params_head [d/2][2])."""
     ph, x = _f64(params_head), _f64(x)
     z = np.zeros_like(x)
-    lib().ref_rotate(_ptr(ph), _ptr(x), _ptr(z), x.shape[-1])
+    lib().ref_rotate_v(rot, _ptr(ph), _ptr(x), _ptr(z), x.shape[-1])
     return z
 
 
-def unrotate(params_head, z) -> np.ndarray:
+def unrotate(params_head, z, rot: int = 0) -> np.ndarray:
     ph, z = _f64(params_head), _f64(z)
     x = np.zeros_like(z)
-    lib().ref_unrotate(_ptr(ph), _ptr(z), _ptr(x), z.shape[-1])
+    lib().ref_unrotate_v(rot, _ptr(ph), _ptr(z), _ptr(x), z.shape[-1])
     return x
 
 
@@ -214,60 +281,61 @@ def fp16_value(h: int) -> float:
 # ------------------------------------------------------------------------------------
 # Quantisation and packing
 # ------------------------------------------------------------------------------------
-def quantize_vector(params_head, x):
+def quantize_vector(params_head, x, bits: int = 3, rot: int = 0):
     """-> (codes uint8[d], norm16 bits, overflow flag, z fp64[d])."""
     ph, x = _f64(params_head), _f64(x)
     d = x.shape[0]
     codes = np.zeros(d, dtype=np.uint8)
     n16 = ctypes.c_uint16(0)
     z = np.zeros(d)
-    ov = lib().ref_quantize_vector(_ptr(ph), _ptr(x), d, _ptr(codes), ctypes.byref(n16), _ptr(z))
+    ov = lib().ref_quantize_vector_v(bits, rot, _ptr(ph), _ptr(x), d, _ptr(codes),
+                                     ctypes.byref(n16), _ptr(z))
     return codes, int(n16.value), int(ov), z
 
 
-def pack_codes(codes) -> np.ndarray:
+def pack_codes(codes, bits: int = 3) -> np.ndarray:
     codes = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
     d = codes.shape[0]
-    out = np.zeros(3 * d // 8, dtype=np.uint8)
-    lib().ref_pack_codes(_ptr(codes), d, _ptr(out))
+    out = np.zeros(bits * d // 8, dtype=np.uint8)
+    lib().ref_pack_codes_v(bits, _ptr(codes), d, _ptr(out))
     return out
 
 
-def unpack_codes(packed, d: int) -> np.ndarray:
+def unpack_codes(packed, d: int, bits: int = 3) -> np.ndarray:
     packed = np.ascontiguousarray(np.asarray(packed, dtype=np.uint8))
     codes = np.zeros(d, dtype=np.uint8)
-    lib().ref_unpack_codes(_ptr(packed), d, _ptr(codes))
+    lib().ref_unpack_codes_v(bits, _ptr(packed), d, _ptr(codes))
     return codes
 
 
-def block_bytes(d: int, page: int = 64) -> int:
-    return int(lib().ref_block_bytes(d, page))
+def block_bytes(d: int, page: int = 64, bits: int = 3) -> int:
+    return int(lib().ref_block_bytes_v(bits, d, page))
 
 
 def quantize_append(params64, d, n_kv_heads, page, blocks, page_table, K, V, seq_ids,
-                    positions) -> int:
+                    positions, bits: int = 3, rot: int = 0) -> int:
     """Quantise K, V ([n_tokens][n_kv_heads][d]) into ``blocks`` (uint8, modified in place).
     Returns the number of saturated norms."""
     assert blocks.dtype == np.uint8 and blocks.flags.c_contiguous
     pt = _i32(page_table)
     K, V = _f64(K), _f64(V)
     sid, pos = _i32(seq_ids), _i32(positions)
-    return int(lib().ref_quantize_append(_ptr(_f64(params64)), d, n_kv_heads, page,
-                                         _ptr(blocks), _ptr(pt), pt.shape[-1], _ptr(K),
-                                         _ptr(V), K.shape[0], _ptr(sid), _ptr(pos)))
+    return int(lib().ref_quantize_append_v(bits, rot, _ptr(_f64(params64)), d, n_kv_heads,
+                                           page, _ptr(blocks), _ptr(pt), pt.shape[-1], _ptr(K),
+                                           _ptr(V), K.shape[0], _ptr(sid), _ptr(pos)))
 
 
 def dequantize_slot(params64, d, n_kv_heads, page, blocks, phys_page, kv_head, slot,
-                    kind) -> np.ndarray:
+                    kind, bits: int = 3, rot: int = 0) -> np.ndarray:
     out = np.zeros(d)
-    lib().ref_dequantize_slot(_ptr(_f64(params64)), d, n_kv_heads, page,
-                              _ptr(np.ascontiguousarray(blocks)), phys_page, kv_head, slot,
-                              kind, _ptr(out))
+    lib().ref_dequantize_slot_v(bits, rot, _ptr(_f64(params64)), d, n_kv_heads, page,
+                                _ptr(np.ascontiguousarray(blocks)), phys_page, kv_head, slot,
+                                kind, _ptr(out))
     return out
 
 
 def decode_attention(params64, d, n_kv_heads, page, blocks, page_table, seq_lens, Q, scale,
-                     sel=None) -> np.ndarray:
+                     sel=None, bits: int = 3, rot: int = 0) -> np.ndarray:
     """Decode attention on the packed cache.  Q: [n_seqs][n_q_heads][d].  ``sel``: optional
     list of (seq, q_head) pairs to compute (others stay NaN)."""
     Q = _f64(Q)
@@ -279,10 +347,10 @@ def decode_attention(params64, d, n_kv_heads, page, blocks, page_table, seq_lens
     if sel is not None:
         sa = _i32(np.asarray(sel).reshape(-1, 2))
         selp, nsel = _ptr(sa), sa.shape[0]
-    lib().ref_decode_attention(_ptr(_f64(params64)), d, n_kv_heads, page,
-                               _ptr(np.ascontiguousarray(blocks)), _ptr(pt), pt.shape[-1],
-                               n_seqs, n_q_heads, _ptr(sl), _ptr(Q), float(scale), _ptr(out),
-                               selp, nsel)
+    lib().ref_decode_attention_v(bits, rot, _ptr(_f64(params64)), d, n_kv_heads, page,
+                                 _ptr(np.ascontiguousarray(blocks)), _ptr(pt), pt.shape[-1],
+                                 n_seqs, n_q_heads, _ptr(sl), _ptr(Q), float(scale), _ptr(out),
+                                 selp, nsel)
     return out
 
 
@@ -296,7 +364,7 @@ def attention_full(K, V, Q, scale) -> np.ndarray:
     return out
 
 
-def quantize_rows(params64, X, with_dist: bool = True):
+def quantize_rows(params64, X, with_dist: bool = True, bits: int = 3, rot: int = 0):
     """Quantise X [n_rows][n_kv_heads][d] (head h with params64[h]).
     -> (codes uint8 [n][H][d], norms uint16 [n][H], dist fp64 [n][H][d] or None), where
     dist is the distance of u to the nearest threshold."""
@@ -305,16 +373,16 @@ def quantize_rows(params64, X, with_dist: bool = True):
     codes = np.zeros((n, H, d), np.uint8)
     norms = np.zeros((n, H), np.uint16)
     dist = np.zeros((n, H, d)) if with_dist else None
-    lib().ref_quantize_rows(_ptr(_f64(params64)), d, H, _ptr(X), n, _ptr(codes), _ptr(norms),
-                            _ptr(dist) if with_dist else None)
+    lib().ref_quantize_rows_v(bits, rot, _ptr(_f64(params64)), d, H, _ptr(X), n, _ptr(codes),
+                              _ptr(norms), _ptr(dist) if with_dist else None)
     return codes, norms, dist
 
 
-def unpack_codes_batch(packed, d: int) -> np.ndarray:
-    """packed uint8 [..., 3d/8] -> codes uint8 [..., d]."""
+def unpack_codes_batch(packed, d: int, bits: int = 3) -> np.ndarray:
+    """packed uint8 [..., bits*d/8] -> codes uint8 [..., d]."""
     packed = np.ascontiguousarray(np.asarray(packed, dtype=np.uint8))
     lead = packed.shape[:-1]
     n = int(np.prod(lead)) if lead else 1
     codes = np.zeros(lead + (d,), np.uint8)
-    lib().ref_unpack_codes_batch(_ptr(packed), d, n, _ptr(codes))
+    lib().ref_unpack_codes_batch_v(bits, _ptr(packed), d, n, _ptr(codes))
     return codes

@@ -30,6 +30,11 @@
  *   - decode: softmax(scale * q.k) over positions 0..len-1 of each sequence, query head
  *     h reading KV head h / G.
  *
+ * Format variants (functions with a _v suffix take bits and rot; the plain names are the
+ * method's 3 bits and SO(4)): 2- and 4-bit Lloyd-Max codebooks of the same family (Max
+ * 1960, N = 4 and 16), and the PlanarQuant variant the same abstract names, read as the
+ * WHT followed by 2x2 (SO(2)) rotation blocks with Haar-uniform angles.
+ *
  * Everything is plain fp64 scalar code in the order the method states it.  The only
  * parallelism is an OpenMP loop over independent vectors / (sequence, head) pairs.
  */
@@ -43,15 +48,31 @@
 #endif
 
 /* ------------------------------------------------------------------------------ */
-/* Codebook: Lloyd-Max 8-level quantiser for N(0,1) (Max, 1960), ascending.         */
+/* Codebooks: Lloyd-Max quantisers for N(0,1) (Max, 1960, Table I), ascending:      */
+/* 8 levels for the method's 3 bits; 4 and 16 levels for the 2- and 4-bit variants  */
+/* of the same family.                                                               */
 /* ------------------------------------------------------------------------------ */
 static const double REF_LEVELS[8] = {-2.1520, -1.3440, -0.7560, -0.2451,
                                      0.2451,  0.7560,  1.3440,  2.1520};
+static const double REF_LEVELS2[4] = {-1.5104, -0.4528, 0.4528, 1.5104};
+static const double REF_LEVELS4[16] = {-2.7326, -2.0690, -1.6180, -1.2562, -0.9424, -0.6568,
+                                       -0.3881, -0.1284, 0.1284,  0.3881,  0.6568,  0.9424,
+                                       1.2562,  1.6180,  2.0690,  2.7326};
+
+static const double *levels_of(int bits) {
+  return bits == 2 ? REF_LEVELS2 : (bits == 4 ? REF_LEVELS4 : REF_LEVELS);
+}
+
+double ref_level_v(int bits, int code) { return levels_of(bits)[code]; }
+
+/* Threshold j (0 .. 2^bits - 2) is the midpoint between levels j and j+1. */
+double ref_threshold_v(int bits, int j) {
+  const double *L = levels_of(bits);
+  return 0.5 * (L[j] + L[j + 1]);
+}
 
 double ref_level(int code) { return REF_LEVELS[code]; }
-
-/* Threshold j (0..6) is the midpoint between levels j and j+1. */
-double ref_threshold(int j) { return 0.5 * (REF_LEVELS[j] + REF_LEVELS[j + 1]); }
+double ref_threshold(int j) { return ref_threshold_v(3, j); }
 
 int ref_num_threads(void) {
 #ifdef _OPENMP
@@ -109,6 +130,30 @@ void ref_make_params(uint64_t seed, int d, int n_kv_heads, double *params, float
       }
 }
 
+/* PlanarQuant variant (a rotation by 2x2 blocks, SO(2)): params [n_kv_heads][d/2][2] =
+ * per block (cos phi, sin phi) with phi = 2 pi u, u uniform in [0, 1) from the top 53 bits
+ * of a SplitMix64 draw -- Haar on SO(2).  params32 (optional) receives binary32 copies. */
+void ref_make_params_so2(uint64_t seed, int d, int n_kv_heads, double *params,
+                         float *params32) {
+  const double two_m53 = 1.0 / 9007199254740992.0;
+  uint64_t state = seed;
+  for (int h = 0; h < n_kv_heads; h++)
+    for (int b = 0; b < d / 2; b++) {
+      double u = (double)(ref_splitmix64_next(&state) >> 11) * two_m53;
+      double phi = 2.0 * M_PI * u;
+      size_t idx = ((size_t)h * (d / 2) + b) * 2;
+      params[idx] = cos(phi);
+      params[idx + 1] = sin(phi);
+      if (params32) {
+        params32[idx] = (float)cos(phi);
+        params32[idx + 1] = (float)sin(phi);
+      }
+    }
+}
+
+/* Floats of rotation parameters per KV head: 2d for SO(4) quaternion pairs, d for SO(2). */
+int ref_params_per_head(int rot, int d) { return rot == 1 ? d : 2 * d; }
+
 /* ------------------------------------------------------------------------------ */
 /* Walsh-Hadamard transform, natural (Sylvester) order, orthonormal (1/sqrt(d)).    */
 /* The O(d log d) butterfly: at stride h, pairs (j, j+h) become (a+b, a-b).         */
@@ -162,22 +207,50 @@ void ref_so4_inverse(const double *p, const double *q, const double *z, double *
   ref_quat_mul(t, q, y);
 }
 
-/* Forward rotation of one d-vector with one head's params: WHT, then the d/4 blocks. */
-void ref_rotate(const double *params_head, const double *x, double *z, int d) {
+/* 2x2 block (dims 2b, 2b+1): z = [c -s; s c] y, and its inverse (transpose). */
+void ref_so2_forward(const double *cs, const double *y, double *z) {
+  z[0] = cs[0] * y[0] - cs[1] * y[1];
+  z[1] = cs[1] * y[0] + cs[0] * y[1];
+}
+
+void ref_so2_inverse(const double *cs, const double *z, double *y) {
+  y[0] = cs[0] * z[0] + cs[1] * z[1];
+  y[1] = -cs[1] * z[0] + cs[0] * z[1];
+}
+
+/* Forward rotation of one d-vector with one head's params: WHT, then the blocks
+ * (rot 0: d/4 SO(4) quaternion blocks; rot 1: d/2 SO(2) blocks). */
+void ref_rotate_v(int rot, const double *params_head, const double *x, double *z, int d) {
   double *y = (double *)malloc(sizeof(double) * d);
   memcpy(y, x, sizeof(double) * d);
   ref_wht(y, d);
-  for (int b = 0; b < d / 4; b++)
-    ref_so4_forward(params_head + b * 8, params_head + b * 8 + 4, y + 4 * b, z + 4 * b);
+  if (rot == 1) {
+    for (int b = 0; b < d / 2; b++) ref_so2_forward(params_head + 2 * b, y + 2 * b, z + 2 * b);
+  } else {
+    for (int b = 0; b < d / 4; b++)
+      ref_so4_forward(params_head + b * 8, params_head + b * 8 + 4, y + 4 * b, z + 4 * b);
+  }
   free(y);
 }
 
 /* Inverse rotation: inverse blocks, then the WHT (orthonormal and symmetric, so it is
  * its own inverse). */
-void ref_unrotate(const double *params_head, const double *z, double *x, int d) {
-  for (int b = 0; b < d / 4; b++)
-    ref_so4_inverse(params_head + b * 8, params_head + b * 8 + 4, z + 4 * b, x + 4 * b);
+void ref_unrotate_v(int rot, const double *params_head, const double *z, double *x, int d) {
+  if (rot == 1) {
+    for (int b = 0; b < d / 2; b++) ref_so2_inverse(params_head + 2 * b, z + 2 * b, x + 2 * b);
+  } else {
+    for (int b = 0; b < d / 4; b++)
+      ref_so4_inverse(params_head + b * 8, params_head + b * 8 + 4, z + 4 * b, x + 4 * b);
+  }
   ref_wht(x, d);
+}
+
+void ref_rotate(const double *params_head, const double *x, double *z, int d) {
+  ref_rotate_v(0, params_head, x, z, d);
+}
+
+void ref_unrotate(const double *params_head, const double *z, double *x, int d) {
+  ref_unrotate_v(0, params_head, z, x, d);
 }
 
 /* ------------------------------------------------------------------------------ */
@@ -214,31 +287,32 @@ double ref_fp16_value(uint16_t h) {
 }
 
 /* ------------------------------------------------------------------------------ */
-/* Quantise one vector: norm, WHT, SO(4) blocks, scalar quantisation.               */
+/* Quantise one vector: norm, WHT, rotation blocks, scalar quantisation.            */
 /* ------------------------------------------------------------------------------ */
-/* codes[i] in 0..7 (ascending level index); *norm16 = binary16 bits of the norm.
- * Returns 1 if the norm overflowed binary16 (stored as 65504), else 0.
+/* codes[i] in 0 .. 2^bits - 1 (ascending level index); *norm16 = binary16 bits of the
+ * norm.  Returns 1 if the norm overflowed binary16 (stored as 65504), else 0.
  * z_out (optional) receives the rotated coordinates z. */
-int ref_quantize_vector(const double *params_head, const double *x, int d, uint8_t *codes,
-                        uint16_t *norm16, double *z_out) {
+int ref_quantize_vector_v(int bits, int rot, const double *params_head, const double *x, int d,
+                          uint8_t *codes, uint16_t *norm16, double *z_out) {
   double ss = 0.0;
   for (int i = 0; i < d; i++) ss += x[i] * x[i];
   double n = sqrt(ss);
 
   double *z = (double *)malloc(sizeof(double) * d);
-  ref_rotate(params_head, x, z, d);
+  ref_rotate_v(rot, params_head, x, z, d);
 
   /* code_i = #{j : u_i >= t_j} with u_i = sqrt(d) z_i / n, compared as
    * sqrt(d) z_i >= n t_j.  A zero vector has no direction: u is taken as 0, which the
-   * tie rule sends to code 4 (the level just above 0). */
+   * tie rule sends to the level just above 0 (code 2^(bits-1)). */
   double sqd = sqrt((double)d);
+  int nl = 1 << bits;
   for (int i = 0; i < d; i++) {
     int c = 0;
     if (n == 0.0) {
-      c = 4;
+      c = nl / 2;
     } else {
-      for (int j = 0; j < 7; j++)
-        if (sqd * z[i] >= n * ref_threshold(j)) c++;
+      for (int j = 0; j < nl - 1; j++)
+        if (sqd * z[i] >= n * ref_threshold_v(bits, j)) c++;
     }
     codes[i] = (uint8_t)c;
   }
@@ -255,13 +329,59 @@ int ref_quantize_vector(const double *params_head, const double *x, int d, uint8
   return overflow;
 }
 
+int ref_quantize_vector(const double *params_head, const double *x, int d, uint8_t *codes,
+                        uint16_t *norm16, double *z_out) {
+  return ref_quantize_vector_v(3, 0, params_head, x, d, codes, norm16, z_out);
+}
+
 /* ------------------------------------------------------------------------------ */
-/* Packed code layout (3 bits per code, d/32 groups of 12 bytes per vector).        */
-/* Group g covers dims 32g..32g+31 and is three little-endian 32-bit words w0..w2:  */
+/* Packed code layouts (bits * d / 8 bytes per vector, little-endian 32-bit words).  */
+/* 3 bits: d/32 groups of three words w0..w2; group g covers dims 32g..32g+31:       */
 /*   dim 32g + 8j + k  (j = 0,1,2; k = 0..7): the code is bits 4k..4k+2 of w_j;       */
 /*   dim 32g + 24 + k  (k = 0..7): code bit (2 - b) is bit 4k+3 of w_b.              */
+/* 4 bits: word j holds dims 8j..8j+7, nibble k = dim 8j+k in sign-magnitude form:   */
+/*   code c >= 8 -> c - 8;  c < 8 -> 8 | (7 - c)  (bit 3 = negative level, bits 0-2 =  */
+/*   index of the level's magnitude, ascending).                                     */
+/* 2 bits: word j holds dims 16j..16j+15; 2-bit slot s (bits 2s, 2s+1) holds dim     */
+/*   16j + 2s (s < 4), 16j + 2(s-4) + 1 (4 <= s < 8), 16j + 8 + 2(s-8) (8 <= s < 12), */
+/*   16j + 9 + 2(s-12) (s >= 12); the code is the level index 0..3.                 */
 /* ------------------------------------------------------------------------------ */
-void ref_pack_codes(const uint8_t *codes, int d, uint8_t *out) {
+static int slot2_dim(int s) {
+  return s < 4 ? 2 * s : (s < 8 ? 2 * (s - 4) + 1 : (s < 12 ? 8 + 2 * (s - 8) : 9 + 2 * (s - 12)));
+}
+
+static void put_words(const uint32_t *w, int n, uint8_t *out) {
+  for (int j = 0; j < n; j++)
+    for (int byte = 0; byte < 4; byte++) out[4 * j + byte] = (uint8_t)(w[j] >> (8 * byte));
+}
+
+static uint32_t get_word(const uint8_t *in, int j) {
+  uint32_t w = 0;
+  for (int byte = 0; byte < 4; byte++) w |= (uint32_t)in[4 * j + byte] << (8 * byte);
+  return w;
+}
+
+void ref_pack_codes_v(int bits, const uint8_t *codes, int d, uint8_t *out) {
+  if (bits == 4) {
+    for (int j = 0; j < d / 8; j++) {
+      uint32_t w = 0;
+      for (int k = 0; k < 8; k++) {
+        uint32_t c = codes[8 * j + k] & 15u;
+        uint32_t nib = c >= 8 ? c - 8 : (8u | (7u - c));
+        w |= nib << (4 * k);
+      }
+      put_words(&w, 1, out + 4 * j);
+    }
+    return;
+  }
+  if (bits == 2) {
+    for (int j = 0; j < d / 16; j++) {
+      uint32_t w = 0;
+      for (int sl = 0; sl < 16; sl++) w |= (uint32_t)(codes[16 * j + slot2_dim(sl)] & 3u) << (2 * sl);
+      put_words(&w, 1, out + 4 * j);
+    }
+    return;
+  }
   for (int g = 0; g < d / 32; g++) {
     uint32_t w[3] = {0, 0, 0};
     for (int e = 0; e < 32; e++) {
@@ -274,20 +394,31 @@ void ref_pack_codes(const uint8_t *codes, int d, uint8_t *out) {
         for (int b = 0; b < 3; b++) w[b] |= ((c >> (2 - b)) & 1u) << (4 * k + 3);
       }
     }
-    for (int j = 0; j < 3; j++)
-      for (int byte = 0; byte < 4; byte++)
-        out[12 * g + 4 * j + byte] = (uint8_t)(w[j] >> (8 * byte));
+    put_words(w, 3, out + 12 * g);
   }
 }
 
-void ref_unpack_codes(const uint8_t *in, int d, uint8_t *codes) {
+void ref_unpack_codes_v(int bits, const uint8_t *in, int d, uint8_t *codes) {
+  if (bits == 4) {
+    for (int j = 0; j < d / 8; j++) {
+      uint32_t w = get_word(in, j);
+      for (int k = 0; k < 8; k++) {
+        uint32_t nib = (w >> (4 * k)) & 15u;
+        codes[8 * j + k] = (uint8_t)((nib & 8u) ? 7u - (nib & 7u) : 8u + nib);
+      }
+    }
+    return;
+  }
+  if (bits == 2) {
+    for (int j = 0; j < d / 16; j++) {
+      uint32_t w = get_word(in, j);
+      for (int sl = 0; sl < 16; sl++) codes[16 * j + slot2_dim(sl)] = (uint8_t)((w >> (2 * sl)) & 3u);
+    }
+    return;
+  }
   for (int g = 0; g < d / 32; g++) {
     uint32_t w[3];
-    for (int j = 0; j < 3; j++) {
-      w[j] = 0;
-      for (int byte = 0; byte < 4; byte++)
-        w[j] |= (uint32_t)in[12 * g + 4 * j + byte] << (8 * byte);
-    }
+    for (int j = 0; j < 3; j++) w[j] = get_word(in + 12 * g, j);
     for (int e = 0; e < 32; e++) {
       uint32_t c = 0;
       if (e < 24) {
@@ -301,31 +432,37 @@ void ref_unpack_codes(const uint8_t *in, int d, uint8_t *codes) {
   }
 }
 
+void ref_pack_codes(const uint8_t *codes, int d, uint8_t *out) { ref_pack_codes_v(3, codes, d, out); }
+void ref_unpack_codes(const uint8_t *in, int d, uint8_t *codes) { ref_unpack_codes_v(3, in, d, codes); }
+
 /* ------------------------------------------------------------------------------ */
 /* Paged cache: blocks[page][kv_head] of block_bytes; a block holds, for 64 (page)  */
-/* token slots: K codes [P][3d/8] | K norms [P] binary16 | V codes | V norms.        */
+/* token slots: K codes [P][cb] | K norms [P] binary16 | V codes | V norms, with     */
+/* cb = bits * d / 8 code bytes per vector.                                          */
 /* ------------------------------------------------------------------------------ */
-size_t ref_block_bytes(int d, int page) { return (size_t)2 * page * (3 * d / 8 + 2); }
+static size_t cbytes(int bits, int d) { return (size_t)bits * d / 8; }
 
-static size_t k_codes_off(int d, int page, int slot) { (void)page; return (size_t)slot * (3 * d / 8); }
-static size_t k_norm_off(int d, int page, int slot) {
-  return (size_t)page * (3 * d / 8) + 2 * (size_t)slot;
+size_t ref_block_bytes_v(int bits, int d, int page) { return (size_t)2 * page * (cbytes(bits, d) + 2); }
+size_t ref_block_bytes(int d, int page) { return ref_block_bytes_v(3, d, page); }
+
+static size_t k_codes_off(size_t cb, int page, int slot) { (void)page; return (size_t)slot * cb; }
+static size_t k_norm_off(size_t cb, int page, int slot) { return (size_t)page * cb + 2 * (size_t)slot; }
+static size_t v_codes_off(size_t cb, int page, int slot) {
+  return (size_t)page * (cb + 2) + (size_t)slot * cb;
 }
-static size_t v_codes_off(int d, int page, int slot) {
-  return (size_t)page * (3 * d / 8 + 2) + (size_t)slot * (3 * d / 8);
-}
-static size_t v_norm_off(int d, int page, int slot) {
-  return (size_t)page * (3 * d / 8 + 2) + (size_t)page * (3 * d / 8) + 2 * (size_t)slot;
+static size_t v_norm_off(size_t cb, int page, int slot) {
+  return (size_t)page * (cb + 2) + (size_t)page * cb + 2 * (size_t)slot;
 }
 
 /* Quantise n_tokens tokens of K and V ([n_tokens][n_kv_heads][d], fp64) into the paged
- * cache at (seq_ids[t], positions[t]).  params: fp64 [n_kv_heads][d/4][2][4].
- * Returns the number of norms that saturated. */
-int ref_quantize_append(const double *params, int d, int n_kv_heads, int page,
-                        uint8_t *blocks, const int32_t *page_table, int max_pages_per_seq,
-                        const double *K, const double *V, int n_tokens,
-                        const int32_t *seq_ids, const int32_t *positions) {
-  size_t bb = ref_block_bytes(d, page);
+ * cache at (seq_ids[t], positions[t]).  params: fp64, ref_params_per_head(rot, d) per
+ * head.  Returns the number of norms that saturated. */
+int ref_quantize_append_v(int bits, int rot, const double *params, int d, int n_kv_heads,
+                          int page, uint8_t *blocks, const int32_t *page_table,
+                          int max_pages_per_seq, const double *K, const double *V, int n_tokens,
+                          const int32_t *seq_ids, const int32_t *positions) {
+  size_t bb = ref_block_bytes_v(bits, d, page), cb = cbytes(bits, d);
+  int pph = ref_params_per_head(rot, d);
   int overflow = 0;
 #pragma omp parallel for schedule(static) reduction(+ : overflow)
   for (int t = 0; t < n_tokens; t++) {
@@ -335,14 +472,14 @@ int ref_quantize_append(const double *params, int d, int n_kv_heads, int page,
       int phys = page_table[(size_t)seq_ids[t] * max_pages_per_seq + pos / page];
       int slot = pos % page;
       uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + h) * bb;
-      const double *ph = params + (size_t)h * (d / 4) * 8;
+      const double *ph = params + (size_t)h * pph;
       for (int kv = 0; kv < 2; kv++) {
         const double *x = (kv == 0 ? K : V) + ((size_t)t * n_kv_heads + h) * d;
         uint16_t n16;
-        overflow += ref_quantize_vector(ph, x, d, codes, &n16, NULL);
-        uint8_t *dst = blk + (kv == 0 ? k_codes_off(d, page, slot) : v_codes_off(d, page, slot));
-        ref_pack_codes(codes, d, dst);
-        uint8_t *nd = blk + (kv == 0 ? k_norm_off(d, page, slot) : v_norm_off(d, page, slot));
+        overflow += ref_quantize_vector_v(bits, rot, ph, x, d, codes, &n16, NULL);
+        uint8_t *dst = blk + (kv == 0 ? k_codes_off(cb, page, slot) : v_codes_off(cb, page, slot));
+        ref_pack_codes_v(bits, codes, d, dst);
+        uint8_t *nd = blk + (kv == 0 ? k_norm_off(cb, page, slot) : v_norm_off(cb, page, slot));
         nd[0] = (uint8_t)(n16 & 0xff);
         nd[1] = (uint8_t)(n16 >> 8);
       }
@@ -351,34 +488,51 @@ int ref_quantize_append(const double *params, int d, int n_kv_heads, int page,
   return overflow;
 }
 
+int ref_quantize_append(const double *params, int d, int n_kv_heads, int page,
+                        uint8_t *blocks, const int32_t *page_table, int max_pages_per_seq,
+                        const double *K, const double *V, int n_tokens,
+                        const int32_t *seq_ids, const int32_t *positions) {
+  return ref_quantize_append_v(3, 0, params, d, n_kv_heads, page, blocks, page_table,
+                               max_pages_per_seq, K, V, n_tokens, seq_ids, positions);
+}
+
 /* Dequantised vector in the rotated space: (stored norm / sqrt(d)) * level[code]. */
-static void dequant_rotated(const uint8_t *packed, const uint8_t *norm_bytes, int d, double *out) {
+static void dequant_rotated(int bits, const uint8_t *packed, const uint8_t *norm_bytes, int d,
+                            double *out) {
   uint8_t codes[1024];
-  ref_unpack_codes(packed, d, codes);
+  ref_unpack_codes_v(bits, packed, d, codes);
   uint16_t n16 = (uint16_t)(norm_bytes[0] | (norm_bytes[1] << 8));
   double s = ref_fp16_value(n16) / sqrt((double)d);
-  for (int i = 0; i < d; i++) out[i] = s * REF_LEVELS[codes[i]];
+  const double *L = levels_of(bits);
+  for (int i = 0; i < d; i++) out[i] = s * L[codes[i]];
 }
 
 /* Materialise one cached vector back in the input space (K-hat or V-hat): inverse
  * rotation of the dequantised rotated vector.  kind 0 = K, 1 = V.  Used by tests to
  * check that attention in the rotated space equals attention over K-hat, V-hat. */
-void ref_dequantize_slot(const double *params, int d, int n_kv_heads, int page,
-                         const uint8_t *blocks, int phys_page, int kv_head, int slot, int kind,
-                         double *out) {
-  size_t bb = ref_block_bytes(d, page);
+void ref_dequantize_slot_v(int bits, int rot, const double *params, int d, int n_kv_heads,
+                           int page, const uint8_t *blocks, int phys_page, int kv_head, int slot,
+                           int kind, double *out) {
+  size_t bb = ref_block_bytes_v(bits, d, page), cb = cbytes(bits, d);
   const uint8_t *blk = blocks + ((size_t)phys_page * n_kv_heads + kv_head) * bb;
   double zr[1024];
   if (kind == 0)
-    dequant_rotated(blk + k_codes_off(d, page, slot), blk + k_norm_off(d, page, slot), d, zr);
+    dequant_rotated(bits, blk + k_codes_off(cb, page, slot), blk + k_norm_off(cb, page, slot), d, zr);
   else
-    dequant_rotated(blk + v_codes_off(d, page, slot), blk + v_norm_off(d, page, slot), d, zr);
-  ref_unrotate(params + (size_t)kv_head * (d / 4) * 8, zr, out, d);
+    dequant_rotated(bits, blk + v_codes_off(cb, page, slot), blk + v_norm_off(cb, page, slot), d, zr);
+  ref_unrotate_v(rot, params + (size_t)kv_head * ref_params_per_head(rot, d), zr, out, d);
+}
+
+void ref_dequantize_slot(const double *params, int d, int n_kv_heads, int page,
+                         const uint8_t *blocks, int phys_page, int kv_head, int slot, int kind,
+                         double *out) {
+  ref_dequantize_slot_v(3, 0, params, d, n_kv_heads, page, blocks, phys_page, kv_head, slot,
+                        kind, out);
 }
 
 /* ------------------------------------------------------------------------------ */
 /* Decode attention on the packed cache, all in the rotated space.                  */
-/*   a6: q~ = R q (same WHT + SO(4) as the KV head's keys);                          */
+/*   a6: q~ = R q (same WHT + blocks as the KV head's keys);                         */
 /*   a7: s_t = scale * q~ . k~_t,  k~_t = (n_t / sqrt d) L[c_t];                      */
 /*   a8: softmax over t = 0..len-1 and o~ = sum_t p_t v~_t;                          */
 /*   a9: out = R^T o~.                                                               */
@@ -386,13 +540,14 @@ void ref_dequantize_slot(const double *params, int d, int n_kv_heads, int page,
 /* The (sequence, head) pairs listed in sel (pairs of ints; n_sel of them; NULL =    */
 /* all) are the ones computed; others in out are left untouched.                     */
 /* ------------------------------------------------------------------------------ */
-void ref_decode_attention(const double *params, int d, int n_kv_heads, int page,
-                          const uint8_t *blocks, const int32_t *page_table,
-                          int max_pages_per_seq, int n_seqs, int n_q_heads,
-                          const int32_t *seq_lens, const double *Q, double scale, double *out,
-                          const int32_t *sel, int n_sel) {
+void ref_decode_attention_v(int bits, int rot, const double *params, int d, int n_kv_heads,
+                            int page, const uint8_t *blocks, const int32_t *page_table,
+                            int max_pages_per_seq, int n_seqs, int n_q_heads,
+                            const int32_t *seq_lens, const double *Q, double scale, double *out,
+                            const int32_t *sel, int n_sel) {
   int G = n_q_heads / n_kv_heads;
-  size_t bb = ref_block_bytes(d, page);
+  size_t bb = ref_block_bytes_v(bits, d, page), cb = cbytes(bits, d);
+  int pph = ref_params_per_head(rot, d);
   int total = sel ? n_sel : n_seqs * n_q_heads;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int w = 0; w < total; w++) {
@@ -400,21 +555,21 @@ void ref_decode_attention(const double *params, int d, int n_kv_heads, int page,
     int h = sel ? sel[2 * w + 1] : w % n_q_heads;
     int kvh = h / G;
     int len = seq_lens[s];
-    const double *ph = params + (size_t)kvh * (d / 4) * 8;
+    const double *ph = params + (size_t)kvh * pph;
     double *o = out + ((size_t)s * n_q_heads + h) * d;
     if (len <= 0) {
       for (int i = 0; i < d; i++) o[i] = 0.0;
       continue;
     }
     double qt[1024], kt[1024], vt[1024], ot[1024];
-    ref_rotate(ph, Q + ((size_t)s * n_q_heads + h) * d, qt, d);
+    ref_rotate_v(rot, ph, Q + ((size_t)s * n_q_heads + h) * d, qt, d);
 
     double *sc = (double *)malloc(sizeof(double) * len);
     for (int t = 0; t < len; t++) {
       int phys = page_table[(size_t)s * max_pages_per_seq + t / page];
       const uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + kvh) * bb;
-      dequant_rotated(blk + k_codes_off(d, page, t % page), blk + k_norm_off(d, page, t % page),
-                      d, kt);
+      dequant_rotated(bits, blk + k_codes_off(cb, page, t % page),
+                      blk + k_norm_off(cb, page, t % page), d, kt);
       double dot = 0.0;
       for (int i = 0; i < d; i++) dot += qt[i] * kt[i];
       sc[t] = scale * dot;
@@ -429,14 +584,24 @@ void ref_decode_attention(const double *params, int d, int n_kv_heads, int page,
       l += p;
       int phys = page_table[(size_t)s * max_pages_per_seq + t / page];
       const uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + kvh) * bb;
-      dequant_rotated(blk + v_codes_off(d, page, t % page), blk + v_norm_off(d, page, t % page),
-                      d, vt);
+      dequant_rotated(bits, blk + v_codes_off(cb, page, t % page),
+                      blk + v_norm_off(cb, page, t % page), d, vt);
       for (int i = 0; i < d; i++) ot[i] += p * vt[i];
     }
     for (int i = 0; i < d; i++) ot[i] /= l;
     free(sc);
-    ref_unrotate(ph, ot, o, d);
+    ref_unrotate_v(rot, ph, ot, o, d);
   }
+}
+
+void ref_decode_attention(const double *params, int d, int n_kv_heads, int page,
+                          const uint8_t *blocks, const int32_t *page_table,
+                          int max_pages_per_seq, int n_seqs, int n_q_heads,
+                          const int32_t *seq_lens, const double *Q, double scale, double *out,
+                          const int32_t *sel, int n_sel) {
+  ref_decode_attention_v(3, 0, params, d, n_kv_heads, page, blocks, page_table,
+                         max_pages_per_seq, n_seqs, n_q_heads, seq_lens, Q, scale, out, sel,
+                         n_sel);
 }
 
 /* Full-precision attention (no quantisation, no rotation) for the error-bound tests:
@@ -478,15 +643,18 @@ void ref_attention_full(int d, int n_kv_heads, int n_q_heads, int n_tokens, cons
  * params) and report, per element, the distance of u = sqrt(d) z / n to the nearest
  * threshold (N(0,1) units; +inf for a zero vector).  codes [n_rows][H][d],
  * norms [n_rows][H] (binary16 bits), dist [n_rows][H][d] (may be NULL). */
-void ref_quantize_rows(const double *params, int d, int n_kv_heads, const double *X, int n_rows,
-                       uint8_t *codes, uint16_t *norms, double *dist) {
+void ref_quantize_rows_v(int bits, int rot, const double *params, int d, int n_kv_heads,
+                         const double *X, int n_rows, uint8_t *codes, uint16_t *norms,
+                         double *dist) {
+  int pph = ref_params_per_head(rot, d);
+  int nt = (1 << bits) - 1;
 #pragma omp parallel for schedule(static)
   for (int r = 0; r < n_rows; r++) {
     double z[1024];
     for (int h = 0; h < n_kv_heads; h++) {
       size_t v = (size_t)r * n_kv_heads + h;
       const double *x = X + v * d;
-      ref_quantize_vector(params + (size_t)h * (d / 4) * 8, x, d, codes + v * d, norms + v, z);
+      ref_quantize_vector_v(bits, rot, params + (size_t)h * pph, x, d, codes + v * d, norms + v, z);
       if (!dist) continue;
       double ss = 0.0;
       for (int i = 0; i < d; i++) ss += x[i] * x[i];
@@ -495,8 +663,8 @@ void ref_quantize_rows(const double *params, int d, int n_kv_heads, const double
         double best = INFINITY;
         if (n > 0.0) {
           double u = sqrt((double)d) * z[i] / n;
-          for (int j = 0; j < 7; j++) {
-            double e = fabs(u - ref_threshold(j));
+          for (int j = 0; j < nt; j++) {
+            double e = fabs(u - ref_threshold_v(bits, j));
             if (e < best) best = e;
           }
         }
@@ -506,8 +674,17 @@ void ref_quantize_rows(const double *params, int d, int n_kv_heads, const double
   }
 }
 
-/* Unpack n records of packed codes (3d/8 bytes each, contiguous) into codes [n][d]. */
-void ref_unpack_codes_batch(const uint8_t *in, int d, long n, uint8_t *codes) {
+void ref_quantize_rows(const double *params, int d, int n_kv_heads, const double *X, int n_rows,
+                       uint8_t *codes, uint16_t *norms, double *dist) {
+  ref_quantize_rows_v(3, 0, params, d, n_kv_heads, X, n_rows, codes, norms, dist);
+}
+
+/* Unpack n records of packed codes (bits * d / 8 bytes each, contiguous) into codes [n][d]. */
+void ref_unpack_codes_batch_v(int bits, const uint8_t *in, int d, long n, uint8_t *codes) {
 #pragma omp parallel for schedule(static)
-  for (long i = 0; i < n; i++) ref_unpack_codes(in + i * (3 * d / 8), d, codes + i * d);
+  for (long i = 0; i < n; i++) ref_unpack_codes_v(bits, in + i * cbytes(bits, d), d, codes + i * d);
+}
+
+void ref_unpack_codes_batch(const uint8_t *in, int d, long n, uint8_t *codes) {
+  ref_unpack_codes_batch_v(3, in, d, n, codes);
 }

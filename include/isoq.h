@@ -90,7 +90,8 @@ int isoq_params_generate(uint64_t seed, int d, int n_kv_heads, float* host_out);
  * Errors: as isoq_params_generate, plus ISOQ_E_DEVICE / ISOQ_E_CUDA. */
 int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out);
 
-/* Copies the binary32 parameters ([n_kv_heads][d/4][2][4]) to host_dst. */
+/* Copies the binary32 parameters ([n_kv_heads][d/4][2][4]; see the variants below for
+ * SO(2) handles) to host_dst. */
 int isoq_params_copy(const isoq_params* params, float* host_dst);
 
 /* d and n_kv_heads of a handle (either pointer may be NULL). */
@@ -98,6 +99,54 @@ int isoq_params_shape(const isoq_params* params, int* d, int* n_kv_heads);
 
 /* Frees the device copy and the handle.  NULL is ignored. */
 void isoq_params_destroy(isoq_params* params);
+
+/* =======================================================================================
+ * Format variants of the same family.
+ *
+ * "RotaryQuant ...", Abstract, places IsoQuant in a family of 3-4 bit methods and names a
+ * planar variant, PlanarQuant, without defining it.  This library offers:
+ *   - bits: 3 (the method), or 2 / 4 bits per code with the 4- and 16-level Lloyd-Max
+ *     quantisers for N(0,1) (J. Max 1960, Table I):
+ *       2 bits: L = {-1.5104, -0.4528, 0.4528, 1.5104}
+ *       4 bits: L = +-{0.1284, 0.3881, 0.6568, 0.9424, 1.2562, 1.6180, 2.0690, 2.7326};
+ *     thresholds are midpoints, ties take the upper code, a zero vector codes 2^(bits-1);
+ *     2 and 4 bits need d = 128 (ISOQ_E_DIM otherwise).
+ *   - rotation: ISOQ_ROT_SO4 (the method: quaternion-pair blocks as above) or
+ *     ISOQ_ROT_SO2 (PlanarQuant read as 2x2 blocks): after the same WHT, dims (2b, 2b+1)
+ *     are rotated by [cos phi_b, -sin phi_b; sin phi_b, cos phi_b], phi_b = 2 pi u with u
+ *     the top 53 bits of one SplitMix64 draw (seeded with `seed`, head-major) times 2^-53
+ *     (Haar on SO(2)); parameters [n_kv_heads][d/2][2] = (cos, sin) rounded to binary32,
+ *     d floats per head.
+ * Packed codes (bits * d / 8 bytes per vector, little-endian 32-bit words):
+ *   3 bits: the layout of the paged-cache section below;
+ *   4 bits: word j holds dims 8j..8j+7, nibble k = dim 8j+k in sign-magnitude form: code
+ *     c >= 8 -> c - 8, c < 8 -> 8 | (7 - c) (bit 3 = negative level, bits 0-2 the index of
+ *     the level's magnitude);
+ *   2 bits: word j holds dims 16j..16j+15, 2-bit slot s (bits 2s, 2s+1) holding dim
+ *     16j + 2s (s < 4), 16j + 2(s-4) + 1 (s < 8), 16j + 8 + 2(s-8) (s < 12) or
+ *     16j + 9 + 2(s-12), code = level index 0..3.
+ * Every other call takes its format from the params handle; a cache (isoq_cache.bits
+ * equal to the handle's bits) holds blocks of isoq_block_bytes_v(d, bits, 64) bytes.
+ * ===================================================================================== */
+#define ISOQ_ROT_SO4 0
+#define ISOQ_ROT_SO2 1
+
+/* Host only: the parameters of `rotation` (SO4: [H][d/4][2][4]; SO2: [H][d/2][2]). */
+int isoq_params_generate_v(uint64_t seed, int d, int n_kv_heads, int rotation,
+                           float* host_out);
+
+/* As isoq_make_params with a format.  Errors: ISOQ_E_ARG (unknown rotation), ISOQ_E_DIM
+ * (d, or bits not 2/3/4, or 2/4 bits with d != 128), ISOQ_E_DEVICE, ISOQ_E_CUDA.
+ * isoq_make_params(seed, d, H, out) = isoq_make_params_v(seed, d, H, 3, ISOQ_ROT_SO4, out). */
+int isoq_make_params_v(uint64_t seed, int d, int n_kv_heads, int bits, int rotation,
+                       isoq_params** out);
+
+/* bits and rotation of a handle (either pointer may be NULL).  isoq_params_copy writes
+ * the rotation's parameter layout (d floats per head for SO2). */
+int isoq_params_format(const isoq_params* params, int* bits, int* rotation);
+
+/* Bytes of one (page, KV head) block: 2 * page_size * (bits * d / 8 + 2); 0 if unsupported. */
+size_t isoq_block_bytes_v(int d, int bits, int page_size);
 
 /* =======================================================================================
  * Paged cache.
@@ -132,6 +181,8 @@ typedef struct isoq_cache {
   uint8_t* blocks;           /* device */
   const int32_t* page_table; /* device */
   uint32_t* status;          /* device, optional */
+  int bits;                  /* bits per code of the blocks (0 = 3, the method); must
+                                equal the params' bits, else ISOQ_E_DIM */
 } isoq_cache;
 
 /* Bytes of one (page, KV head) block: 2 * page_size * (3d/8 + 2); 0 if unsupported. */

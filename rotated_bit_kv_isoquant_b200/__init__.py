@@ -40,6 +40,7 @@ ISOQ_ST_NORM_SAT = 0x8
 ISOQ_ST_LEN_RANGE = 0x10
 
 ISOQ_F32, ISOQ_BF16, ISOQ_F16 = 0, 1, 2
+ISOQ_ROT_SO4, ISOQ_ROT_SO2 = 0, 1
 ISOQ_PAGE_SIZE = 64
 ISOQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -57,7 +58,8 @@ class isoq_cache(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("n_kv_heads", ctypes.c_int), ("page_size", ctypes.c_int),
                 ("n_pages", ctypes.c_int), ("max_pages_per_seq", ctypes.c_int),
                 ("n_seqs", ctypes.c_int), ("blocks", ctypes.c_void_p),
-                ("page_table", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+                ("page_table", ctypes.c_void_p), ("status", ctypes.c_void_p),
+                ("bits", ctypes.c_int)]
 
 
 _p, _i, _sz, _u64, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_float
@@ -65,6 +67,10 @@ _cp = ctypes.POINTER(isoq_cache)
 
 _SIGS = {
     "isoq_params_generate": (_i, [_u64, _i, _i, _p]),
+    "isoq_params_generate_v": (_i, [_u64, _i, _i, _i, _p]),
+    "isoq_make_params_v": (_i, [_u64, _i, _i, _i, _i, ctypes.POINTER(_p)]),
+    "isoq_params_format": (_i, [_p, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "isoq_block_bytes_v": (_sz, [_i, _i, _i]),
     "isoq_make_params": (_i, [_u64, _i, _i, ctypes.POINTER(_p)]),
     "isoq_params_copy": (_i, [_p, _p]),
     "isoq_params_shape": (_i, [_p, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
@@ -127,20 +133,30 @@ def _stream_ptr(stream):
 # ------------------------------------------------------------------------------------
 # Parameters
 # ------------------------------------------------------------------------------------
-def isoq_params_generate(seed: int, d: int, n_kv_heads: int) -> np.ndarray:
-    """Host-side rotation parameters, float32 [n_kv_heads][d/4][2][4] (no GPU needed)."""
-    out = np.zeros((n_kv_heads, d // 4, 2, 4), dtype=np.float32)
-    _check(_lib.isoq_params_generate(seed, d, n_kv_heads, out.ctypes.data), "isoq_params_generate")
+def _params_shape(d: int, n_kv_heads: int, rotation: int):
+    return (n_kv_heads, d // 2, 2) if rotation == ISOQ_ROT_SO2 else (n_kv_heads, d // 4, 2, 4)
+
+
+def isoq_params_generate(seed: int, d: int, n_kv_heads: int,
+                         rotation: int = ISOQ_ROT_SO4) -> np.ndarray:
+    """Host-side rotation parameters, float32 [n_kv_heads][d/4][2][4] (SO(4) quaternion
+    pairs) or [n_kv_heads][d/2][2] (SO(2) cos, sin); no GPU needed."""
+    out = np.zeros(_params_shape(d, n_kv_heads, rotation), dtype=np.float32)
+    _check(_lib.isoq_params_generate_v(seed, d, n_kv_heads, rotation, out.ctypes.data),
+           "isoq_params_generate_v")
     return out
 
 
 class Params:
     """Owning wrapper of an ``isoq_params*`` handle."""
 
-    def __init__(self, handle: int, d: int, n_kv_heads: int):
+    def __init__(self, handle: int, d: int, n_kv_heads: int, bits: int = 3,
+                 rotation: int = ISOQ_ROT_SO4):
         self.handle = handle
         self.d = d
         self.n_kv_heads = n_kv_heads
+        self.bits = bits
+        self.rotation = rotation
 
     def __del__(self):
         h, self.handle = getattr(self, "handle", None), None
@@ -148,14 +164,24 @@ class Params:
             _lib.isoq_params_destroy(h)
 
 
-def isoq_make_params(seed: int, d: int, n_kv_heads: int) -> Params:
+def isoq_make_params(seed: int, d: int, n_kv_heads: int, bits: int = 3,
+                     rotation: int = ISOQ_ROT_SO4) -> Params:
+    """Parameters of the method (3 bits, SO(4) blocks) or of a format variant."""
     h = _p()
-    _check(_lib.isoq_make_params(seed, d, n_kv_heads, ctypes.byref(h)), "isoq_make_params")
-    return Params(h.value, d, n_kv_heads)
+    _check(_lib.isoq_make_params_v(seed, d, n_kv_heads, bits, rotation, ctypes.byref(h)),
+           "isoq_make_params_v")
+    return Params(h.value, d, n_kv_heads, bits, rotation)
+
+
+def isoq_params_format(params: Params):
+    b, r = _i(), _i()
+    _check(_lib.isoq_params_format(params.handle, ctypes.byref(b), ctypes.byref(r)),
+           "isoq_params_format")
+    return b.value, r.value
 
 
 def isoq_params_copy(params: Params) -> np.ndarray:
-    out = np.zeros((params.n_kv_heads, params.d // 4, 2, 4), dtype=np.float32)
+    out = np.zeros(_params_shape(params.d, params.n_kv_heads, params.rotation), dtype=np.float32)
     _check(_lib.isoq_params_copy(params.handle, out.ctypes.data), "isoq_params_copy")
     return out
 
@@ -176,18 +202,19 @@ def isoq_params_destroy(params: Params) -> None:
 # ------------------------------------------------------------------------------------
 # Cache
 # ------------------------------------------------------------------------------------
-def isoq_block_bytes(d: int, page_size: int = ISOQ_PAGE_SIZE) -> int:
-    return int(_lib.isoq_block_bytes(d, page_size))
+def isoq_block_bytes(d: int, page_size: int = ISOQ_PAGE_SIZE, bits: int = 3) -> int:
+    return int(_lib.isoq_block_bytes_v(d, bits, page_size))
 
 
 class PagedCache:
     """Device memory of a paged cache (torch tensors) plus its ``isoq_cache`` view."""
 
-    def __init__(self, d: int, n_kv_heads: int, n_pages: int, page_table, device=None):
+    def __init__(self, d: int, n_kv_heads: int, n_pages: int, page_table, device=None,
+                 bits: int = 3):
         import torch
         device = device or torch.device("cuda")
-        self.d, self.n_kv_heads, self.n_pages = d, n_kv_heads, n_pages
-        bb = isoq_block_bytes(d)
+        self.d, self.n_kv_heads, self.n_pages, self.bits = d, n_kv_heads, n_pages, bits
+        bb = isoq_block_bytes(d, bits=bits)
         if bb == 0:
             raise IsoqError(ISOQ_E_DIM, "PagedCache")
         self.blocks = torch.zeros((n_pages, n_kv_heads, bb), dtype=torch.uint8, device=device)
@@ -195,7 +222,7 @@ class PagedCache:
         self.status = torch.zeros((1,), dtype=torch.int32, device=device)
         self._c = isoq_cache(d, n_kv_heads, ISOQ_PAGE_SIZE, n_pages, self.page_table.shape[1],
                              self.page_table.shape[0], self.blocks.data_ptr(),
-                             self.page_table.data_ptr(), self.status.data_ptr())
+                             self.page_table.data_ptr(), self.status.data_ptr(), bits)
 
     @property
     def c(self) -> isoq_cache:

@@ -53,13 +53,14 @@ class CacheSlice:
     def __init__(self, cache: PagedCache, page_table):
         from . import isoq_cache
         self.d, self.n_kv_heads, self.n_pages = cache.d, cache.n_kv_heads, cache.n_pages
+        self.bits = getattr(cache, "bits", 3)
         self.blocks, self.status = cache.blocks, cache.status
         self.page_table = page_table.to(device=cache.blocks.device,
                                         dtype=page_table.dtype).int().contiguous()
         self._c = isoq_cache(cache.d, cache.n_kv_heads, ISOQ_PAGE_SIZE, cache.n_pages,
                              self.page_table.shape[1], self.page_table.shape[0],
                              cache.blocks.data_ptr(), self.page_table.data_ptr(),
-                             cache.status.data_ptr())
+                             cache.status.data_ptr(), self.bits)
 
     @property
     def c(self):

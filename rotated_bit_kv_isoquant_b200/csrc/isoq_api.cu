@@ -15,10 +15,13 @@
 struct isoq_params {
   int d;
   int n_kv_heads;
+  int bits;                 // 2, 3 or 4 bits per code
+  int rotation;             // ISOQ_ROT_SO4 or ISOQ_ROT_SO2
   int device;
-  float* dev;               // [n_kv_heads][d/4][2][4] quaternions (the 256 parameters/head)
-  float* dev_mat;           // [n_kv_heads][d/4][4][4] derived: matrix of y -> p y conj(q)
-  std::vector<float> host;  // quaternions, same values as dev
+  float* dev;               // the parameters as generated (SO(4): [H][d/4][2][4] quaternions,
+                            // the 256 parameters/head; SO(2): [H][d/2][2] cos, sin)
+  float* dev_mat;           // [n_kv_heads][d/4][4][4] derived: each 4-dim block's matrix
+  std::vector<float> host;  // same values as dev
 };
 
 namespace {
@@ -31,6 +34,8 @@ int cuda_fail(cudaError_t e) {
 }
 
 bool supported_d(int d) { return d == 128 || d == 256; }
+// 3 bits at d = 128 and 256; the 2- and 4-bit variants at d = 128.
+bool supported_format(int d, int bits) { return bits == 3 || ((bits == 2 || bits == 4) && d == 128); }
 
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014).
 uint64_t splitmix64(uint64_t& state) {
@@ -118,6 +123,7 @@ int check_cache(const isoq_cache* c, const isoq_params* p) {
   if (!c->blocks || !c->page_table) return ISOQ_E_ARG;
   if (c->page_size != ISOQ_PAGE_SIZE || !supported_d(c->d)) return ISOQ_E_DIM;
   if (c->d != p->d || c->n_kv_heads != p->n_kv_heads) return ISOQ_E_DIM;
+  if ((c->bits == 0 ? 3 : c->bits) != p->bits) return ISOQ_E_DIM;
   if (c->n_pages < 0 || c->max_pages_per_seq < 1 || c->n_seqs < 1 || c->n_kv_heads < 1)
     return ISOQ_E_ARG;
   return ISOQ_OK;
@@ -140,6 +146,23 @@ bool valid_dtype(int t) { return t == ISOQ_F32 || t == ISOQ_BF16 || t == ISOQ_F1
 
 extern "C" {
 
+int isoq_params_generate_v(uint64_t seed, int d, int n_kv_heads, int rotation,
+                           float* host_out) {
+  if (rotation != ISOQ_ROT_SO2) return isoq_params_generate(seed, d, n_kv_heads, host_out);
+  if (!host_out || n_kv_heads < 1) return ISOQ_E_ARG;
+  if (!supported_d(d)) return ISOQ_E_DIM;
+  // Haar on SO(2): phi = 2 pi u, u from the top 53 bits of one SplitMix64 draw
+  const double two_m53 = 1.0 / 9007199254740992.0;
+  const double two_pi = 2.0 * 3.14159265358979323846;
+  uint64_t state = seed;
+  for (size_t b = 0; b < (size_t)n_kv_heads * (d / 2); ++b) {
+    const double phi = two_pi * (double)(splitmix64(state) >> 11) * two_m53;
+    host_out[2 * b] = (float)cos(phi);
+    host_out[2 * b + 1] = (float)sin(phi);
+  }
+  return ISOQ_OK;
+}
+
 int isoq_params_generate(uint64_t seed, int d, int n_kv_heads, float* host_out) {
   if (!host_out || n_kv_heads < 1) return ISOQ_E_ARG;
   if (!supported_d(d)) return ISOQ_E_DIM;
@@ -160,18 +183,22 @@ int isoq_params_generate(uint64_t seed, int d, int n_kv_heads, float* host_out) 
   return ISOQ_OK;
 }
 
-int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
+int isoq_make_params_v(uint64_t seed, int d, int n_kv_heads, int bits, int rotation,
+                       isoq_params** out) {
   if (!out) return ISOQ_E_ARG;
   *out = nullptr;
   if (n_kv_heads < 1) return ISOQ_E_ARG;
-  if (!supported_d(d)) return ISOQ_E_DIM;
+  if (rotation != ISOQ_ROT_SO4 && rotation != ISOQ_ROT_SO2) return ISOQ_E_ARG;
+  if (!supported_d(d) || !supported_format(d, bits)) return ISOQ_E_DIM;
   isoq_params* p = new isoq_params();
   p->d = d;
   p->n_kv_heads = n_kv_heads;
+  p->bits = bits;
+  p->rotation = rotation;
   p->dev = nullptr;
   p->dev_mat = nullptr;
-  p->host.resize((size_t)n_kv_heads * d * 2);
-  isoq_params_generate(seed, d, n_kv_heads, p->host.data());
+  p->host.resize((size_t)n_kv_heads * (rotation == ISOQ_ROT_SO2 ? d : 2 * d));
+  isoq_params_generate_v(seed, d, n_kv_heads, rotation, p->host.data());
   cudaError_t e = cudaGetDevice(&p->device);
   if (e != cudaSuccess) {
     g_last_cuda_error = (int)e;
@@ -179,20 +206,33 @@ int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
     delete p;
     return ISOQ_E_DEVICE;
   }
-  // Derived copy for the quantiser: each block rotation as a 4x4 row-major matrix, column j
-  // = p * e_j * conj(q), computed in binary64 from the binary32 quaternions.
+  // Derived copy used by every kernel: each 4-dim block's rotation as a 4x4 row-major
+  // matrix, computed in binary64 from the binary32 parameters.  SO(4): column j =
+  // p * e_j * conj(q).  SO(2): two 2x2 blocks [c -s; s c] on the diagonal.
   const size_t nq = p->host.size();
-  std::vector<float> mats((size_t)n_kv_heads * (d / 4) * 16);
+  std::vector<float> mats((size_t)n_kv_heads * (d / 4) * 16, 0.f);
   for (size_t blk = 0; blk < (size_t)n_kv_heads * (d / 4); ++blk) {
+    float* M = mats.data() + blk * 16;
+    if (rotation == ISOQ_ROT_SO2) {
+      for (int half = 0; half < 2; ++half) {
+        const float* cs = p->host.data() + (2 * blk + half) * 2;
+        const int o = 2 * half;
+        M[o * 4 + o] = cs[0];
+        M[o * 4 + o + 1] = -cs[1];
+        M[(o + 1) * 4 + o] = cs[1];
+        M[(o + 1) * 4 + o + 1] = cs[0];
+      }
+      continue;
+    }
     const float* pq = p->host.data() + blk * 8;
     const double P[4] = {pq[0], pq[1], pq[2], pq[3]};
     const double Qc[4] = {pq[4], -(double)pq[5], -(double)pq[6], -(double)pq[7]};
     for (int j = 0; j < 4; ++j) {
-      double e[4] = {0, 0, 0, 0}, tq[4], z[4];
-      e[j] = 1.0;
-      hamilton(P, e, tq);
+      double ev[4] = {0, 0, 0, 0}, tq[4], z[4];
+      ev[j] = 1.0;
+      hamilton(P, ev, tq);
       hamilton(tq, Qc, z);
-      for (int i = 0; i < 4; ++i) mats[blk * 16 + i * 4 + j] = (float)z[i];
+      for (int i = 0; i < 4; ++i) M[i * 4 + j] = (float)z[i];
     }
   }
   const size_t bytes = (nq + mats.size()) * sizeof(float);
@@ -209,6 +249,17 @@ int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
     return cuda_fail(e);
   }
   *out = p;
+  return ISOQ_OK;
+}
+
+int isoq_make_params(uint64_t seed, int d, int n_kv_heads, isoq_params** out) {
+  return isoq_make_params_v(seed, d, n_kv_heads, 3, ISOQ_ROT_SO4, out);
+}
+
+int isoq_params_format(const isoq_params* p, int* bits, int* rotation) {
+  if (!p) return ISOQ_E_ARG;
+  if (bits) *bits = p->bits;
+  if (rotation) *rotation = p->rotation;
   return ISOQ_OK;
 }
 
@@ -231,10 +282,12 @@ void isoq_params_destroy(isoq_params* p) {
   delete p;
 }
 
-size_t isoq_block_bytes(int d, int page_size) {
-  if (!supported_d(d) || page_size != ISOQ_PAGE_SIZE) return 0;
-  return (size_t)2 * page_size * (3 * d / 8 + 2);
+size_t isoq_block_bytes_v(int d, int bits, int page_size) {
+  if (!supported_d(d) || !supported_format(d, bits) || page_size != ISOQ_PAGE_SIZE) return 0;
+  return (size_t)2 * page_size * (bits * d / 8 + 2);
 }
+
+size_t isoq_block_bytes(int d, int page_size) { return isoq_block_bytes_v(d, 3, page_size); }
 
 int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, const void* K,
                          const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
@@ -247,6 +300,7 @@ int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, con
   if ((rc = check_device(params))) return rc;
   isoq::QuantizeArgs a;
   a.params = params->dev;
+  a.bits = params->bits;
   a.mats = params->dev_mat;
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;
@@ -315,7 +369,8 @@ int decode_common(const isoq_params* params, const isoq_cache* cache, const void
       plan_splits(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len, n_q);
   isoq::DecodeArgs a{};
   a.n_q = n_q;
-  a.params = params->dev;
+  a.params = params->dev_mat;
+  a.bits = params->bits;
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;
   a.n_pages = cache->n_pages;
@@ -389,7 +444,7 @@ int isoq_decode_merge_states(const isoq_params* params, const float* states, int
   if (!states || !out || ((uintptr_t)states & 15u) != 0) return ISOQ_E_ARG;
   int rc = check_device(params);
   if (rc) return rc;
-  cudaError_t e = isoq::launch_merge_states(params->dev, params->n_kv_heads, params->d, n_seqs,
+  cudaError_t e = isoq::launch_merge_states(params->dev_mat, params->n_kv_heads, params->d, n_seqs,
                                             n_q_heads, n_states, states, out,
                                             (cudaStream_t)stream);
   return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
@@ -430,7 +485,8 @@ const char* isoq_error_string(int code) {
 
 // Internal accessors for other translation units of the library (not part of the C ABI).
 namespace isoq {
-const float* params_device_ptr(const isoq_params* p) { return p ? p->dev : nullptr; }
+const float* params_device_mats(const isoq_params* p) { return p ? p->dev_mat : nullptr; }
+int params_bits(const isoq_params* p) { return p ? p->bits : 3; }
 int params_device(const isoq_params* p) { return p ? p->device : -1; }
 }  // namespace isoq
 namespace isoq {

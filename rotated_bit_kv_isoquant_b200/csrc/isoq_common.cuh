@@ -39,14 +39,47 @@ __host__ __device__ constexpr float threshold_f32(int j) {
                   : 1.748f;
 }
 
-// Bytes of packed codes per vector and per (page, head) block.
-__host__ __device__ constexpr int code_bytes(int D) { return 3 * D / 8; }
-__host__ __device__ constexpr int block_bytes(int D) { return 2 * kPage * (code_bytes(D) + 2); }
-// Offsets inside a block.
-__host__ __device__ constexpr int k_norm_off(int D) { return kPage * code_bytes(D); }
-__host__ __device__ constexpr int v_codes_off(int D) { return kPage * (code_bytes(D) + 2); }
-__host__ __device__ constexpr int v_norm_off(int D) {
-  return kPage * (code_bytes(D) + 2) + kPage * code_bytes(D);
+// Variants of the same family (Max 1960, Table I): 4 levels (2 bits) and 16 levels
+// (4 bits), ascending; only the non-negative halves are stored (the codebooks are
+// symmetric).  mag_f32(bits, k) = level 2^(bits-1) + k.
+__host__ __device__ constexpr float mag_f32(int bits, int k) {
+  return bits == 2 ? (k == 0 ? 0.4528f : 1.5104f)
+         : bits == 4
+             ? (k == 0   ? 0.1284f
+                : k == 1 ? 0.3881f
+                : k == 2 ? 0.6568f
+                : k == 3 ? 0.9424f
+                : k == 4 ? 1.2562f
+                : k == 5 ? 1.6180f
+                : k == 6 ? 2.0690f
+                         : 2.7326f)
+             : level_f32(4 + k);
+}
+__host__ __device__ constexpr float level_f32(int bits, int c) {
+  return c >= (1 << (bits - 1)) ? mag_f32(bits, c - (1 << (bits - 1)))
+                                : -mag_f32(bits, (1 << (bits - 1)) - 1 - c);
+}
+// Positive decision thresholds: midpoint of magnitudes k and k+1 (k = 0 .. 2^(bits-1)-2),
+// computed in double and rounded once to binary32 (3 bits: the decimal 0.50055, 1.05,
+// 1.748 of threshold_f32).
+__host__ __device__ constexpr float pos_threshold_f32(int bits, int k) {
+  return bits == 3 ? threshold_f32(4 + k)
+                   : (float)(0.5 * ((double)mag_f32(bits, k) + (double)mag_f32(bits, k + 1)));
+}
+
+// Bytes of packed codes per vector and per (page, head) block; offsets inside a block.
+__host__ __device__ constexpr int code_bytes(int D, int bits = 3) { return bits * D / 8; }
+__host__ __device__ constexpr int block_bytes(int D, int bits = 3) {
+  return 2 * kPage * (code_bytes(D, bits) + 2);
+}
+__host__ __device__ constexpr int k_norm_off(int D, int bits = 3) {
+  return kPage * code_bytes(D, bits);
+}
+__host__ __device__ constexpr int v_codes_off(int D, int bits = 3) {
+  return kPage * (code_bytes(D, bits) + 2);
+}
+__host__ __device__ constexpr int v_norm_off(int D, int bits = 3) {
+  return kPage * (code_bytes(D, bits) + 2) + kPage * code_bytes(D, bits);
 }
 
 template <typename T>
@@ -131,58 +164,34 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Hamilton product of quaternions (w, x, y, z).
-__device__ __forceinline__ void qmul(const float* a, const float* b, float* o) {
-  float w = a[0] * b[0] - a[1] * b[1] - a[2] * b[2] - a[3] * b[3];
-  float x = a[0] * b[1] + a[1] * b[0] + a[2] * b[3] - a[3] * b[2];
-  float y = a[0] * b[2] - a[1] * b[3] + a[2] * b[0] + a[3] * b[1];
-  float z = a[0] * b[3] + a[1] * b[2] - a[2] * b[1] + a[3] * b[0];
-  o[0] = w;
-  o[1] = x;
-  o[2] = y;
-  o[3] = z;
-}
-
-// z = p * y * conj(q)  (one SO(4) block).  pq: 8 floats, p then q.
-__device__ __forceinline__ void so4_fwd(const float* pq, const float* y, float* z) {
-  float t[4];
-  qmul(pq, y, t);
-  const float qc[4] = {pq[4], -pq[5], -pq[6], -pq[7]};
-  qmul(t, qc, z);
-}
-
-// y = conj(p) * z * q  (inverse block).
-__device__ __forceinline__ void so4_inv(const float* pq, const float* z, float* y) {
-  const float pc[4] = {pq[0], -pq[1], -pq[2], -pq[3]};
-  float t[4];
-  qmul(pc, z, t);
-  qmul(t, pq + 4, y);
-}
-
-// Loads the 8 parameters (p, q) of block b of one head into registers.
-__device__ __forceinline__ void load_block_params(const float* __restrict__ head_params, int b,
-                                                  float (&pq)[8]) {
-  const float4* s = reinterpret_cast<const float4*>(head_params + 8 * b);
-  float4 a = __ldg(s), c = __ldg(s + 1);
-  pq[0] = a.x;
-  pq[1] = a.y;
-  pq[2] = a.z;
-  pq[3] = a.w;
-  pq[4] = c.x;
-  pq[5] = c.y;
-  pq[6] = c.z;
-  pq[7] = c.w;
-}
-
-// Code of one packed element: element e (0..31) of a 12-byte group (w0, w1, w2).
-__device__ __forceinline__ int group_code(uint32_t w0, uint32_t w1, uint32_t w2, int e) {
-  if (e < 24) {
-    uint32_t w = e < 8 ? w0 : (e < 16 ? w1 : w2);
-    return (w >> (4 * (e & 7))) & 7;
+// The rotation blocks of a head as 4x4 row-major matrices (one per 4 dims: an SO(4)
+// block p y conj(q), or two SO(2) blocks on the diagonal), derived from the parameters in
+// binary64 when the parameter handle is made.  head_mats = mats + head * (d / 4) * 16.
+__device__ __forceinline__ void load_block_mat(const float* __restrict__ head_mats, int b,
+                                               float (&M)[16]) {
+  const float4* s = reinterpret_cast<const float4*>(head_mats + 16 * b);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float4 v = __ldg(s + r);
+    M[4 * r + 0] = v.x;
+    M[4 * r + 1] = v.y;
+    M[4 * r + 2] = v.z;
+    M[4 * r + 3] = v.w;
   }
-  int k = e - 24;
-  return (((w0 >> (4 * k + 3)) & 1) << 2) | (((w1 >> (4 * k + 3)) & 1) << 1) |
-         ((w2 >> (4 * k + 3)) & 1);
+}
+
+// z = M y (forward block rotation).
+__device__ __forceinline__ void mat_fwd(const float (&M)[16], const float* y, float* z) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    z[r] = fmaf(M[4 * r + 3], y[3], fmaf(M[4 * r + 2], y[2], fmaf(M[4 * r + 1], y[1], M[4 * r] * y[0])));
+}
+
+// y = M^T z (inverse block rotation: the blocks are orthogonal).
+__device__ __forceinline__ void mat_inv(const float (&M)[16], const float* z, float* y) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    y[c] = fmaf(M[12 + c], z[3], fmaf(M[8 + c], z[2], fmaf(M[4 + c], z[1], M[c] * z[0])));
 }
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {

@@ -119,13 +119,13 @@ __global__ void __launch_bounds__(128)
     const int dd = lane * E + i;
     o[i] = (red_acc[0][dd] + red_acc[1][dd] + red_acc[2][dd] + red_acc[3][dd]) * inv;
   }
-  const float* hp = params + (size_t)((h % n_q_heads) / G) * D * 2;
+  const float* hp = params + (size_t)((h % n_q_heads) / G) * D * 4;  // block matrices
   float y[E];
 #pragma unroll
   for (int k = 0; k < NB; ++k) {
-    float pq[8];
-    load_block_params(hp, lane * NB + k, pq);
-    so4_inv(pq, o + 4 * k, y + 4 * k);
+    float M[16];
+    load_block_mat(hp, lane * NB + k, M);
+    mat_inv(M, o + 4 * k, y + 4 * k);
   }
   wht_warp<E>(y, lane);
   const float r = rsqrtf((float)D);
@@ -136,8 +136,9 @@ __global__ void __launch_bounds__(128)
 
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
-  cudaError_t e = (kUseTc128 && D == 128 && a.n_q == 1) ? launch_decode_split_tc(a, stream)
-                                                         : launch_decode_split_mma(a, stream);
+  cudaError_t e = (kUseTc128 && D == 128 && a.n_q == 1 && a.bits == 3)
+                      ? launch_decode_split_tc(a, stream)
+                      : launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
   const int rows = a.n_q * a.n_q_heads;
   dim3 grid(rows, a.n_seqs);

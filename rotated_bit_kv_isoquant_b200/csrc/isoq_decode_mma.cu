@@ -23,6 +23,9 @@
 // exactly a prmt byte selector; the other 8 come from the spare bit 3 of three words.
 // Levels are scaled by ALPHA, a constant for which all four magnitudes round to binary16
 // with relative error < 2e-5 (1/ALPHA is folded into the score and output scales).
+// The 2- and 4-bit variants (d = 128) swap in their own unit dequantisers (isoq_ptx.cuh):
+// 4 bits look up the magnitude nibble and flip the sign bit; 2 bits turn two codes into
+// one selector with a multiply-add and look up an f16x2 in a single byte permute.
 #include <math_constants.h>
 
 #include <type_traits>
@@ -38,9 +41,9 @@ using namespace ptx;
 // Dynamic shared memory: [kWarps][NST] page stages of block_bytes(D), then the mbarriers,
 // then the score mma's A fragments of the rotated queries (one uint4 per k-step and lane,
 // shared by the four warps).  The stage area is reused for the final merge.
-template <int D, int NST>
+template <int D, int NST, int BITS = 3>
 struct MmaSmem {
-  static constexpr int kStageBytes = block_bytes(D);
+  static constexpr int kStageBytes = block_bytes(D, BITS);
   static constexpr int kRing = kWarps * NST * kStageBytes;
   static constexpr int kBarOff = kRing;
   static constexpr int kAOff = kBarOff + kWarps * NST * 8;
@@ -58,18 +61,20 @@ constexpr int dec_min_blocks() { return D == 128 ? 4 : 2; }
 
 // MQ: chunks of several query tokens per sequence with causal limits; the decode (one
 // query token, every row attending the whole context) is compiled without them.
-template <int D, int NST, typename TQ, bool MQ>
+template <int D, int NST, typename TQ, bool MQ, int BITS>
 __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     decode_mma_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
                       const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                       const TQ* __restrict__ Q, int n_q_heads, int n_q,
                       const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
                       int n_splits, float* __restrict__ partials, uint32_t* status) {
-  using SM = MmaSmem<D, NST>;
+  using SM = MmaSmem<D, NST, BITS>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
-  constexpr int CB = code_bytes(D);
-  constexpr int BB = block_bytes(D);
+  constexpr int CB = code_bytes(D, BITS);
+  constexpr int BB = block_bytes(D, BITS);
+  constexpr int W = BITS;             // words per 32-dim group of a packed vector
+  constexpr float ALPHA = alpha_of<BITS>();
   constexpr int KS = D / 16;          // k-steps of the score mma = m-tiles of the PV mma
   constexpr int NG = D / 128;         // 32-dim groups per thread and token (score: t, t+4)
   constexpr int PS = D + 4;
@@ -157,10 +162,10 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   //   a0 = hi(g; base, base+1)  a1 = lo(g; base, base+1)
   //   a2 = hi(g; base+2, +3)    a3 = lo(g; base+2, +3)
   {
-    const float* hp = params + (size_t)hk * D * 2;
-    float pq[NB][8];
+    const float* hp = params + (size_t)hk * D * 4;  // this head's block matrices
+    float pq[NB][16];
 #pragma unroll
-    for (int k = 0; k < NB; ++k) load_block_params(hp, lane * NB + k, pq[k]);
+    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, pq[k]);
     for (int h = warp; h < 8; h += kWarps) {
       float v[E];
       if (h < nh) {
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
       wht_warp<E>(v, lane);
       float z[E];
 #pragma unroll
-      for (int k = 0; k < NB; ++k) so4_fwd(pq[k], v + 4 * k, z + 4 * k);
+      for (int k = 0; k < NB; ++k) mat_fwd(pq[k], v + 4 * k, z + 4 * k);
 #pragma unroll
       for (int k = 0; k < NB; ++k) {
         const int base = lane * E + 4 * k;  // dims base..base+3
@@ -194,20 +199,9 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   }
   __syncthreads();
 
-  // level byte tables: tl = low bytes, th = high bytes of f16(ALPHA * L[c]), c = 0..7
-  uint32_t tl0 = 0, tl1 = 0, th0 = 0, th1 = 0;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint32_t hbits = __half_as_ushort(__float2half_rn(kAlpha * level_f32(c)));
-    const uint32_t lo = hbits & 0xffu, hi = hbits >> 8;
-    if (c < 4) {
-      tl0 |= lo << (8 * c);
-      th0 |= hi << (8 * c);
-    } else {
-      tl1 |= lo << (8 * (c - 4));
-      th1 |= hi << (8 * (c - 4));
-    }
-  }
+  // level byte tables of the format (f16 of ALPHA times the levels or magnitudes)
+  uint32_t tl0, tl1, th0, th1;
+  level_tables<BITS>(tl0, tl1, th0, th1);
 
   // Softmax state of head g (the score rows of this lane); the PV accumulator columns of
   // this lane are heads 2t, 2t+1, whose rescale factors come from lanes 8t and 8t + 4.
@@ -218,7 +212,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   float acc[KS][4];
 #pragma unroll
   for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  const float kf = scale * kLog2e / (kAlpha * (float)D);  // log2 score per (dot * nK)
+  const float kf = scale * kLog2e / (ALPHA * (float)D);  // log2 score per (dot * nK)
 
   bool timed_out = false;
   int k = 0;
@@ -244,14 +238,13 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
       for (int n = 0; n < 4; ++n) C[n][0] = C[n][1] = C[n][2] = C[n][3] = 0.f;
 #pragma unroll
       for (int gq = 0; gq < NG; ++gq) {
-        uint32_t w[4][3];
+        uint32_t w[4][W];
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
           const uint32_t* p =
-              reinterpret_cast<const uint32_t*>(blk + (tb + 8 * n + g) * CB) + 3 * (t + 4 * gq);
-          w[n][0] = p[0];
-          w[n][1] = p[1];
-          w[n][2] = p[2];
+              reinterpret_cast<const uint32_t*>(blk + (tb + 8 * n + g) * CB) + W * (t + 4 * gq);
+#pragma unroll
+          for (int i = 0; i < W; ++i) w[n][i] = p[i];
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -259,10 +252,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
           const uint4 A1 = qa[(8 * gq + 2 * j + 1) * 32 + lane];
           uint32_t f[4][4];
 #pragma unroll
-          for (int n = 0; n < 4; ++n) {
-            const uint32_t S = j < 3 ? (w[n][j] & 0x77777777u) : spare_codes(w[n][0], w[n][1], w[n][2]);
-            deq8(S, tl0, tl1, th0, th1, f[n]);
-          }
+          for (int n = 0; n < 4; ++n) kdeq<BITS>(w[n], j, tl0, tl1, th0, th1, f[n]);
 #pragma unroll
           for (int n = 0; n < 4; ++n) mma16816(C[n], A0.x, A0.y, A0.z, A0.w, f[n][0], f[n][1]);
 #pragma unroll
@@ -279,9 +269,9 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
       for (int n = 0; n < 4; ++n) {
         const int tk = tb + 8 * n + 2 * t;
         const float2 nk2 = __half22float2(
-            *reinterpret_cast<const __half2*>(blk + k_norm_off(D) + 2 * tk));
+            *reinterpret_cast<const __half2*>(blk + k_norm_off(D, BITS) + 2 * tk));
         const float2 nv2 = __half22float2(
-            *reinterpret_cast<const __half2*>(blk + v_norm_off(D) + 2 * tk));
+            *reinterpret_cast<const __half2*>(blk + v_norm_off(D, BITS) + 2 * tk));
         sv[n][0] = (C[n][0] + C[n][2]) * (nk2.x * kf);
         sv[n][1] = (C[n][1] + C[n][3]) * (nk2.y * kf);
         nv[n][0] = nv2.x;
@@ -354,16 +344,25 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
 #pragma unroll
         for (int gq = 0; gq < NG; ++gq) {
           const int q = (g >> 1) + 4 * gq;
-          const uint8_t* vbase = blk + v_codes_off(D);
-          const bool odd = (g & 1) != 0;  // odd g: words 2, 3 (w2 and the spare bits)
-          uint32_t S[4][2];  // [token 2t, 2t+1, 2t+8, 2t+9][word j0, j0+1]
+          const uint8_t* vbase = blk + v_codes_off(D, BITS);
+          const bool odd = (g & 1) != 0;  // odd g: units 2, 3 of the group, even g: 0, 1
+          uint32_t S[4][2];  // [token 2t, 2t+1, 2t+8, 2t+9][unit j0, j0+1]
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
             const int tk = r + 2 * t + (x & 1) + 8 * (x >> 1);
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + 3 * q;
-            const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
-            S[x][0] = (odd ? w2 : w0) & 0x77777777u;
-            S[x][1] = odd ? spare_codes(w0, w1, w2) : (w1 & 0x77777777u);
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + W * q;
+            if constexpr (BITS == 3) {  // unit 3 = the spare bits of the three words
+              const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
+              S[x][0] = (odd ? w2 : w0) & 0x77777777u;
+              S[x][1] = odd ? spare_codes(w0, w1, w2) : (w1 & 0x77777777u);
+            } else if constexpr (BITS == 4) {  // unit = word
+              S[x][0] = w[odd ? 2 : 0];
+              S[x][1] = w[odd ? 3 : 1];
+            } else {  // two units per word, low half first
+              const uint32_t w0 = w[odd ? 1 : 0];
+              S[x][0] = w0;
+              S[x][1] = w0 >> 16;
+            }
           }
           // m-tile 4 ww + 2 part + hh: row g = nibble 4 part + 2 hh of word j0 + ww, row g+8
           // = the next nibble, so each A quad is two output pairs of two lookups
@@ -372,8 +371,8 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
               uint32_t fa[4], fb[4];  // tokens (2t, 2t+1) and (2t+8, 2t+9)
-              deq4_pair(S[0][ww], S[1][ww], part, tl0, tl1, th0, th1, fa);
-              deq4_pair(S[2][ww], S[3][ww], part, tl0, tl1, th0, th1, fb);
+              vdeq<BITS>(S[0][ww], S[1][ww], part, tl0, tl1, th0, th1, fa);
+              vdeq<BITS>(S[2][ww], S[3][ww], part, tl0, tl1, th0, th1, fb);
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh)
                 mma16816(acc[8 * gq + 4 * ww + 2 * part + hh], fa[2 * hh], fa[2 * hh + 1],
@@ -415,7 +414,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   float* mb = reinterpret_cast<float*>(smem);  // [kWarps][8 heads][D + 4]
   {
     // acc_true = acc * sigma / ALPHA (times 1 / exp2(m2) in the log2 frame)
-    const float f = sigma / kAlpha;
+    const float f = sigma / ALPHA;
 #pragma unroll
     for (int gq = 0; gq < NG; ++gq) {
 #pragma unroll
@@ -462,42 +461,52 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   }
 }
 
-template <int D, int NST, typename TQ, bool MQ>
+template <int D, int NST, typename TQ, bool MQ, int BITS>
 static cudaError_t launch_mma_t(const DecodeArgs& a, cudaStream_t stream) {
-  using SM = MmaSmem<D, NST>;
+  using SM = MmaSmem<D, NST, BITS>;
   // the dynamic shared-memory opt-in is per function and per device
   static unsigned long long attr_set = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !((attr_set >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(decode_mma_kernel<D, NST, TQ, MQ>,
+    e = cudaFuncSetAttribute(decode_mma_kernel<D, NST, TQ, MQ, BITS>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
     if (e != cudaSuccess) return e;
     attr_set |= 1ull << dev;
   }
   const int G = a.n_q_heads / a.n_kv_heads;
   dim3 grid(a.n_splits, a.n_kv_heads * ((a.n_q * G + 7) / 8), a.n_seqs);
-  decode_mma_kernel<D, NST, TQ, MQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
+  decode_mma_kernel<D, NST, TQ, MQ, BITS><<<grid, kWarps * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
       a.n_splits, a.partials, a.status);
   return cudaGetLastError();
 }
 
-template <int D, int NST>
-cudaError_t launch_decode_mma_d(const DecodeArgs& a, cudaStream_t stream) {
+template <int D, int NST, int BITS>
+cudaError_t launch_decode_mma_b(const DecodeArgs& a, cudaStream_t stream) {
   const bool mq = a.n_q > 1;
   switch (a.q_dtype) {
     case ISOQ_F32:
-      return mq ? launch_mma_t<D, NST, float, true>(a, stream)
-                : launch_mma_t<D, NST, float, false>(a, stream);
+      return mq ? launch_mma_t<D, NST, float, true, BITS>(a, stream)
+                : launch_mma_t<D, NST, float, false, BITS>(a, stream);
     case ISOQ_BF16:
-      return mq ? launch_mma_t<D, NST, __nv_bfloat16, true>(a, stream)
-                : launch_mma_t<D, NST, __nv_bfloat16, false>(a, stream);
+      return mq ? launch_mma_t<D, NST, __nv_bfloat16, true, BITS>(a, stream)
+                : launch_mma_t<D, NST, __nv_bfloat16, false, BITS>(a, stream);
     case ISOQ_F16:
-      return mq ? launch_mma_t<D, NST, __half, true>(a, stream)
-                : launch_mma_t<D, NST, __half, false>(a, stream);
+      return mq ? launch_mma_t<D, NST, __half, true, BITS>(a, stream)
+                : launch_mma_t<D, NST, __half, false, BITS>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int NST>
+cudaError_t launch_decode_mma_d(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.bits == 3) return launch_decode_mma_b<D, NST, 3>(a, stream);
+  if constexpr (D == 128) {  // the 2- and 4-bit variants exist at d = 128
+    if (a.bits == 2) return launch_decode_mma_b<D, NST, 2>(a, stream);
+    if (a.bits == 4) return launch_decode_mma_b<D, NST, 4>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -530,18 +539,18 @@ int decode_resident_ctas(int d) {
     cudaError_t e;
     if (d == 256) {
       using SM = MmaSmem<256, ISOQ_DEC_NST256>;
-      e = cudaFuncSetAttribute(decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false>,
+      e = cudaFuncSetAttribute(decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false, 3>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false>, kWarps * 32, SM::kBytes);
+            &n, decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false, 3>, kWarps * 32, SM::kBytes);
     } else {
       using SM = MmaSmem<128, ISOQ_DEC_NST128>;
-      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false>,
+      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false, 3>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false>, kWarps * 32, SM::kBytes);
+            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false, 3>, kWarps * 32, SM::kBytes);
     }
     if (e != cudaSuccess || n < 1) {
       cudaGetLastError();

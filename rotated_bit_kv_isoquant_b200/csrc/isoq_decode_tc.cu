@@ -243,10 +243,10 @@ __global__ void __launch_bounds__(kTcTile)
   // ---- a6: rotate the CTA's queries (unnormalised WHT + SO(4)), staged fp32 in the V tile
   {
     float* qs = reinterpret_cast<float*>(smem + kOffV);  // [8][D], reused later
-    const float* hp = params + (size_t)hk * D * 2;
-    float pq[NB][8];
+    const float* hp = params + (size_t)hk * D * 4;  // this head's block matrices
+    float pq[NB][16];
 #pragma unroll
-    for (int k = 0; k < NB; ++k) load_block_params(hp, lane * NB + k, pq[k]);
+    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, pq[k]);
     for (int h = warp; h < 8; h += 4) {
       float v[E];
       if (h < nh) {
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kTcTile)
       wht_warp<E>(v, lane);
       float z[E];
 #pragma unroll
-      for (int k = 0; k < NB; ++k) so4_fwd(pq[k], v + 4 * k, z + 4 * k);
+      for (int k = 0; k < NB; ++k) mat_fwd(pq[k], v + 4 * k, z + 4 * k);
 #pragma unroll
       for (int i = 0; i < E; ++i) qs[h * D + lane * E + i] = z[i];
     }

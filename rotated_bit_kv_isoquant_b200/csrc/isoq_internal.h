@@ -10,8 +10,9 @@ struct isoq_params;
 namespace isoq {
 
 struct QuantizeArgs {
-  const float* params;  // device [H][d/4][2][4]
+  const float* params;  // device: the parameters as generated (unused by the kernels)
   const float* mats;    // device [H][d/4][4][4]: block rotations as matrices
+  int bits;             // bits per code (2, 3, 4)
   uint8_t* blocks;
   const int32_t* page_table;
   int n_pages, max_pages, n_seqs, n_kv_heads, d;
@@ -25,7 +26,8 @@ struct QuantizeArgs {
 };
 
 struct DecodeArgs {
-  const float* params;
+  const float* params;  // the heads' 4x4 block matrices [n_kv_heads][d/4][16]
+  int bits;             // bits per code (2, 3, 4)
   const uint8_t* blocks;
   const int32_t* page_table;
   int n_pages, max_pages, n_kv_heads, d;
@@ -66,7 +68,8 @@ constexpr bool kUseTc128 = false;
 #endif
 
 // Accessors of the opaque parameter handle (defined in isoq_api.cu).
-const float* params_device_ptr(const struct ::isoq_params* p);
+const float* params_device_mats(const struct ::isoq_params* p);  // [H][d/4][4][4]
+int params_bits(const struct ::isoq_params* p);
 int params_device(const struct ::isoq_params* p);
 // Records e as the thread's last CUDA error and returns ISOQ_E_CUDA.
 int record_cuda_error(cudaError_t e);

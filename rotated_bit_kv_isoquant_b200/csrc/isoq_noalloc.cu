@@ -70,6 +70,7 @@ extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const is
   if (cache->page_size != ISOQ_PAGE_SIZE || (cache->d != 128 && cache->d != 256))
     return ISOQ_E_DIM;
   if (cache->d != pd || cache->n_kv_heads != ph) return ISOQ_E_DIM;
+  if ((cache->bits == 0 ? 3 : cache->bits) != isoq::params_bits(params)) return ISOQ_E_DIM;
   if (cache->n_pages < 0 || cache->max_pages_per_seq < 1 || cache->n_seqs < 1 ||
       cache->n_kv_heads < 1)
     return ISOQ_E_ARG;
@@ -102,7 +103,8 @@ extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const is
   if (!scratch) return isoq::record_cuda_error(e);
 
   isoq::DecodeArgs a{};
-  a.params = isoq::params_device_ptr(params);
+  a.params = isoq::params_device_mats(params);
+  a.bits = isoq::params_bits(params);
   a.blocks = cache->blocks;
   a.page_table = cache->page_table;
   a.n_pages = cache->n_pages;

@@ -5,6 +5,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "isoq_common.cuh"
+
 namespace isoq {
 namespace ptx {
 
@@ -134,6 +136,94 @@ __device__ __forceinline__ void deq4_pair(uint32_t Sa, uint32_t Sb, int part, ui
     const uint32_t hi = prmt(th0, th1, sel);
     o[2 * hh + 0] = prmt(lo, hi, 0x6240);
     o[2 * hh + 1] = prmt(lo, hi, 0x7351);
+  }
+}
+
+// ---- per-format dequantisation ---------------------------------------------------------
+// A 32-dim group of a packed vector is BITS little-endian words; it splits into four
+// "units" of 8 dims (dims 8u..8u+7).  kdeq<BITS> turns unit u of a token into four f16x2
+// (dims 8u+2i, 8u+2i+1) -- a K fragment; vdeq<BITS> turns the same unit of two tokens a, b
+// into four f16x2 (a, b) of dims 8u + 4 part + i -- a V fragment.  Values are ALPHA(BITS)
+// times the level.  ALPHA is chosen so that every level magnitude is (nearly) exact in
+// binary16: relative error < 2e-5 (3 bits), exact (2 bits), < 6e-5 (4 bits).
+template <int BITS>
+constexpr float alpha_of() { return BITS == 3 ? kAlpha : (BITS == 2 ? 7500.0f : 5992.94213044f); }
+
+// Level-byte tables.  3 bits: lo/hi bytes of the 8 levels (tl0,tl1 | th0,th1); 4 bits:
+// of the 8 magnitudes; 2 bits: tl0 = low bytes of the 4 levels, th0 = high bytes.
+template <int BITS>
+__device__ __forceinline__ void level_tables(uint32_t& tl0, uint32_t& tl1, uint32_t& th0,
+                                             uint32_t& th1) {
+  tl0 = tl1 = th0 = th1 = 0;
+  constexpr int N = BITS == 2 ? 4 : 8;
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    const float v = BITS == 4 ? mag_f32(4, c) : level_f32(BITS, c);
+    const uint32_t hbits = __half_as_ushort(__float2half_rn(alpha_of<BITS>() * v));
+    const uint32_t lo = hbits & 0xffu, hi = hbits >> 8;
+    if (c < 4) {
+      tl0 |= lo << (8 * c);
+      th0 |= hi << (8 * c);
+    } else {
+      tl1 |= lo << (8 * (c - 4));
+      th1 |= hi << (8 * (c - 4));
+    }
+  }
+}
+
+// 4 bits: flip the f16 sign of o (values of nibbles n, n') where the selected sign bits
+// (bit 3 of the nibbles, replicated by prmt's sign mode from S / S << 4) are set.
+__device__ __forceinline__ uint32_t apply_sign(uint32_t o, uint32_t S, uint32_t S4, uint32_t sel) {
+  return o ^ (prmt(S, S4, sel) & 0x80008000u);
+}
+
+// 2 bits: f16x2 of the codes in bits 0-1 and 8-9 of x (the rest of the low 16 bits zero):
+// selector nibbles (c0, 4 + c0, c1, 4 + c1) on the pool (low bytes | high bytes).
+__device__ __forceinline__ uint32_t deq2(uint32_t x, uint32_t tl0, uint32_t th0) {
+  return prmt(tl0, th0, x * 0x11u + 0x4040u);
+}
+
+template <int BITS>
+__device__ __forceinline__ void kdeq(const uint32_t* w, int u, uint32_t tl0, uint32_t tl1,
+                                     uint32_t th0, uint32_t th1, uint32_t (&o)[4]) {
+  if constexpr (BITS == 3) {
+    const uint32_t S = u < 3 ? (w[u] & 0x77777777u) : spare_codes(w[0], w[1], w[2]);
+    deq8(S, tl0, tl1, th0, th1, o);
+  } else if constexpr (BITS == 4) {
+    const uint32_t S = w[u], S4 = S << 4;
+    deq8(S & 0x77777777u, tl0, tl1, th0, th1, o);
+    o[0] = apply_sign(o[0], S, S4, 0x80C0u);
+    o[1] = apply_sign(o[1], S, S4, 0x90D0u);
+    o[2] = apply_sign(o[2], S, S4, 0xA0E0u);
+    o[3] = apply_sign(o[3], S, S4, 0xB0F0u);
+  } else {
+    const uint32_t U = w[u >> 1] >> (16 * (u & 1));  // slots 0..7 of the unit
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = deq2((U >> (2 * i)) & 0x0303u, tl0, th0);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void vdeq(uint32_t Sa, uint32_t Sb, int part, uint32_t tl0,
+                                     uint32_t tl1, uint32_t th0, uint32_t th1,
+                                     uint32_t (&o)[4]) {
+  if constexpr (BITS == 3) {
+    deq4_pair(Sa, Sb, part, tl0, tl1, th0, th1, o);
+  } else if constexpr (BITS == 4) {
+    const uint32_t X = prmt(Sa, Sb, part == 0 ? 0x5140u : 0x7362u), X4 = X << 4;
+    deq4_pair(Sa & 0x77777777u, Sb & 0x77777777u, part, tl0, tl1, th0, th1, o);
+    o[0] = apply_sign(o[0], X, X4, 0xD0C0u);
+    o[1] = apply_sign(o[1], X, X4, 0x9080u);
+    o[2] = apply_sign(o[2], X, X4, 0xF0E0u);
+    o[3] = apply_sign(o[3], X, X4, 0xB0A0u);
+  } else {
+    // units = slots 0..7 in the low 16 bits; M bytes: a slots 0-3, b 0-3, a 4-7, b 4-7
+    const uint32_t M = prmt(Sa, Sb, 0x5140u);
+    // dims 4 part + i -> slots (2 part, 2 part + 4, 2 part + 1, 2 part + 5)
+    o[0] = deq2((M >> (4 * part)) & 0x0303u, tl0, th0);
+    o[1] = deq2((M >> (16 + 4 * part)) & 0x0303u, tl0, th0);
+    o[2] = deq2((M >> (4 * part + 2)) & 0x0303u, tl0, th0);
+    o[3] = deq2((M >> (16 + 4 * part + 2)) & 0x0303u, tl0, th0);
   }
 }
 

@@ -32,6 +32,24 @@ __device__ __forceinline__ uint32_t code_of(float z, const uint32_t (&tb)[3]) {
   return (4u + m) ^ (neg * 7u);
 }
 
+// The same decision for a 2^BITS-level symmetric codebook: T[k] = n * (positive threshold
+// k), k < 2^(BITS-1) - 1; code = (half + m) ^ (neg * (2 half - 1)), half = 2^(BITS-1).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_of_b(float z, const uint32_t (&tb)[(1 << (BITS - 1)) - 1]) {
+  constexpr uint32_t half = 1u << (BITS - 1);
+  const uint32_t neg = z < 0.f ? 1u : 0u;
+  const uint32_t ai = (__float_as_uint(z) & 0x7fffffffu) - neg;
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < (int)half - 1; ++k) m += ai >= tb[k] ? 1u : 0u;
+  return (half + m) ^ (neg * (2 * half - 1));
+}
+
+// 2-bit layout: the slot (0..15) of dim e (0..15) of a 16-dim word.
+__host__ __device__ constexpr int slot2(int e) {
+  return e < 8 ? ((e & 1) ? (e >> 1) + 4 : (e >> 1)) : ((e & 1) ? ((e - 8) >> 1) + 12 : ((e - 8) >> 1) + 8);
+}
+
 // One warp per token; it walks the KV heads and, per head, quantises K and V together
 // (two independent chains for the scheduler).
 template <int D, typename T>
@@ -211,14 +229,16 @@ constexpr int kTpvThreads = 128;
 #define ISOQ_TPV_MINB 3
 #endif
 
-template <typename T>
+template <typename T, int BITS>
 __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     quantize_tpv_kernel(const float* __restrict__ mats, uint8_t* __restrict__ blocks,
                         const int32_t* __restrict__ page_table, int n_pages, int max_pages,
                         int n_seqs, int H, const T* __restrict__ K, const T* __restrict__ V,
                         int n_tokens, const int32_t* __restrict__ seq_ids,
                         const int32_t* __restrict__ positions, uint32_t* status) {
-  constexpr int D = 128, CB = code_bytes(D), BB = block_bytes(D);
+  constexpr int D = 128, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
+  constexpr int NT = (1 << (BITS - 1)) - 1;  // positive thresholds
+  constexpr uint32_t kZeroCode = 1u << (BITS - 1);
   extern __shared__ __align__(16) float smats[];  // [H][32 blocks][16]
   for (int i = threadIdx.x; i < H * (D / 4) * 16 / 4; i += blockDim.x)
     reinterpret_cast<float4*>(smats)[i] = __ldg(reinterpret_cast<const float4*>(mats) + i);
@@ -283,12 +303,15 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
       }
     }
 
-    // a3 + a4: SO(4) block (matrix from shared memory) and codes, block by block
-    uint32_t tb[3];
+    // a3 + a4: rotation block (matrix from shared memory) and codes, block by block
+    uint32_t tb[NT];
 #pragma unroll
-    for (int k = 0; k < 3; ++k) tb[k] = __float_as_uint(n * threshold_f32(4 + k));
+    for (int k = 0; k < NT; ++k) tb[k] = __float_as_uint(n * pos_threshold_f32(BITS, k));
     const float4* mh = reinterpret_cast<const float4*>(smats) + (size_t)h * (D / 4) * 4;
-    uint32_t nib[D / 8];  // nibble words: word j holds dims 8j..8j+7
+    uint32_t rec[CB / 4];
+    uint32_t nib[D / 8];  // 3 bits: nibble words, word j holds dims 8j..8j+7
+#pragma unroll
+    for (int i = 0; i < CB / 4; ++i) rec[i] = 0u;
 #pragma unroll
     for (int b = 0; b < D / 4; ++b) {
       float z[4];
@@ -297,27 +320,41 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
         const float4 m = mh[4 * b + rr];
         z[rr] = fmaf(m.w, x[4 * b + 3], fmaf(m.z, x[4 * b + 2], fmaf(m.y, x[4 * b + 1], m.x * x[4 * b])));
       }
-      uint32_t w = (b & 1) ? nib[b >> 1] : 0u;
+      if constexpr (BITS == 3) {
+        uint32_t w = (b & 1) ? nib[b >> 1] : 0u;
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const uint32_t c = n == 0.f ? 4u : code_of(z[rr], tb);
-        w |= c << (4 * (4 * (b & 1) + rr));
+        for (int rr = 0; rr < 4; ++rr) {
+          const uint32_t c = n == 0.f ? kZeroCode : code_of(z[rr], tb);
+          w |= c << (4 * (4 * (b & 1) + rr));
+        }
+        nib[b >> 1] = w;
+      } else {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int dim = 4 * b + rr;
+          const uint32_t c = n == 0.f ? kZeroCode : code_of_b<BITS>(z[rr], tb);
+          if constexpr (BITS == 4)  // sign-magnitude nibble
+            rec[dim >> 3] |= (c ^ ((c & 8u) ? 8u : 15u)) << (4 * (dim & 7));
+          else
+            rec[dim >> 4] |= c << (2 * slot2(dim & 15));
+        }
       }
-      nib[b >> 1] = w;
     }
 
-    // a5: pack: per 32-dim group, words 0..2 = nibble words + bit 3 from the trailing 8 codes
-    uint32_t rec[CB / 4];
+    // a5: pack (3 bits): per 32-dim group, words 0..2 = nibble words + bit 3 from the
+    // trailing 8 codes
+    if constexpr (BITS == 3) {
 #pragma unroll
-    for (int g = 0; g < D / 32; ++g) {
-      const uint32_t N3 = nib[4 * g + 3];
+      for (int g = 0; g < D / 32; ++g) {
+        const uint32_t N3 = nib[4 * g + 3];
 #pragma unroll
-      for (int j = 0; j < 3; ++j)
-        rec[3 * g + j] = nib[4 * g + j] | (((N3 >> (2 - j)) & 0x11111111u) << 3);
+        for (int j = 0; j < 3; ++j)
+          rec[3 * g + j] = nib[4 * g + j] | (((N3 >> (2 - j)) & 0x11111111u) << 3);
+      }
     }
     uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
     const int slot = pos & (kPage - 1);
-    uint4* dst = reinterpret_cast<uint4*>(blk + (kind == 0 ? 0 : v_codes_off(D)) + slot * CB);
+    uint4* dst = reinterpret_cast<uint4*>(blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB);
 #pragma unroll
     for (int q = 0; q < CB / 16; ++q)
       dst[q] = make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
@@ -326,7 +363,8 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
       nb = 0x7bffu;
       set_status(status, ISOQ_ST_NORM_SAT);
     }
-    *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D) : v_norm_off(D)) + 2 * slot) = nb;
+    *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
+                                 2 * slot) = nb;
   }
 }
 
@@ -345,11 +383,11 @@ static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, int BITS>
 static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   const size_t smem = (size_t)a.n_kv_heads * 32 * 16 * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T>,
+    cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T, BITS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
@@ -359,23 +397,34 @@ static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_
   const long long cap = (long long)n_sm * 3 * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  quantize_tpv_kernel<T><<<(unsigned)grid, kTpvThreads, smem, stream>>>(
+  quantize_tpv_kernel<T, BITS><<<(unsigned)grid, kTpvThreads, smem, stream>>>(
       a.mats, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_seqs, a.n_kv_heads,
       static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.n_tokens, a.seq_ids, a.positions,
       a.status);
   return cudaGetLastError();
 }
 
+template <typename T>
+static cudaError_t launch_tpv_b(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  switch (a.bits) {
+    case 2: return launch_tpv<T, 2>(a, stream, n_sm);
+    case 3: return launch_tpv<T, 3>(a, stream, n_sm);
+    case 4: return launch_tpv<T, 4>(a, stream, n_sm);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int D>
 static cudaError_t launch_d(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   if constexpr (D == 128) {
     switch (a.dtype) {
-      case ISOQ_F32: return launch_tpv<float>(a, stream, n_sm);
-      case ISOQ_BF16: return launch_tpv<__nv_bfloat16>(a, stream, n_sm);
-      case ISOQ_F16: return launch_tpv<__half>(a, stream, n_sm);
+      case ISOQ_F32: return launch_tpv_b<float>(a, stream, n_sm);
+      case ISOQ_BF16: return launch_tpv_b<__nv_bfloat16>(a, stream, n_sm);
+      case ISOQ_F16: return launch_tpv_b<__half>(a, stream, n_sm);
     }
     return cudaErrorInvalidValue;
   }
+  if (a.bits != 3) return cudaErrorInvalidValue;  // the variants exist at d = 128
   switch (a.dtype) {
     case ISOQ_F32: return launch_t<D, float>(a, stream, n_sm);
     case ISOQ_BF16: return launch_t<D, __nv_bfloat16>(a, stream, n_sm);

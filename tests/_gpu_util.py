@@ -28,13 +28,15 @@ def log_record(record: dict) -> None:
 class Run:
     """One workload on the GPU: params, cache, prefill, appended tokens, decode."""
 
-    def __init__(self, cfg: wl.Workload, device="cuda", seed: int = wl.PARAM_SEED):
+    def __init__(self, cfg: wl.Workload, device="cuda", seed: int = wl.PARAM_SEED,
+                 bits: int = 3, rot: int = 0):
         self.cfg = cfg
         self.device = device
-        self.params = iq.isoq_make_params(seed, cfg.d, cfg.n_kv_heads)
+        self.bits, self.rot = bits, rot
+        self.params = iq.isoq_make_params(seed, cfg.d, cfg.n_kv_heads, bits=bits, rotation=rot)
         self.layout = wl.page_layout(cfg)
         self.cache = iq.PagedCache(cfg.d, cfg.n_kv_heads, self.layout.n_pages,
-                                   self.layout.page_table, device=device)
+                                   self.layout.page_table, device=device, bits=bits)
 
     def prefill(self):
         cfg = self.cfg
@@ -65,15 +67,16 @@ class Run:
     def params64(self):
         """The oracle's own parameters (binary32 values promoted), for the parity path."""
         import oracle
-        _, p32 = oracle.make_params(wl.PARAM_SEED, self.cfg.d, self.cfg.n_kv_heads)
+        _, p32 = oracle.make_params_v(wl.PARAM_SEED, self.cfg.d, self.cfg.n_kv_heads, self.rot)
         return p32.astype(np.float64)
 
 
-def gather_records(cache: iq.PagedCache, page_table: torch.Tensor, seqs, positions, d: int):
+def gather_records(cache: iq.PagedCache, page_table: torch.Tensor, seqs, positions, d: int,
+                   bits: int = 3):
     """Device -> host: per (token, KV head) the packed K codes, K norm, V codes, V norm.
-    Returns (kcodes [n][H][3d/8], knorm [n][H], vcodes, vnorm) as numpy."""
+    Returns (kcodes [n][H][bits*d/8], knorm [n][H], vcodes, vnorm) as numpy."""
     dev = cache.blocks.device
-    cb = 3 * d // 8
+    cb = bits * d // 8
     seqs = torch.as_tensor(np.asarray(seqs), dtype=torch.long, device=dev)
     positions = torch.as_tensor(np.asarray(positions), dtype=torch.long, device=dev)
     pt = page_table.to(dev).long()
@@ -97,11 +100,11 @@ def gather_records(cache: iq.PagedCache, page_table: torch.Tensor, seqs, positio
     return kc.cpu().numpy(), to16(kn), vc.cpu().numpy(), to16(vn)
 
 
-def check_codes(oracle, params64, X, gpu_codes_packed, gpu_norms, d):
+def check_codes(oracle, params64, X, gpu_codes_packed, gpu_norms, d, bits: int = 3, rot: int = 0):
     """Compare GPU packed codes / norms of X ([n][H][d] host) with the oracle.
     Returns a dict of statistics; raises AssertionError on a violation."""
-    codes, norms, dist = oracle.quantize_rows(params64, X)
-    g = oracle.unpack_codes_batch(gpu_codes_packed, d)
+    codes, norms, dist = oracle.quantize_rows(params64, X, bits=bits, rot=rot)
+    g = oracle.unpack_codes_batch(gpu_codes_packed, d, bits=bits)
     diff = g != codes
     n_diff = int(diff.sum())
     in_band = dist < BAND
@@ -122,7 +125,8 @@ def check_attention(oracle, run: Run, Q, out, lens, sel=None):
     blocks = run.cache.blocks.cpu().numpy()
     ref = oracle.decode_attention(run.params64(), cfg.d, cfg.n_kv_heads, 64, blocks,
                                   run.layout.page_table.numpy(), lens,
-                                  Q.float().cpu().numpy().astype(np.float64), cfg.scale, sel=sel)
+                                  Q.float().cpu().numpy().astype(np.float64), cfg.scale, sel=sel,
+                                  bits=run.bits, rot=run.rot)
     got = out.cpu().numpy().astype(np.float64)
     pairs = sel if sel is not None else [(s, h) for s in range(Q.shape[0])
                                          for h in range(Q.shape[1])]
@@ -139,3 +143,26 @@ def check_attention(oracle, run: Run, Q, out, lens, sel=None):
     assert np.all(np.isfinite(got)), "non-finite output"
     assert errs.max() <= ATTN_TOL, f"max rel L2 {errs.max()} > {ATTN_TOL}"
     return {"pairs": len(pairs), "max_rel": float(errs.max()), "mean_rel": float(errs.mean())}
+
+
+def codes_all(oracle, run, seqs, positions):
+    """Check K and V codes of the given tokens against the oracle."""
+    cfg = run.cfg
+    kc, kn, vc, vn = gather_records(run.cache, run.layout.page_table, seqs, positions, cfg.d,
+                                    run.bits)
+    # regenerate the same inputs (chunked seeds) on the device, copy to host
+    Ks, Vs = [], []
+    order = np.lexsort((positions, seqs))
+    assert np.array_equal(order, np.arange(len(order))), "tokens must be sorted by (seq, pos)"
+    for s in np.unique(seqs):
+        p = np.asarray(positions)[np.asarray(seqs) == s]
+        K, V = wl.kv_tokens(cfg, int(s), int(p.min()), int(p.max() - p.min() + 1), device="cuda")
+        idx = torch.as_tensor(p - p.min(), device="cuda")
+        Ks.append(K[idx].float().cpu().numpy())
+        Vs.append(V[idx].float().cpu().numpy())
+    K = np.concatenate(Ks).astype(np.float64)
+    V = np.concatenate(Vs).astype(np.float64)
+    p64 = run.params64()
+    sk = check_codes(oracle, p64, K, kc, kn, cfg.d, run.bits, run.rot)
+    sv = check_codes(oracle, p64, V, vc, vn, cfg.d, run.bits, run.rot)
+    return {k: sk[k] + sv[k] for k in sk}

@@ -49,6 +49,29 @@ def test_params_generate_rejects():
     assert lib.isoq_params_generate(0, 128, 1, None) == iq.ISOQ_E_ARG
 
 
+@pytest.mark.parametrize("seed,d,h", [(0, 128, 8), (99, 256, 3)])
+def test_so2_params_generator_matches_oracle_bitwise(oracle, seed, d, h):
+    lib_params = iq.isoq_params_generate(seed, d, h, rotation=iq.ISOQ_ROT_SO2)
+    _, ref32 = oracle.make_params_so2(seed, d, h)
+    assert lib_params.shape == ref32.shape == (h, d // 2, 2)
+    assert np.array_equal(lib_params.view(np.uint32), ref32.view(np.uint32))
+
+
+def test_variant_formats_host_checks():
+    assert iq.isoq_block_bytes(128, bits=2) == 2 * 64 * (32 + 2)
+    assert iq.isoq_block_bytes(128, bits=4) == 2 * 64 * (64 + 2)
+    assert iq.isoq_block_bytes(128, bits=4) % 16 == 0 and iq.isoq_block_bytes(128, bits=2) % 16 == 0
+    assert iq.isoq_block_bytes(256, bits=2) == 0          # variants are d = 128 only
+    assert iq.isoq_block_bytes(128, bits=5) == 0
+    lib = iq.raw_lib()
+    h = ctypes.c_void_p()
+    # validated before any device call
+    assert lib.isoq_make_params_v(0, 128, 2, 5, iq.ISOQ_ROT_SO4, ctypes.byref(h)) == iq.ISOQ_E_DIM
+    assert lib.isoq_make_params_v(0, 256, 2, 4, iq.ISOQ_ROT_SO4, ctypes.byref(h)) == iq.ISOQ_E_DIM
+    assert lib.isoq_make_params_v(0, 128, 2, 3, 7, ctypes.byref(h)) == iq.ISOQ_E_ARG
+    assert lib.isoq_params_format(None, None, None) == iq.ISOQ_E_ARG
+
+
 def test_block_bytes():
     assert iq.isoq_block_bytes(128) == 6400
     assert iq.isoq_block_bytes(256) == 12544

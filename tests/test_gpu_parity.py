@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from _gpu_util import Run, check_attention, check_codes, gather_records
+from _gpu_util import Run, check_attention, check_codes, codes_all, gather_records
 
 import rotated_bit_kv_isoquant_b200 as iq
 import workloads as wl
@@ -37,26 +37,7 @@ def _cuda():
         pytest.skip("needs a CUDA device")
 
 
-def _codes_all(oracle, run, seqs, positions):
-    """Check K and V codes of the given tokens against the oracle."""
-    cfg = run.cfg
-    kc, kn, vc, vn = gather_records(run.cache, run.layout.page_table, seqs, positions, cfg.d)
-    # regenerate the same inputs (chunked seeds) on the device, copy to host
-    Ks, Vs = [], []
-    order = np.lexsort((positions, seqs))
-    assert np.array_equal(order, np.arange(len(order))), "tokens must be sorted by (seq, pos)"
-    for s in np.unique(seqs):
-        p = np.asarray(positions)[np.asarray(seqs) == s]
-        K, V = wl.kv_tokens(cfg, int(s), int(p.min()), int(p.max() - p.min() + 1), device="cuda")
-        idx = torch.as_tensor(p - p.min(), device="cuda")
-        Ks.append(K[idx].float().cpu().numpy())
-        Vs.append(V[idx].float().cpu().numpy())
-    K = np.concatenate(Ks).astype(np.float64)
-    V = np.concatenate(Vs).astype(np.float64)
-    p64 = run.params64()
-    sk = check_codes(oracle, p64, K, kc, kn, cfg.d)
-    sv = check_codes(oracle, p64, V, vc, vn, cfg.d)
-    return {k: sk[k] + sv[k] for k in sk}
+_codes_all = codes_all
 
 
 def _all_tokens(cfg):
@@ -166,6 +147,7 @@ def _len_run(cfg, lens):
     run._lens = lens
     run.cfg = cfg
     run.device = "cuda"
+    run.bits, run.rot = 3, 0
     run.params = iq.isoq_make_params(wl.PARAM_SEED, cfg.d, cfg.n_kv_heads)
     npg = [max(1, -(-n // 64)) for n in lens]
     rng = np.random.default_rng(sum(lens))

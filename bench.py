@@ -426,6 +426,9 @@ def run_ours(args, cfg):
         line["context_parallel"] = _bench_context_parallel(
             args, cfg, params, cache, layout, lens, Q, flush, stream, rank_max, world, rank,
             packed, peak, peak_kind)
+        if cfg.d == 128:
+            line["formats"] = _bench_formats(cfg, layout, inputs, app, Q, lens, flush, stream,
+                                             rank_max, peak, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:
@@ -479,6 +482,52 @@ def _bench_multi_token(args, cfg, params, cache, lens, flush, stream, rank_max, 
                          "frac": gbs / peak, "peak_kind": peak_kind,
                          "note": "packed KV counted once per call; this version streams it "
                                  "once per 8 (query token, head) rows"}}
+
+
+def _bench_formats(cfg, layout, inputs, app, Q, lens, flush, stream, rank_max, peak,
+                   peak_kind):
+    """The format variants on the same workload: quantize-append of the whole prefill and
+    one decode per (bits, rotation), each with its own cache."""
+    import torch
+
+    import rotated_bit_kv_isoquant_b200 as iq
+    import workloads as wl
+    dev = Q.device
+    res = {}
+    for bits, rot in ((2, 0), (4, 0), (3, 1), (2, 1), (4, 1)):
+        params = iq.isoq_make_params(wl.PARAM_SEED, cfg.d, cfg.n_kv_heads, bits=bits, rotation=rot)
+        cache = iq.PagedCache(cfg.d, cfg.n_kv_heads, layout.n_pages, layout.page_table, device=dev,
+                              bits=bits)
+
+        def quantize_all():
+            for K, V, sid, pos in inputs:
+                iq.isoq_quantize_append(params, cache, K, V, sid, pos, stream=stream)
+            if app[0].shape[0]:
+                iq.isoq_quantize_append(params, cache, app[0], app[1], app[2], app[3],
+                                        stream=stream)
+
+        q_ms = rank_max(_time_calls(quantize_all, flush, stream, iters=2, warmup=1))
+        sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+        out = torch.empty((cfg.n_seqs, cfg.n_q_heads, cfg.d), dtype=torch.float32, device=dev)
+        nb = iq.isoq_decode_workspace_bytes(cfg.n_seqs, cfg.n_q_heads, cfg.n_kv_heads, cfg.d,
+                                            max(lens))
+        ws = torch.empty((nb,), dtype=torch.uint8, device=dev)
+        fn = lambda: iq.isoq_decode_attention(params, cache, Q, sl, max(lens), out, cfg.scale, ws,
+                                              stream=stream)
+        d_ms = rank_max(_time_calls(fn, flush, stream))
+        packed = sum(lens) * cfg.n_kv_heads * 2 * (bits * cfg.d // 8 + 2)
+        n_vec = 2 * cfg.n_kv_heads * (sum(c for _, _, c in wl.prefill_calls(cfg)) + app[0].shape[0])
+        q_bytes = n_vec * (cfg.d * (4 if cfg.in_dtype == torch.float32 else 2) + bits * cfg.d // 8 + 2)
+        gbs = packed / (d_ms / 1e3) / 1e9
+        res[f"{bits}bit_{'so2' if rot else 'so4'}"] = {
+            "decode_GBps": gbs, "decode_frac": gbs / peak, "decode_ms": d_ms,
+            "quantize_Mvec_s": n_vec / (q_ms / 1e3) / 1e6,
+            "quantize_frac": q_bytes / (q_ms / 1e3) / 1e9 / peak,
+            "packed_bytes_per_decode": packed}
+        del cache, params
+        torch.cuda.empty_cache()
+    res["peak_kind"] = peak_kind
+    return res
 
 
 def _bench_context_parallel(args, cfg, params, cache, layout, lens, Q, flush, stream, rank_max,

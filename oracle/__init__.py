@@ -104,6 +104,8 @@ def _declare(L):
     L.ref_unpack_codes_batch.argtypes = [_p, _i, ctypes.c_long, _p]
     L.ref_attention_full.restype = None
     L.ref_attention_full.argtypes = [_i, _i, _i, _i, _p, _p, _p, _d, _p]
+    L.ref_rope.restype = None
+    L.ref_rope.argtypes = [_p, _i, _i, _d, _p]
     L.ref_level_v.restype = _d
     L.ref_level_v.argtypes = [_i, _i]
     L.ref_threshold_v.restype = _d
@@ -265,6 +267,21 @@ def unrotate(params_head, z, rot: int = 0) -> np.ndarray:
     x = np.zeros_like(z)
     lib().ref_unrotate_v(rot, _ptr(ph), _ptr(z), _ptr(x), z.shape[-1])
     return x
+
+
+def rope(x, pos, base: float = 10000.0) -> np.ndarray:
+    """Rotary embedding of each row of x (last axis d) at positions pos (scalar or one per
+    row): dims (i, i + d/2) rotated by pos * base^(-2i/d)."""
+    x = _f64(x)
+    flat = x.reshape(-1, x.shape[-1])
+    pos = np.broadcast_to(np.asarray(pos, dtype=np.int64), (flat.shape[0],))
+    out = np.zeros_like(flat)
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        o = np.zeros_like(row)
+        lib().ref_rope(_ptr(row), row.shape[0], int(pos[r]), float(base), _ptr(o))
+        out[r] = o
+    return out.reshape(x.shape)
 
 
 # ------------------------------------------------------------------------------------

@@ -254,6 +254,22 @@ void ref_unrotate(const double *params_head, const double *z, double *x, int d) 
 }
 
 /* ------------------------------------------------------------------------------ */
+/* Rotary position embedding of a key before quantisation (the fused RoPE epilogue): */
+/* half-split pairing, dims (i, i + d/2) rotated by pos * theta_i,                   */
+/* theta_i = base^(-2i/d) (RoFormer's frequencies; NeoX pairing).                    */
+/* ------------------------------------------------------------------------------ */
+void ref_rope(const double *x, int d, int pos, double base, double *out) {
+  int h = d / 2;
+  for (int i = 0; i < h; i++) {
+    double theta = pow(base, -2.0 * i / d);
+    double c = cos(pos * theta), s = sin(pos * theta);
+    double a = x[i], b = x[i + h];
+    out[i] = a * c - b * s;
+    out[i + h] = a * s + b * c;
+  }
+}
+
+/* ------------------------------------------------------------------------------ */
 /* IEEE 754 binary16, round to nearest, ties to even (from the format definition).   */
 /* ------------------------------------------------------------------------------ */
 uint16_t ref_fp16_bits(double v) {

@@ -225,3 +225,30 @@ def test_variant_mse_matches_codebook_distortion(oracle, bits, want):
         xh = oracle.unrotate(p64[0], oracle.fp16_value(n16) / math.sqrt(d) * L[codes])
         errs.append(np.sum((x - xh) ** 2) / np.sum(x ** 2))
     assert abs(np.mean(errs) - want) < 0.08 * want
+
+
+# ------------------------------------------------------------------------------------
+# RoPE of the fused quantize epilogue
+# ------------------------------------------------------------------------------------
+def test_rope_is_complex_multiplication_by_position_phases(oracle):
+    d, base = 128, 10000.0
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal(d)
+    for pos in (0, 1, 7, 1000, 131071):
+        got = oracle.rope(x, pos, base)
+        theta = base ** (-np.arange(d // 2) * 2.0 / d)
+        w = (x[:d // 2] + 1j * x[d // 2:]) * np.exp(1j * pos * theta)
+        assert np.allclose(got[:d // 2], w.real, atol=1e-12)
+        assert np.allclose(got[d // 2:], w.imag, atol=1e-12)
+    assert np.array_equal(oracle.rope(x, 0, base), x)
+
+
+def test_rope_preserves_norm_and_depends_on_relative_position(oracle):
+    d = 64
+    rng = np.random.default_rng(22)
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    assert abs(np.linalg.norm(oracle.rope(q, 12345)) - np.linalg.norm(q)) < 1e-12
+    for m, n in ((10, 3), (500, 499), (70000, 12)):
+        lhs = oracle.rope(q, m) @ oracle.rope(k, n)
+        rhs = oracle.rope(q, m - n) @ k
+        assert abs(lhs - rhs) < 1e-9 * (1 + abs(rhs))

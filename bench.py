@@ -426,6 +426,8 @@ def run_ours(args, cfg):
         line["context_parallel"] = _bench_context_parallel(
             args, cfg, params, cache, layout, lens, Q, flush, stream, rank_max, world, rank,
             packed, peak, peak_kind)
+        line["fused"] = _bench_fused(cfg, params, cache, inputs, lens, flush, stream,
+                                     rank_max, peak, peak_kind)
         if cfg.d == 128:
             line["formats"] = _bench_formats(cfg, layout, inputs, app, Q, lens, flush, stream,
                                              rank_max, peak, peak_kind)
@@ -482,6 +484,54 @@ def _bench_multi_token(args, cfg, params, cache, lens, flush, stream, rank_max, 
                          "frac": gbs / peak, "peak_kind": peak_kind,
                          "note": "packed KV counted once per call; this version streams it "
                                  "once per 8 (query token, head) rows"}}
+
+
+def _bench_fused(cfg, params, cache, inputs, lens, flush, stream, rank_max, peak, peak_kind):
+    """Fused epilogues: the prefill quantize-append with RoPE applied to K in the kernel
+    (pre-RoPE keys in, same cache), and one decode step's appends (one token per sequence)
+    into 32 layers' caches as 32 calls versus one layer-batched call."""
+    import torch
+
+    import rotated_bit_kv_isoquant_b200 as iq
+    import workloads as wl
+    dev = cache.blocks.device
+    tab = iq.isoq_rope_table(cfg.d, max(lens) + 1, device=dev)
+
+    def quantize_rope():
+        for K, V, sid, pos in inputs:
+            iq.isoq_quantize_append_rope(params, cache, K, V, sid, pos, tab, stream=stream)
+
+    n_vec = 2 * cfg.n_kv_heads * sum(K.shape[0] for K, _, _, _ in inputs)
+    rope_ms = rank_max(_time_calls(quantize_rope, flush, stream, iters=2, warmup=1))
+    n_layers = 32
+    pt = torch.arange(cfg.n_seqs, dtype=torch.int32).reshape(cfg.n_seqs, 1)
+    ps = [iq.isoq_make_params(wl.PARAM_SEED + l, cfg.d, cfg.n_kv_heads) for l in range(n_layers)]
+    cs = [iq.PagedCache(cfg.d, cfg.n_kv_heads, cfg.n_seqs, pt, device=dev) for _ in range(n_layers)]
+    g = torch.Generator(device=dev).manual_seed(3)
+    Ks = [torch.randn((cfg.n_seqs, cfg.n_kv_heads, cfg.d), generator=g, device=dev).to(cfg.in_dtype)
+          for _ in range(n_layers)]
+    Vs = [torch.randn_like(k, dtype=torch.float32).to(cfg.in_dtype) for k in Ks]
+    sid = torch.arange(cfg.n_seqs, dtype=torch.int32, device=dev)
+    pos = torch.full((cfg.n_seqs,), 5, dtype=torch.int32, device=dev)
+    step_tab = iq.isoq_rope_table(cfg.d, 64, device=dev)
+
+    def per_layer():
+        for l in range(n_layers):
+            iq.isoq_quantize_append_rope(ps[l], cs[l], Ks[l], Vs[l], sid, pos, step_tab,
+                                         stream=stream)
+
+    def batched():
+        iq.isoq_quantize_append_layers(ps, cs, Ks, Vs, sid, pos, rope_table=step_tab,
+                                       stream=stream)
+
+    t_sep = rank_max(_time_calls(per_layer, flush, stream, iters=20, warmup=3))
+    t_bat = rank_max(_time_calls(batched, flush, stream, iters=20, warmup=3))
+    return {"rope_quantize_Mvec_s": n_vec / (rope_ms / 1e3) / 1e6,
+            "rope_quantize_ms": rope_ms,
+            "decode_step_append_32_layers_us": {"per_layer_calls": t_sep * 1e3,
+                                                "one_batched_call": t_bat * 1e3},
+            "what": "RoPE applied to pre-RoPE K inside quantize-append (same cache and tokens as "
+                    "the step); a decode step's 1-token-per-sequence appends into 32 layers"}
 
 
 def _bench_formats(cfg, layout, inputs, app, Q, lens, flush, stream, rank_max, peak,

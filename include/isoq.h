@@ -211,6 +211,41 @@ int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, con
                          const int32_t* positions, void* stream);
 
 /* =======================================================================================
+ * Fused epilogues of the K/V projection (no model weights involved).
+ *
+ * isoq_quantize_append_rope: as isoq_quantize_append, with the rotary position embedding
+ *   applied to each K vector (given before RoPE) at its token's position, inside the same
+ *   kernel and before the norm and the rotation: dims (i, i + d/2) are rotated by the
+ *   angle with (cos, sin) = rope_table[position][i] (half-split pairing).  V is stored as
+ *   given.  rope_table: device fp32 [rope_max_pos][d/2][2], e.g. from isoq_rope_table; a
+ *   position >= rope_max_pos skips the token with ISOQ_ST_POS_RANGE.
+ * isoq_rope_table: fills dst (device, isoq_rope_table_bytes(d, max_pos) bytes) with
+ *   cos / sin (pos * base^(-2i/d)) for pos < max_pos, i < d/2, computed in binary64 on the
+ *   device and rounded to binary32 (RoFormer frequencies).  Asynchronous on `stream`.
+ *   Errors: ISOQ_E_ARG (null, max_pos < 1, base <= 1), ISOQ_E_DIM.
+ * isoq_quantize_append_layers: the same tokens (seq_ids, positions, element type, count)
+ *   appended to n_layers caches in one launch per 32 layers (a decode step's appends for
+ *   a whole model): params[l], caches[l], K[l], V[l] are layer l's (host arrays of
+ *   pointers).  All layers share d, n_kv_heads and bits (else ISOQ_E_DIM); rope_table may
+ *   be NULL (no RoPE) or as for isoq_quantize_append_rope.  Per-layer errors as
+ *   isoq_quantize_append.
+ * ===================================================================================== */
+int isoq_quantize_append_rope(const isoq_params* params, const isoq_cache* cache, const void* K,
+                              const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
+                              const int32_t* positions, const float* rope_table,
+                              int rope_max_pos, void* stream);
+
+size_t isoq_rope_table_bytes(int d, int max_pos);
+
+int isoq_rope_table(float* dst, int d, int max_pos, double base, void* stream);
+
+int isoq_quantize_append_layers(const isoq_params* const* params,
+                                const isoq_cache* const* caches, const void* const* K,
+                                const void* const* V, int n_layers, int dtype, int n_tokens,
+                                const int32_t* seq_ids, const int32_t* positions,
+                                const float* rope_table, int rope_max_pos, void* stream);
+
+/* =======================================================================================
  * Decode attention on the packed cache (one query token per sequence).
  *
  * For sequence s and query head h (KV head g = h / (n_q_heads / n_kv_heads)):

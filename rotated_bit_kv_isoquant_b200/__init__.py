@@ -77,6 +77,10 @@ _SIGS = {
     "isoq_params_destroy": (None, [_p]),
     "isoq_block_bytes": (_sz, [_i, _i]),
     "isoq_quantize_append": (_i, [_p, _cp, _p, _p, _i, _i, _p, _p, _p]),
+    "isoq_quantize_append_rope": (_i, [_p, _cp, _p, _p, _i, _i, _p, _p, _p, _i, _p]),
+    "isoq_quantize_append_layers": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p, _p, _i, _p]),
+    "isoq_rope_table_bytes": (_sz, [_i, _i]),
+    "isoq_rope_table": (_i, [_p, _i, _i, ctypes.c_double, _p]),
     "isoq_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "isoq_decode_num_splits": (_i, [_i, _i, _i, _i, _i]),
     "isoq_decode_attention": (_i, [_p, _cp, _p, _i, _i, _i, _p, _i, _p, _f, _p, _sz, _p]),
@@ -243,6 +247,56 @@ def isoq_quantize_append(params: Params, cache: PagedCache, K, V, seq_ids, posit
         params.handle, ctypes.byref(cache.c), _dev_ptr(K, "K"), _dev_ptr(V, "V"), _dtype_code(K),
         n, _dev_ptr(seq_ids, "seq_ids", torch.int32), _dev_ptr(positions, "positions", torch.int32),
         _stream_ptr(stream)), "isoq_quantize_append")
+
+
+def isoq_rope_table(d: int, max_pos: int, base: float = 10000.0, device=None, stream=None):
+    """Device fp32 [max_pos][d/2][2] table of (cos, sin)(pos * base^(-2i/d)), computed in
+    fp64 on the GPU, for the fused RoPE quantize-append."""
+    import torch
+    nbytes = int(_lib.isoq_rope_table_bytes(d, max_pos))
+    if nbytes == 0:
+        raise IsoqError(ISOQ_E_DIM, "isoq_rope_table")
+    t = torch.empty((max_pos, d // 2, 2), dtype=torch.float32, device=device or "cuda")
+    _check(_lib.isoq_rope_table(t.data_ptr(), d, max_pos, float(base), _stream_ptr(stream)),
+           "isoq_rope_table")
+    return t
+
+
+def isoq_quantize_append_rope(params: Params, cache: PagedCache, K, V, seq_ids, positions,
+                              rope_table, stream=None) -> None:
+    """isoq_quantize_append with the rotary embedding applied to K (pre-RoPE keys) at each
+    token's position, from rope_table (isoq_rope_table)."""
+    import torch
+    if K.dtype != V.dtype or K.shape != V.shape:
+        raise ValueError("K and V must have the same shape and dtype")
+    _check(_lib.isoq_quantize_append_rope(
+        params.handle, ctypes.byref(cache.c), _dev_ptr(K, "K"), _dev_ptr(V, "V"), _dtype_code(K),
+        K.shape[0], _dev_ptr(seq_ids, "seq_ids", torch.int32),
+        _dev_ptr(positions, "positions", torch.int32),
+        _dev_ptr(rope_table, "rope_table", torch.float32), rope_table.shape[0],
+        _stream_ptr(stream)), "isoq_quantize_append_rope")
+
+
+def isoq_quantize_append_layers(params_list, caches, Ks, Vs, seq_ids, positions,
+                                rope_table=None, stream=None) -> None:
+    """One quantize-append of the same tokens into several layers' caches (one launch per
+    up to 32 layers): params_list, caches, Ks, Vs are per-layer sequences."""
+    import torch
+    n = len(params_list)
+    if not (n == len(caches) == len(Ks) == len(Vs)) or n == 0:
+        raise ValueError("one params, cache, K and V per layer")
+    if any(t.dtype != Ks[0].dtype or t.shape != Ks[0].shape for t in list(Ks) + list(Vs)):
+        raise ValueError("every layer's K and V must have the same shape and dtype")
+    P = (_p * n)(*[p.handle for p in params_list])
+    C = (_p * n)(*[ctypes.addressof(c.c) for c in caches])
+    Kp = (_p * n)(*[_dev_ptr(k, "K") for k in Ks])
+    Vp = (_p * n)(*[_dev_ptr(v, "V") for v in Vs])
+    _check(_lib.isoq_quantize_append_layers(
+        P, C, Kp, Vp, n, _dtype_code(Ks[0]), Ks[0].shape[0],
+        _dev_ptr(seq_ids, "seq_ids", torch.int32), _dev_ptr(positions, "positions", torch.int32),
+        _dev_ptr(rope_table, "rope_table", torch.float32) if rope_table is not None else None,
+        rope_table.shape[0] if rope_table is not None else 0, _stream_ptr(stream)),
+        "isoq_quantize_append_layers")
 
 
 def isoq_decode_workspace_bytes(n_seqs, n_q_heads, n_kv_heads, d, max_seq_len) -> int:

@@ -289,34 +289,122 @@ size_t isoq_block_bytes_v(int d, int bits, int page_size) {
 
 size_t isoq_block_bytes(int d, int page_size) { return isoq_block_bytes_v(d, 3, page_size); }
 
-int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, const void* K,
-                         const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
-                         const int32_t* positions, void* stream) {
-  int rc = check_cache(cache, params);
-  if (rc) return rc;
+}  // extern "C"
+
+namespace {
+
+// Shared by the quantize-append entry points: every layer's params and cache are checked
+// (same d, heads and bits), then the layers go out in launches of up to kMaxLayers.
+int quantize_common(const isoq_params* const* params, const isoq_cache* const* caches,
+                    const void* const* K, const void* const* V, int n_layers, int dtype,
+                    int n_tokens, const int32_t* seq_ids, const int32_t* positions,
+                    const float* rope, int rope_max_pos, void* stream) {
+  if (!params || !caches || !K || !V || n_layers < 1) return ISOQ_E_ARG;
+  for (int i = 0; i < n_layers; ++i) {
+    const int rc = check_cache(caches[i], params[i]);
+    if (rc) return rc;
+    if (params[i]->d != params[0]->d || params[i]->n_kv_heads != params[0]->n_kv_heads ||
+        params[i]->bits != params[0]->bits)
+      return ISOQ_E_DIM;
+  }
   if (n_tokens < 0 || !valid_dtype(dtype)) return ISOQ_E_ARG;
+  if (rope && rope_max_pos < 1) return ISOQ_E_ARG;
   if (n_tokens == 0) return ISOQ_OK;
-  if (!K || !V || !seq_ids || !positions) return ISOQ_E_ARG;
-  if ((rc = check_device(params))) return rc;
-  isoq::QuantizeArgs a;
-  a.params = params->dev;
-  a.bits = params->bits;
-  a.mats = params->dev_mat;
-  a.blocks = cache->blocks;
-  a.page_table = cache->page_table;
-  a.n_pages = cache->n_pages;
-  a.max_pages = cache->max_pages_per_seq;
-  a.n_seqs = cache->n_seqs;
-  a.n_kv_heads = cache->n_kv_heads;
-  a.d = cache->d;
-  a.K = K;
-  a.V = V;
+  if (!seq_ids || !positions) return ISOQ_E_ARG;
+  for (int i = 0; i < n_layers; ++i) {
+    if (!K[i] || !V[i]) return ISOQ_E_ARG;
+    const int rc = check_device(params[i]);
+    if (rc) return rc;
+  }
+  isoq::QuantizeArgs a{};
+  a.bits = params[0]->bits;
+  a.n_kv_heads = params[0]->n_kv_heads;
+  a.d = params[0]->d;
   a.dtype = dtype;
   a.n_tokens = n_tokens;
   a.seq_ids = seq_ids;
   a.positions = positions;
-  a.status = cache->status;
-  cudaError_t e = isoq::launch_quantize_append(a, (cudaStream_t)stream, sm_count());
+  a.rope = rope;
+  a.rope_max_pos = rope ? rope_max_pos : 0;
+  for (int l0 = 0; l0 < n_layers; l0 += isoq::kMaxLayers) {
+    a.layers.n = n_layers - l0 < isoq::kMaxLayers ? n_layers - l0 : isoq::kMaxLayers;
+    for (int i = 0; i < a.layers.n; ++i) {
+      const isoq_params* p = params[l0 + i];
+      const isoq_cache* c = caches[l0 + i];
+      isoq::QuantLayer& L = a.layers.l[i];
+      L.mats = p->dev_mat;
+      L.blocks = c->blocks;
+      L.page_table = c->page_table;
+      L.K = K[l0 + i];
+      L.V = V[l0 + i];
+      L.status = c->status;
+      L.n_pages = c->n_pages;
+      L.max_pages = c->max_pages_per_seq;
+      L.n_seqs = c->n_seqs;
+    }
+    cudaError_t e = isoq::launch_quantize_append(a, (cudaStream_t)stream, sm_count());
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return ISOQ_OK;
+}
+
+// Device fp64 cos/sin table of the rotary embedding.
+__global__ void rope_table_kernel(float* dst, int d, int max_pos, double base) {
+  const int h = d / 2;
+  const long long n = (long long)max_pos * h;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int pos = (int)(i / h), k = (int)(i % h);
+    const double theta = pow(base, -2.0 * k / d);
+    double sn, cs;
+    sincos((double)pos * theta, &sn, &cs);
+    dst[2 * i] = (float)cs;
+    dst[2 * i + 1] = (float)sn;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int isoq_quantize_append(const isoq_params* params, const isoq_cache* cache, const void* K,
+                         const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
+                         const int32_t* positions, void* stream) {
+  return quantize_common(&params, &cache, &K, &V, 1, dtype, n_tokens, seq_ids, positions,
+                         nullptr, 0, stream);
+}
+
+int isoq_quantize_append_rope(const isoq_params* params, const isoq_cache* cache, const void* K,
+                              const void* V, int dtype, int n_tokens, const int32_t* seq_ids,
+                              const int32_t* positions, const float* rope_table,
+                              int rope_max_pos, void* stream) {
+  if (!rope_table) return ISOQ_E_ARG;
+  return quantize_common(&params, &cache, &K, &V, 1, dtype, n_tokens, seq_ids, positions,
+                         rope_table, rope_max_pos, stream);
+}
+
+int isoq_quantize_append_layers(const isoq_params* const* params,
+                                const isoq_cache* const* caches, const void* const* K,
+                                const void* const* V, int n_layers, int dtype, int n_tokens,
+                                const int32_t* seq_ids, const int32_t* positions,
+                                const float* rope_table, int rope_max_pos, void* stream) {
+  return quantize_common(params, caches, K, V, n_layers, dtype, n_tokens, seq_ids, positions,
+                         rope_table, rope_max_pos, stream);
+}
+
+size_t isoq_rope_table_bytes(int d, int max_pos) {
+  if (!supported_d(d) || max_pos < 1) return 0;
+  return (size_t)max_pos * d * sizeof(float);
+}
+
+int isoq_rope_table(float* dst, int d, int max_pos, double base, void* stream) {
+  if (!dst || max_pos < 1 || !(base > 1.0)) return ISOQ_E_ARG;
+  if (!supported_d(d)) return ISOQ_E_DIM;
+  const long long n = (long long)max_pos * (d / 2);
+  long long grid = (n + 255) / 256;
+  if (grid > 4096) grid = 4096;
+  rope_table_kernel<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(dst, d, max_pos, base);
+  cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
 }
 

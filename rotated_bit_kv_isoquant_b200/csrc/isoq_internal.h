@@ -9,20 +9,35 @@ struct isoq_params;
 
 namespace isoq {
 
-struct QuantizeArgs {
-  const float* params;  // device: the parameters as generated (unused by the kernels)
+// One layer's cache and inputs for a quantize-append launch.
+struct QuantLayer {
   const float* mats;    // device [H][d/4][4][4]: block rotations as matrices
-  int bits;             // bits per code (2, 3, 4)
   uint8_t* blocks;
   const int32_t* page_table;
-  int n_pages, max_pages, n_seqs, n_kv_heads, d;
   const void* K;
   const void* V;
+  uint32_t* status;
+  int n_pages, max_pages, n_seqs;
+};
+
+// Layers quantised by one launch (blockIdx.y = layer), passed by value as a kernel
+// parameter (32 * 64 bytes).
+constexpr int kMaxLayers = 32;
+struct QuantLayers {
+  QuantLayer l[kMaxLayers];
+  int n;
+};
+
+struct QuantizeArgs {
+  QuantLayers layers;
+  int bits;             // bits per code (2, 3, 4), the same for every layer
+  int n_kv_heads, d;
   int dtype;
   int n_tokens;
   const int32_t* seq_ids;
   const int32_t* positions;
-  uint32_t* status;
+  const float* rope;    // optional device [rope_max_pos][d/2][2] (cos, sin): RoPE applied to K
+  int rope_max_pos;
 };
 
 struct DecodeArgs {

@@ -54,11 +54,18 @@ __host__ __device__ constexpr int slot2(int e) {
 // (two independent chains for the scheduler).
 template <int D, typename T>
 __global__ void __launch_bounds__(256)
-    quantize_append_kernel(const float* __restrict__ mats, uint8_t* __restrict__ blocks,
-                           const int32_t* __restrict__ page_table, int n_pages, int max_pages,
-                           int n_seqs, int H, const T* __restrict__ K, const T* __restrict__ V,
-                           int n_tokens, const int32_t* __restrict__ seq_ids,
-                           const int32_t* __restrict__ positions, uint32_t* status) {
+    quantize_append_kernel(const __grid_constant__ QuantLayers layers, int H, int n_tokens,
+                           const int32_t* __restrict__ seq_ids,
+                           const int32_t* __restrict__ positions,
+                           const float* __restrict__ rope, int rope_max_pos) {
+  const QuantLayer& L = layers.l[blockIdx.y];  // this launch row's layer
+  const float* __restrict__ mats = L.mats;
+  uint8_t* __restrict__ blocks = L.blocks;
+  const int32_t* __restrict__ page_table = L.page_table;
+  const int n_pages = L.n_pages, max_pages = L.max_pages, n_seqs = L.n_seqs;
+  const T* __restrict__ K = static_cast<const T*>(L.K);
+  const T* __restrict__ V = static_cast<const T*>(L.V);
+  uint32_t* status = L.status;
   constexpr int E = D / 32;       // elements per lane
   constexpr int NB = E / 4;       // quaternion blocks per lane
   constexpr int CB = code_bytes(D);
@@ -78,7 +85,7 @@ __global__ void __launch_bounds__(256)
     int phys = -1;
     if (sid < 0 || sid >= n_seqs) {
       bad = ISOQ_ST_SEQ_RANGE;
-    } else if (pos < 0 || (pos >> 6) >= max_pages) {
+    } else if (pos < 0 || (pos >> 6) >= max_pages || (rope && pos >= rope_max_pos)) {
       bad = ISOQ_ST_POS_RANGE;
     } else {
       phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
@@ -96,6 +103,23 @@ __global__ void __launch_bounds__(256)
       float x[2][E];
       load_vec<T, E>(K + row, x[0]);
       load_vec<T, E>(V + row, x[1]);
+      if (rope) {  // RoPE of K at its position: dims (i, i + D/2) live on lanes l, l ^ 16
+        float pv[E];
+#pragma unroll
+        for (int j = 0; j < E; ++j) pv[j] = __shfl_xor_sync(kFull, x[0][j], 16);
+        const float4* tab = reinterpret_cast<const float4*>(rope + (size_t)pos * D) +
+                            (E * (lane & 15)) / 2;
+#pragma unroll
+        for (int jj = 0; jj < E / 2; ++jj) {
+          const float4 cs = __ldg(tab + jj);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 2 * jj + e;
+            const float c = e ? cs.z : cs.x, sn = e ? cs.w : cs.y;
+            x[0][j] = lane < 16 ? fmaf(x[0][j], c, -pv[j] * sn) : fmaf(pv[j], sn, x[0][j] * c);
+          }
+        }
+      }
 
       // a1: norms (both vectors' reductions interleaved)
       float ss[2] = {0.f, 0.f};
@@ -229,13 +253,20 @@ constexpr int kTpvThreads = 128;
 #define ISOQ_TPV_MINB 3
 #endif
 
-template <typename T, int BITS>
+template <typename T, int BITS, bool ROPE>
 __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
-    quantize_tpv_kernel(const float* __restrict__ mats, uint8_t* __restrict__ blocks,
-                        const int32_t* __restrict__ page_table, int n_pages, int max_pages,
-                        int n_seqs, int H, const T* __restrict__ K, const T* __restrict__ V,
-                        int n_tokens, const int32_t* __restrict__ seq_ids,
-                        const int32_t* __restrict__ positions, uint32_t* status) {
+    quantize_tpv_kernel(const __grid_constant__ QuantLayers layers, int H, int n_tokens,
+                        const int32_t* __restrict__ seq_ids,
+                        const int32_t* __restrict__ positions, const float* __restrict__ rope,
+                        int rope_max_pos) {
+  const QuantLayer& L = layers.l[blockIdx.y];  // this launch row's layer
+  const float* __restrict__ mats = L.mats;
+  uint8_t* __restrict__ blocks = L.blocks;
+  const int32_t* __restrict__ page_table = L.page_table;
+  const int n_pages = L.n_pages, max_pages = L.max_pages, n_seqs = L.n_seqs;
+  const T* __restrict__ K = static_cast<const T*>(L.K);
+  const T* __restrict__ V = static_cast<const T*>(L.V);
+  uint32_t* status = L.status;
   constexpr int D = 128, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
   constexpr int NT = (1 << (BITS - 1)) - 1;  // positive thresholds
   constexpr uint32_t kZeroCode = 1u << (BITS - 1);
@@ -261,7 +292,7 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     int phys = -1;
     if (sid < 0 || sid >= n_seqs) {
       bad = ISOQ_ST_SEQ_RANGE;
-    } else if (pos < 0 || (pos >> 6) >= max_pages) {
+    } else if (pos < 0 || (pos >> 6) >= max_pages || (rope && pos >= rope_max_pos)) {
       bad = ISOQ_ST_POS_RANGE;
     } else {
       phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
@@ -277,6 +308,18 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     const T* src = (kind == 0 ? K : V) + ((size_t)t * H + h) * D;
 #pragma unroll
     for (int i = 0; i < D; i += 8) load_vec<T, 8>(src + i, *reinterpret_cast<float(*)[8]>(x + i));
+    if (ROPE && kind == 0) {  // RoPE of K at its position: dims (i, i + D/2)
+      const float4* tab = reinterpret_cast<const float4*>(rope + (size_t)pos * D);
+#pragma unroll
+      for (int i = 0; i < D / 4; ++i) {
+        const float4 cs = __ldg(tab + i);
+        const float a0 = x[2 * i], b0 = x[2 * i + D / 2], a1 = x[2 * i + 1], b1 = x[2 * i + 1 + D / 2];
+        x[2 * i] = fmaf(a0, cs.x, -b0 * cs.y);
+        x[2 * i + D / 2] = fmaf(a0, cs.y, b0 * cs.x);
+        x[2 * i + 1] = fmaf(a1, cs.z, -b1 * cs.w);
+        x[2 * i + 1 + D / 2] = fmaf(a1, cs.w, b1 * cs.z);
+      }
+    }
 
     // a1: norm (four partial sums)
     float ss0 = 0.f, ss1 = 0.f, ss2 = 0.f, ss3 = 0.f;
@@ -373,43 +416,41 @@ static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm
   const long long warps = a.n_tokens;  // one warp per token
   const int wpb = 8;
   long long grid = (warps + wpb - 1) / wpb;
-  const long long cap = (long long)n_sm * 16;
+  const long long cap = (long long)n_sm * 16 / a.layers.n + 1;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  quantize_append_kernel<D, T><<<(unsigned)grid, wpb * 32, 0, stream>>>(
-      a.mats, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_seqs, a.n_kv_heads,
-      static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.n_tokens, a.seq_ids, a.positions,
-      a.status);
+  quantize_append_kernel<D, T><<<dim3((unsigned)grid, a.layers.n), wpb * 32, 0, stream>>>(
+      a.layers, a.n_kv_heads, a.n_tokens, a.seq_ids, a.positions, a.rope, a.rope_max_pos);
   return cudaGetLastError();
 }
 
-template <typename T, int BITS>
+template <typename T, int BITS, bool ROPE>
 static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   const size_t smem = (size_t)a.n_kv_heads * 32 * 16 * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T, BITS>,
+    cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T, BITS, ROPE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   const long long tasks = (long long)a.n_kv_heads * 2 * ((a.n_tokens + 31) / 32);
   const int wpb = kTpvThreads / 32;
   long long grid = (tasks + wpb - 1) / wpb;
-  const long long cap = (long long)n_sm * 3 * 8;
+  const long long cap = (long long)n_sm * 3 * 8 / a.layers.n + 1;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  quantize_tpv_kernel<T, BITS><<<(unsigned)grid, kTpvThreads, smem, stream>>>(
-      a.mats, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_seqs, a.n_kv_heads,
-      static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.n_tokens, a.seq_ids, a.positions,
-      a.status);
+  quantize_tpv_kernel<T, BITS, ROPE><<<dim3((unsigned)grid, a.layers.n), kTpvThreads, smem,
+                                       stream>>>(
+      a.layers, a.n_kv_heads, a.n_tokens, a.seq_ids, a.positions, a.rope, a.rope_max_pos);
   return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_tpv_b(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  const bool r = a.rope != nullptr;
   switch (a.bits) {
-    case 2: return launch_tpv<T, 2>(a, stream, n_sm);
-    case 3: return launch_tpv<T, 3>(a, stream, n_sm);
-    case 4: return launch_tpv<T, 4>(a, stream, n_sm);
+    case 2: return r ? launch_tpv<T, 2, true>(a, stream, n_sm) : launch_tpv<T, 2, false>(a, stream, n_sm);
+    case 3: return r ? launch_tpv<T, 3, true>(a, stream, n_sm) : launch_tpv<T, 3, false>(a, stream, n_sm);
+    case 4: return r ? launch_tpv<T, 4, true>(a, stream, n_sm) : launch_tpv<T, 4, false>(a, stream, n_sm);
   }
   return cudaErrorInvalidValue;
 }

@@ -150,8 +150,10 @@ def _rope_(k: torch.Tensor, pos0: int) -> torch.Tensor:
     return torch.cat([a * c - b * s, a * s + b * c], dim=-1)
 
 
-def _kv_chunk(cfg: Workload, tag: int, seq: int, chunk: int, device) -> torch.Tensor:
-    """fp32 [CHUNK][n_kv_heads][d] values of K (tag _K) or V (tag _V) for one chunk."""
+def _kv_chunk(cfg: Workload, tag: int, seq: int, chunk: int, device,
+              rope: bool = True) -> torch.Tensor:
+    """fp32 [CHUNK][n_kv_heads][d] values of K (tag _K) or V (tag _V) for one chunk
+    (rope=False: a RoPE workload's keys before the rotary embedding)."""
     g = _gen(device, _seed(cfg.idx, tag, seq, chunk))
     shape = (CHUNK, cfg.n_kv_heads, cfg.d)
     dist = cfg.kv_dist
@@ -167,7 +169,7 @@ def _kv_chunk(cfg: Workload, tag: int, seq: int, chunk: int, device) -> torch.Te
         n_ch = round(0.02 * cfg.d)
         x *= _outlier_mult(cfg.n_kv_heads, cfg.d, n_ch, 10.0,
                            _seed(cfg.idx, _KOUT if tag == _K else _VOUT, 0, 0), device)
-        if tag == _K:
+        if tag == _K and rope:
             x = _rope_(x, chunk * CHUNK)
     elif dist == "student_t5":
         x = _student_t(shape, 5, g, device)
@@ -179,15 +181,16 @@ def _kv_chunk(cfg: Workload, tag: int, seq: int, chunk: int, device) -> torch.Te
     return x
 
 
-def kv_tokens(cfg: Workload, seq: int, start: int, count: int, device="cpu"):
+def kv_tokens(cfg: Workload, seq: int, start: int, count: int, device="cpu", rope: bool = True):
     """K, V of tokens [start, start+count) of sequence `seq`: [count][n_kv_heads][d] in
-    cfg.in_dtype.  Any range can be regenerated independently (chunked seeds)."""
+    cfg.in_dtype.  Any range can be regenerated independently (chunked seeds).  rope=False
+    gives a RoPE workload's keys before the rotary embedding (for the fused epilogue)."""
     outs = []
     for tag in (_K, _V):
         parts = []
         c0, c1 = start // CHUNK, (start + count - 1) // CHUNK
         for c in range(c0, c1 + 1):
-            x = _kv_chunk(cfg, tag, seq, c, device)
+            x = _kv_chunk(cfg, tag, seq, c, device, rope=rope)
             lo = max(start, c * CHUNK) - c * CHUNK
             hi = min(start + count, (c + 1) * CHUNK) - c * CHUNK
             parts.append(x[lo:hi])

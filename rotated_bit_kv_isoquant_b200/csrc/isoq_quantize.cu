@@ -14,35 +14,33 @@
 // squares.  Codes are decided against the thresholds scaled by the norm (no division),
 // packed with shuffles into the 12-byte group layout of isoq.h and written as 16-byte
 // stores.
+#include <math_constants.h>
+
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 
 namespace isoq {
 
-// Code of one rotated coordinate z (scaled by sqrt(d)) against thresholds T[k] = n * tau_k
-// (tau = 0.50055, 1.05, 1.748, the positive midpoints; the codebook is symmetric).  The
-// definition code = #{j : z >= t_j} over t = (-T3, -T2, -T1, 0, T1, T2, T3) equals
-//   z >= 0: 4 + #{k : |z| >= T_k}         z < 0: 3 - #{k : |z| > T_k}
-// and for non-negative floats "a > T" is "bits(a) - 1 >= bits(T)", so one set of integer
-// compares on bits(|z|) - [z < 0] serves both signs exactly; 3 - m = (4 + m) ^ 7.
-__device__ __forceinline__ uint32_t code_of(float z, const uint32_t (&tb)[3]) {
-  const uint32_t neg = z < 0.f ? 1u : 0u;
-  const uint32_t ai = (__float_as_uint(z) & 0x7fffffffu) - neg;
-  const uint32_t m = (ai >= tb[0] ? 1u : 0u) + (ai >= tb[1] ? 1u : 0u) + (ai >= tb[2] ? 1u : 0u);
-  return (4u + m) ^ (neg * 7u);
-}
-
-// The same decision for a 2^BITS-level symmetric codebook: T[k] = n * (positive threshold
-// k), k < 2^(BITS-1) - 1; code = (half + m) ^ (neg * (2 half - 1)), half = 2^(BITS-1).
+// The stored field of one rotated coordinate z (scaled by sqrt(d)) on the FMA pipe, with
+// TB[k] = n * (positive threshold k) * 2^64 (+inf for a zero vector).  Each
+// sat(|z| 2^64 - TB[k]) is 1 when |z| > n t_k and 0 below; a coordinate exactly on a
+// threshold (a difference of 0, the only case decided differently from the >= of the
+// definition) lies inside any parity band around the thresholds.  With m thresholds
+// exceeded, code = half + m for z >= 0 and half - 1 - m for z < 0 (-0 counts as +0, so a
+// zero vector codes half), i.e. code = (half - 0.5) + sign(z) (m + 0.5).  4 bits store the
+// sign-magnitude nibble m + 8 [z < 0] instead.
 template <int BITS>
-__device__ __forceinline__ uint32_t code_of_b(float z, const uint32_t (&tb)[(1 << (BITS - 1)) - 1]) {
-  constexpr uint32_t half = 1u << (BITS - 1);
-  const uint32_t neg = z < 0.f ? 1u : 0u;
-  const uint32_t ai = (__float_as_uint(z) & 0x7fffffffu) - neg;
-  uint32_t m = 0;
+__device__ __forceinline__ uint32_t code_sat(float z, const float (&TB)[(1 << (BITS - 1)) - 1]) {
+  constexpr int NT = (1 << (BITS - 1)) - 1;
+  constexpr float kHalf = (float)(1 << (BITS - 1));
+  const float zp = z + 0.0f;  // -0 -> +0
+  const float a = fabsf(zp);
+  float acc = 0.5f;
 #pragma unroll
-  for (int k = 0; k < (int)half - 1; ++k) m += ai >= tb[k] ? 1u : 0u;
-  return (half + m) ^ (neg * (2 * half - 1));
+  for (int k = 0; k < NT; ++k) acc += __saturatef(fmaf(a, 0x1p64f, -TB[k]));
+  const float sg = copysignf(1.0f, zp);
+  const float cf = BITS == 4 ? fmaf(-4.0f, sg, acc + 3.5f) : fmaf(sg, acc, kHalf - 0.5f);
+  return __float_as_uint(cf + 8388608.0f) & 0xFu;  // small exact integer in the mantissa
 }
 
 // 2-bit layout: the slot (0..15) of dim e (0..15) of a 16-dim word.
@@ -190,13 +188,14 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         // a4: codes against n * tau (a zero vector codes 4 everywhere)
-        uint32_t tb[3];
+        float TB[3];
 #pragma unroll
-        for (int k = 0; k < 3; ++k) tb[k] = __float_as_uint(n[kv] * threshold_f32(4 + k));
+        for (int k = 0; k < 3; ++k)
+          TB[k] = n[kv] == 0.f ? CUDART_INF_F : n[kv] * threshold_f32(4 + k) * 0x1p64f;
         uint32_t nib = 0;  // this lane's codes, one per nibble
 #pragma unroll
         for (int i = 0; i < E; ++i) {
-          const uint32_t c = n[kv] == 0.f ? 4u : code_of(z[kv][i], tb);
+          const uint32_t c = code_sat<3>(z[kv][i], TB);
           nib |= c << (4 * i);
         }
 
@@ -269,7 +268,6 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
   uint32_t* status = L.status;
   constexpr int D = 128, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
   constexpr int NT = (1 << (BITS - 1)) - 1;  // positive thresholds
-  constexpr uint32_t kZeroCode = 1u << (BITS - 1);
   extern __shared__ __align__(16) float smats[];  // [H][32 blocks][16]
   for (int i = threadIdx.x; i < H * (D / 4) * 16 / 4; i += blockDim.x)
     reinterpret_cast<float4*>(smats)[i] = __ldg(reinterpret_cast<const float4*>(mats) + i);
@@ -347,9 +345,10 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     }
 
     // a3 + a4: rotation block (matrix from shared memory) and codes, block by block
-    uint32_t tb[NT];
+    float TB[NT];
 #pragma unroll
-    for (int k = 0; k < NT; ++k) tb[k] = __float_as_uint(n * pos_threshold_f32(BITS, k));
+    for (int k = 0; k < NT; ++k)
+      TB[k] = n == 0.f ? CUDART_INF_F : n * pos_threshold_f32(BITS, k) * 0x1p64f;
     const float4* mh = reinterpret_cast<const float4*>(smats) + (size_t)h * (D / 4) * 4;
     uint32_t rec[CB / 4];
     uint32_t nib[D / 8];  // 3 bits: nibble words, word j holds dims 8j..8j+7
@@ -366,18 +365,15 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
       if constexpr (BITS == 3) {
         uint32_t w = (b & 1) ? nib[b >> 1] : 0u;
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-          const uint32_t c = n == 0.f ? kZeroCode : code_of(z[rr], tb);
-          w |= c << (4 * (4 * (b & 1) + rr));
-        }
+        for (int rr = 0; rr < 4; ++rr) w |= code_sat<3>(z[rr], TB) << (4 * (4 * (b & 1) + rr));
         nib[b >> 1] = w;
       } else {
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           const int dim = 4 * b + rr;
-          const uint32_t c = n == 0.f ? kZeroCode : code_of_b<BITS>(z[rr], tb);
-          if constexpr (BITS == 4)  // sign-magnitude nibble
-            rec[dim >> 3] |= (c ^ ((c & 8u) ? 8u : 15u)) << (4 * (dim & 7));
+          const uint32_t c = code_sat<BITS>(z[rr], TB);  // 4 bits: the sign-magnitude nibble
+          if constexpr (BITS == 4)
+            rec[dim >> 3] |= c << (4 * (dim & 7));
           else
             rec[dim >> 4] |= c << (2 * slot2(dim & 15));
         }

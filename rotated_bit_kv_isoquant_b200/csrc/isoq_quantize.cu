@@ -268,21 +268,68 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
   uint32_t* status = L.status;
   constexpr int D = 128, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
   constexpr int NT = (1 << (BITS - 1)) - 1;  // positive thresholds
-  extern __shared__ __align__(16) float smats[];  // [H][32 blocks][16]
+  // shared memory: the heads' block matrices [H][32 blocks][16], then one vector slot per
+  // thread (padded so that a warp's 16-byte reads of its 32 slots hit distinct banks) into
+  // which the next task's vector is copied (cp.async) while the current one is processed
+  constexpr int VB = D * (int)sizeof(T), VS = VB + 16;
+  extern __shared__ __align__(16) float smats[];
   for (int i = threadIdx.x; i < H * (D / 4) * 16 / 4; i += blockDim.x)
     reinterpret_cast<float4*>(smats)[i] = __ldg(reinterpret_cast<const float4*>(mats) + i);
+  uint8_t* slot_mem = reinterpret_cast<uint8_t*>(smats + H * (D / 4) * 16) + threadIdx.x * VS;
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   const int chunks = (n_tokens + 31) >> 5;
   const int n_tasks = H * 2 * chunks;  // task = (32-token chunk, head, kind), chunk-major
-  for (int task = blockIdx.x * wpb + (threadIdx.x >> 5); task < n_tasks;
-       task += gridDim.x * wpb) {
+  const int stride = gridDim.x * wpb;
+  // copy this lane's vector of task tk into its slot (nothing for a missing token); the
+  // source address needs only the task, not the token's validity.  The copy is issued
+  // after this thread's reads of the slot's previous contents (program order, and the
+  // "memory" clobber keeps the compiler from moving them); its shared-memory write lands
+  // only once the global read has returned.
+  auto prefetch = [&](int tk) {
+    if (tk < n_tasks) {
+      const int ck = tk / (2 * H), rr = tk - ck * 2 * H;
+      const int tt = ck * 32 + lane;
+      if (tt < n_tokens) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(((rr & 1) == 0 ? K : V) +
+                                                              ((size_t)tt * H + (rr >> 1)) * D);
+#pragma unroll
+        for (int q = 0; q < VB / 16; ++q)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                           static_cast<uint32_t>(__cvta_generic_to_shared(slot_mem + 16 * q))),
+                       "l"(src + 16 * q)
+                       : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  int task = blockIdx.x * wpb + (threadIdx.x >> 5);
+  prefetch(task);
+  for (; task < n_tasks; task += stride) {
     const int chunk = task / (2 * H);
     const int r = task - chunk * 2 * H;
     const int h = r >> 1, kind = r & 1;
     const int t = chunk * 32 + lane;
+    // this task's vector: wait for the copy, read the slot, then start the next task's copy
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    float x[D];
+#pragma unroll
+    for (int i = 0; i < D; i += 8) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(slot_mem + i * sizeof(T));
+      if constexpr (sizeof(T) == 4) {
+        const uint4 raw2 = *reinterpret_cast<const uint4*>(slot_mem + (i + 4) * sizeof(T));
+        const uint32_t w[8] = {raw.x, raw.y, raw.z, raw.w, raw2.x, raw2.y, raw2.z, raw2.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[i + k] = __uint_as_float(w[k]);
+      } else {
+        const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[i + k] = to_f32<T>(e[k]);
+      }
+    }
+    prefetch(task + stride);
     if (t >= n_tokens) continue;
     const int sid = __ldg(seq_ids + t);
     const int pos = __ldg(positions + t);
@@ -301,11 +348,6 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
       continue;
     }
 
-    // load the vector (contiguous D elements)
-    float x[D];
-    const T* src = (kind == 0 ? K : V) + ((size_t)t * H + h) * D;
-#pragma unroll
-    for (int i = 0; i < D; i += 8) load_vec<T, 8>(src + i, *reinterpret_cast<float(*)[8]>(x + i));
     if (ROPE && kind == 0) {  // RoPE of K at its position: dims (i, i + D/2)
       const float4* tab = reinterpret_cast<const float4*>(rope + (size_t)pos * D);
 #pragma unroll
@@ -422,7 +464,8 @@ static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm
 
 template <typename T, int BITS, bool ROPE>
 static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
-  const size_t smem = (size_t)a.n_kv_heads * 32 * 16 * sizeof(float);
+  const size_t smem = (size_t)a.n_kv_heads * 32 * 16 * sizeof(float) +
+                      (size_t)kTpvThreads * (128 * sizeof(T) + 16);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T, BITS, ROPE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

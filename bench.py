@@ -90,18 +90,25 @@ def _peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def _kernel_sources_sha() -> str:
+_KERNEL_SOURCES = {
+    "decode": ["isoq_decode_mma.cu", "isoq_decode.cu", "isoq_ptx.cuh", "isoq_common.cuh"],
+    "quantize": ["isoq_quantize.cu", "isoq_common.cuh"],
+}
+
+
+def _kernel_sources_sha(kernel: str) -> str:
+    """Hash of the sources that build one kernel group (a profile summary records it)."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "rotated_bit_kv_isoquant_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for name in _KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "rotated_bit_kv_isoquant_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def _ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture in profiles/, if the kernel sources
-    have not changed since (else None)."""
-    sha = _kernel_sources_sha()
+    """DRAM bytes per launch recorded from an ncu capture in profiles/, if the kernel's
+    sources have not changed since (else None)."""
+    sha = _kernel_sources_sha(kernel)
     for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         txt = open(p).read()
         m_k = re.search(r"^kernel_group:\s*(\S+)", txt, re.M)

@@ -101,12 +101,18 @@ struct SplitPlan {
 // number of pages and at least min_pages pages when the context allows.
 SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len,
                       int n_q = 1) {
-  const bool tc = isoq::kUseTc128 && d == 128;
-  const int n_sm = sm_count() * (tc ? isoq::decode_tc_resident_ctas() : isoq::decode_resident_ctas(d));
-  const int min_pages = tc ? 8 : 16;  // per CTA: 4 tiles of 2 pages, or 4 pages per warp
-  const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const int group = n_kv_heads > 0 ? n_q_heads / n_kv_heads : 1;
-  const long long units = (long long)n_seqs * n_kv_heads * (((long long)n_q * group + 7) / 8);
+  // the shared-page multi-token kernel (64 rows per CTA, 2 CTAs per SM) when a chunk gives
+  // a KV head at least 16 rows; else the per-row kernel (8 rows per CTA)
+  const bool shared_mq = d == 128 && n_q > 1 && (long long)n_q * group >= 16;
+  const bool tc = !shared_mq && n_q == 1 && isoq::kUseTc128 && d == 128;
+  const int n_sm = sm_count() * (shared_mq ? 2 : tc ? isoq::decode_tc_resident_ctas()
+                                                    : isoq::decode_resident_ctas(d));
+  const int min_pages = shared_mq ? 4 : tc ? 8 : 16;  // pages per CTA worth a launch
+  const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
+  const int rows_per_cta = shared_mq ? 64 : 8;
+  const long long units =
+      (long long)n_seqs * n_kv_heads * (((long long)n_q * group + rows_per_cta - 1) / rows_per_cta);
   const long long target = (long long)n_sm * ISOQ_DEC_WAVES;
   long long want = units > 0 ? (target + units - 1) / units : 1;
   const long long cap = (max_pages + min_pages - 1) / min_pages;

@@ -70,6 +70,10 @@ cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int 
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
 // Resident CTAs per SM of that kernel for head dimension d on the current device.
 int decode_resident_ctas(int d);
+// Multi-token chunks with many rows per KV head (d = 128): the page dequantised once per
+// CTA into shared memory and shared by 64 (query token, head) rows (partials only).
+bool use_shared_mq(const DecodeArgs& a);
+cudaError_t launch_decode_split_mq(const DecodeArgs& a, cudaStream_t stream);
 // Tensor-memory (tcgen05) split kernel, head dimension 128 (partials only).
 cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t stream);
 int decode_tc_resident_ctas();

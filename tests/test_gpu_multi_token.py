@@ -95,7 +95,7 @@ def test_multi_token_causal_rows_see_only_their_prefix(run2):
         _, ref = run2.decode(Q=Q[:, i].contiguous(), lens=[L - n_q + i + 1], max_len=L)
         torch.cuda.synchronize()
         rel = ((out[:, i] - ref).norm() / ref.norm()).item()
-        assert rel < 1e-5, (i, rel)
+        assert rel < 1e-3, (i, rel)   # another kernel: rounding only; a causality error is O(1)
 
 
 @pytest.mark.parametrize("variant", ["batched_ragged_G4", "gqa1_d128", "gqa16_d128", "d256"])

@@ -48,6 +48,40 @@ __host__ __device__ constexpr int slot2(int e) {
   return e < 8 ? ((e & 1) ? (e >> 1) + 4 : (e >> 1)) : ((e & 1) ? ((e - 8) >> 1) + 12 : ((e - 8) >> 1) + 8);
 }
 
+// The same decision as code_sat, added into the sum W = sum coef * code of a 16-bit
+// half-word (coef = 16^nibble, or 4^slot at 2 bits): W gains coef * code minus the
+// sign-independent part coef * base, which the caller puts in W's initial value
+// (base = half - 0.5, or 4 at 4 bits).  z is never -0 here.  W stays an exact binary32
+// integer + 0.5 multiple below 2^17, and no per-code conversion or shift is needed.
+template <int BITS>
+__device__ __forceinline__ float add_code(float W, float z, float coef,
+                                          const float (&TB)[(1 << (BITS - 1)) - 1]) {
+  constexpr int NT = (1 << (BITS - 1)) - 1;
+  const float a = fabsf(z);
+  const float c = copysignf(coef, z);
+  float s[NT];
+#pragma unroll
+  for (int k = 0; k < NT; ++k) s[k] = __saturatef(fmaf(a, 0x1p64f, -TB[k]));
+  if constexpr (BITS == 2) {
+    return fmaf(c, s[0] + 0.5f, W);  // sign(z) (m + 0.5)
+  } else if constexpr (BITS == 3) {
+    return fmaf(c, (s[0] + s[1]) + (s[2] + 0.5f), W);
+  } else {  // m - 4 sign(z)
+    const float m = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + s[6]);
+    return fmaf(c, -4.0f, fmaf(coef, m, W));
+  }
+}
+template <int BITS>
+constexpr float code_base() { return BITS == 4 ? 4.0f : (float)(1 << (BITS - 1)) - 0.5f; }
+
+// Two half-word sums, each as the bits of W + 2^23 (0x4B000000 | W), joined into one word:
+// the high half's exponent bits leave the 32-bit product.
+__device__ __forceinline__ uint32_t join_halves(uint32_t lo, uint32_t hi) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, 65536, %2;" : "=r"(r) : "r"(hi), "r"(lo & 0xffffu));
+  return r;
+}
+
 // One warp per token; it walks the KV heads and, per head, quantises K and V together
 // (two independent chains for the scheduler).
 template <int D, typename T>
@@ -246,10 +280,17 @@ __global__ void __launch_bounds__(256)
 // (KV head, K|V) pair.  The whole vector lives in the thread's registers, so the WHT needs
 // no shuffles and every per-vector cost (addressing, validation, norm, packing) is paid
 // once per 128 elements instead of once per 4.  A warp's 32 vectors share the head, so the
-// 4x4 block matrices are read as warp-uniform (broadcast) 16-byte loads from shared memory.
+// 4x4 block matrices are read as warp-uniform (broadcast) 16-byte loads from shared memory;
+// they hold B H4, which takes over the WHT's two innermost stages.  Codes are summed into
+// exact float half-words (add_code) instead of being converted and shifted one by one.
+// The next task's vector, sequence and position are fetched while the current one is
+// processed; the page-table entry is loaded before the arithmetic and used after it.
 constexpr int kTpvThreads = 128;
 #ifndef ISOQ_TPV_MINB
 #define ISOQ_TPV_MINB 3
+#endif
+#ifndef ISOQ_TPV_WAVES  // grid cap in waves of resident CTAs
+#define ISOQ_TPV_WAVES 3
 #endif
 
 template <typename T, int BITS, bool ROPE>
@@ -273,10 +314,7 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
   // which the next task's vector is copied (cp.async) while the current one is processed
   constexpr int VB = D * (int)sizeof(T), VS = VB + 16;
   extern __shared__ __align__(16) float smats[];
-  for (int i = threadIdx.x; i < H * (D / 4) * 16 / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(smats)[i] = __ldg(reinterpret_cast<const float4*>(mats) + i);
   uint8_t* slot_mem = reinterpret_cast<uint8_t*>(smats + H * (D / 4) * 16) + threadIdx.x * VS;
-  __syncthreads();
 
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
@@ -288,7 +326,9 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
   // after this thread's reads of the slot's previous contents (program order, and the
   // "memory" clobber keeps the compiler from moving them); its shared-memory write lands
   // only once the global read has returned.
+  int nsid = -1, npos = -1;  // token of the prefetched task, read with its vector
   auto prefetch = [&](int tk) {
+    nsid = npos = -1;
     if (tk < n_tasks) {
       const int ck = tk / (2 * H), rr = tk - ck * 2 * H;
       const int tt = ck * 32 + lane;
@@ -301,12 +341,29 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
                            static_cast<uint32_t>(__cvta_generic_to_shared(slot_mem + 16 * q))),
                        "l"(src + 16 * q)
                        : "memory");
+        nsid = __ldg(seq_ids + tt);
+        npos = __ldg(positions + tt);
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
+  // the first task's copy is in flight while the block matrices are staged
   int task = blockIdx.x * wpb + (threadIdx.x >> 5);
   prefetch(task);
+  // The WHT's two innermost butterfly stages act inside each 4-element block as the 4x4
+  // Sylvester matrix H4[k][c] = (-1)^popc(k & c); the stages commute, so they are applied
+  // last and folded into the block matrix: smats holds B H4 for every block.
+  for (int i = threadIdx.x; i < H * (D / 4); i += blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(mats) + 4 * i;
+    float4* dst = reinterpret_cast<float4*>(smats) + 4 * i;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 v = __ldg(src + r);  // row r of B
+      dst[r] = make_float4((v.x + v.y) + (v.z + v.w), (v.x - v.y) + (v.z - v.w),
+                           (v.x + v.y) - (v.z + v.w), (v.x - v.y) - (v.z - v.w));
+    }
+  }
+  __syncthreads();
   for (; task < n_tasks; task += stride) {
     const int chunk = task / (2 * H);
     const int r = task - chunk * 2 * H;
@@ -329,19 +386,18 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
         for (int k = 0; k < 8; ++k) x[i + k] = to_f32<T>(e[k]);
       }
     }
+    const int sid = nsid, pos = npos;
     prefetch(task + stride);
     if (t >= n_tokens) continue;
-    const int sid = __ldg(seq_ids + t);
-    const int pos = __ldg(positions + t);
+    // the page-table entry is loaded here and first used by the stores at the end
     uint32_t bad = 0;
     int phys = -1;
     if (sid < 0 || sid >= n_seqs) {
       bad = ISOQ_ST_SEQ_RANGE;
-    } else if (pos < 0 || (pos >> 6) >= max_pages || (rope && pos >= rope_max_pos)) {
+    } else if (pos < 0 || (pos >> 6) >= max_pages || (ROPE && pos >= rope_max_pos)) {
       bad = ISOQ_ST_POS_RANGE;
     } else {
       phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
-      if (phys < 0 || phys >= n_pages) bad = ISOQ_ST_PAGE_RANGE;
     }
     if (bad) {
       set_status(status, bad);
@@ -372,9 +428,10 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     }
     const float n = sqrtf((ss0 + ss1) + (ss2 + ss3));
 
-    // a2: unnormalised WHT, natural order, all 7 butterfly stages in registers
+    // a2: unnormalised WHT, natural order: the five outer butterfly stages here, the two
+    // innermost ones inside the block matrices
 #pragma unroll
-    for (int hs = 1; hs < D; hs <<= 1) {
+    for (int hs = 4; hs < D; hs <<= 1) {
 #pragma unroll
       for (int i = 0; i < D; i += 2 * hs) {
 #pragma unroll
@@ -386,52 +443,56 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
       }
     }
 
-    // a3 + a4: rotation block (matrix from shared memory) and codes, block by block
+    // a3 + a4: rotation (B H4 of each block, from shared memory) and codes.  The codes of a
+    // 16-bit half of a packed word (4 dims at 3 and 4 bits, 8 at 2 bits) are summed as an
+    // exact float W = sum coef * code, converted once per half-word.
     float TB[NT];
 #pragma unroll
     for (int k = 0; k < NT; ++k)
       TB[k] = n == 0.f ? CUDART_INF_F : n * pos_threshold_f32(BITS, k) * 0x1p64f;
     const float4* mh = reinterpret_cast<const float4*>(smats) + (size_t)h * (D / 4) * 4;
-    uint32_t rec[CB / 4];
-    uint32_t nib[D / 8];  // 3 bits: nibble words, word j holds dims 8j..8j+7
+    constexpr int HPB = BITS == 2 ? 2 : 1;  // blocks per 16-bit half-word
+    uint32_t half[D / 4 / HPB];
 #pragma unroll
-    for (int i = 0; i < CB / 4; ++i) rec[i] = 0u;
+    for (int hw = 0; hw < D / 4 / HPB; ++hw) {
+      float W = code_base<BITS>() * (BITS == 2 ? 21845.0f : 4369.0f);  // sum coef * base
 #pragma unroll
-    for (int b = 0; b < D / 4; ++b) {
-      float z[4];
-#pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const float4 m = mh[4 * b + rr];
-        z[rr] = fmaf(m.w, x[4 * b + 3], fmaf(m.z, x[4 * b + 2], fmaf(m.y, x[4 * b + 1], m.x * x[4 * b])));
-      }
-      if constexpr (BITS == 3) {
-        uint32_t w = (b & 1) ? nib[b >> 1] : 0u;
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) w |= code_sat<3>(z[rr], TB) << (4 * (4 * (b & 1) + rr));
-        nib[b >> 1] = w;
-      } else {
+      for (int hb = 0; hb < HPB; ++hb) {
+        const int b = hw * HPB + hb;
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
-          const int dim = 4 * b + rr;
-          const uint32_t c = code_sat<BITS>(z[rr], TB);  // 4 bits: the sign-magnitude nibble
-          if constexpr (BITS == 4)
-            rec[dim >> 3] |= c << (4 * (dim & 7));
-          else
-            rec[dim >> 4] |= c << (2 * slot2(dim & 15));
+          const float4 m = mh[4 * b + rr];
+          // the chain starts from +0, so z is never -0 (which would code as negative)
+          const float z = fmaf(m.w, x[4 * b + 3],
+                               fmaf(m.z, x[4 * b + 2], fmaf(m.y, x[4 * b + 1], fmaf(m.x, x[4 * b], 0.0f))));
+          const int e = 4 * hb + rr;  // dim inside the half-word's dims
+          const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + e) & 7)))
+                                       : (float)(1 << (4 * e));
+          W = add_code<BITS>(W, z, coef, TB);
         }
       }
+      half[hw] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W (W in [0, 65535])
     }
-
-    // a5: pack (3 bits): per 32-dim group, words 0..2 = nibble words + bit 3 from the
-    // trailing 8 codes
+    uint32_t rec[CB / 4];
     if constexpr (BITS == 3) {
+      // a5: per 32-dim group, words 0..2 = nibble words of dims 8j..8j+7 with bit 3 taken
+      // from the group's trailing 8 codes (bit 2 - j of each)
+      uint32_t nib[D / 8];
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) nib[j] = join_halves(half[2 * j], half[2 * j + 1]);
 #pragma unroll
       for (int g = 0; g < D / 32; ++g) {
         const uint32_t N3 = nib[4 * g + 3];
 #pragma unroll
-        for (int j = 0; j < 3; ++j)
-          rec[3 * g + j] = nib[4 * g + j] | (((N3 >> (2 - j)) & 0x11111111u) << 3);
+        for (int j = 0; j < 3; ++j) rec[3 * g + j] = nib[4 * g + j] | ((N3 << (j + 1)) & 0x88888888u);
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CB / 4; ++j) rec[j] = join_halves(half[2 * j], half[2 * j + 1]);
+    }
+    if (phys < 0 || phys >= n_pages) {
+      set_status(status, ISOQ_ST_PAGE_RANGE);
+      continue;
     }
     uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
     const int slot = pos & (kPage - 1);
@@ -474,7 +535,7 @@ static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_
   const long long tasks = (long long)a.n_kv_heads * 2 * ((a.n_tokens + 31) / 32);
   const int wpb = kTpvThreads / 32;
   long long grid = (tasks + wpb - 1) / wpb;
-  const long long cap = (long long)n_sm * 3 * 8 / a.layers.n + 1;
+  const long long cap = (long long)n_sm * ISOQ_TPV_MINB * ISOQ_TPV_WAVES / a.layers.n + 1;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   quantize_tpv_kernel<T, BITS, ROPE><<<dim3((unsigned)grid, a.layers.n), kTpvThreads, smem,

@@ -102,15 +102,15 @@ struct SplitPlan {
 SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_seq_len,
                       int n_q = 1) {
   const int group = n_kv_heads > 0 ? n_q_heads / n_kv_heads : 1;
-  // the shared-page multi-token kernel (64 rows per CTA, 2 CTAs per SM) when a chunk gives
-  // a KV head at least 16 rows; else the per-row kernel (8 rows per CTA)
+  // the multi-token kernels (64 or 128 rows per CTA, 2 CTAs per SM) when a chunk gives a
+  // KV head at least 16 rows; else the per-row kernel (8 rows per CTA)
   const bool shared_mq = d == 128 && n_q > 1 && (long long)n_q * group >= 16;
   const bool tc = !shared_mq && n_q == 1 && isoq::kUseTc128 && d == 128;
   const int n_sm = sm_count() * (shared_mq ? 2 : tc ? isoq::decode_tc_resident_ctas()
                                                     : isoq::decode_resident_ctas(d));
   const int min_pages = shared_mq ? 4 : tc ? 8 : 16;  // pages per CTA worth a launch
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
-  const int rows_per_cta = shared_mq ? 64 : 8;
+  const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group) : 8;
   const long long units =
       (long long)n_seqs * n_kv_heads * (((long long)n_q * group + rows_per_cta - 1) / rows_per_cta);
   const long long target = (long long)n_sm * ISOQ_DEC_WAVES;

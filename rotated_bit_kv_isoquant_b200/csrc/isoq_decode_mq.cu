@@ -485,6 +485,8 @@ bool use_shared_mq(const DecodeArgs& a) {
 }
 
 cudaError_t launch_decode_split_mq(const DecodeArgs& a, cudaStream_t stream) {
+  if (attention_rows_per_cta(a.d, a.n_q, a.n_q_heads / a.n_kv_heads) == 128)
+    return launch_decode_split_mqtc(a, stream);
   switch (a.bits) {
     case 2: return launch_mq_b<2>(a, stream);
     case 3: return launch_mq_b<3>(a, stream);

@@ -1,0 +1,461 @@
+// Multi-token attention on the packed cache with the 5th-generation tensor cores (tcgen05,
+// accumulators in tensor memory), head dimension 128.
+//
+// Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
+// Compressed-Space Attention", Abstract: attention on the packed codes, full-precision K/V
+// never written to memory; the queries are rotated once, and the scores and the value sum
+// run on codebook levels in the rotated space.
+//
+// One CTA of 128 threads owns 128 (query token, head) rows of one KV head (thread r owns
+// row r) and one context chunk.  Per 64-token page:
+//   - thread 0 streams the page blocks through a 2-stage ring (1-D bulk copies, mbarrier
+//     completion, bounded waits);
+//   - the 128 threads dequantise the page's K_hat and V_hat once into f16 tiles in shared
+//     memory, written directly in the tensor core's no-swizzle operand layouts;
+//   - thread 0 issues S[128 rows x 64 tok] = Q~ . K_hat^T: the rotated queries' f16 high
+//     and low parts are two A operands in shared memory, both products go to one f32
+//     accumulator in tensor memory;
+//   - each thread reads its row's 64 scores from tensor memory and runs the lazy online
+//     softmax of its row on its own (no cross-thread reduction), then writes the weights
+//     P' = p |v| / sigma as f16 into tensor memory;
+//   - thread 0 issues O[128 rows x 128 dims] += P' . V_hat with A = P' in tensor memory and
+//     B = the V_hat tile; O stays in tensor memory for the whole chunk and is rescaled in
+//     place, row by row, on the rare tiles that raise a row's running maximum.
+// At the end each thread reads its row of O once and writes the chunk's partial result in
+// the layout of the other decode kernels, which the same combine merges.
+#include <math_constants.h>
+
+#include "isoq_common.cuh"
+#include "isoq_internal.h"
+#include "isoq_ptx.cuh"
+#include "isoq_tc.cuh"
+
+namespace isoq {
+using namespace ptx;
+namespace {
+
+constexpr int kXD = 128;    // head dimension
+constexpr int kXRows = 128; // rows per CTA = threads per CTA
+constexpr uint32_t kXCols = 256;  // tensor-memory columns: S 64 | O 128 | P' 32
+constexpr uint32_t kColS = 0, kColO = 64, kColP = 192;
+
+// Shared memory (bytes).  Operand tiles, no swizzle, core matrix = 8 rows x 16 bytes:
+//   Q~ hi / lo (A, K-major, 128 rows x 128 dims): (k/8) 2048 + (m/8) 128 + (m%8) 16 + (k%8) 2
+//   K_hat (B of the scores, K-major, 64 tok x 128 dims): (k/8) 1024 + (n/8) 128 + ...
+//   V_hat (B of the value product, MN-major: K = 64 tok, N = 128 dims):
+//         (tok/8) 2048 + (dim/8) 128 + (tok%8) 16 + (dim%8) 2
+template <int BITS>
+struct MqtcSmem {
+  static constexpr int kBB = block_bytes(kXD, BITS);
+  static constexpr int kOffQh = 0;
+  static constexpr int kOffQl = 32768;
+  static constexpr int kOffK = 65536;
+  static constexpr int kOffV = 81920;
+  static constexpr int kOffRing = 98304;                               // [2][kBB]
+  static constexpr int kOffNorm = kOffRing + (2 * kBB + 15) / 16 * 16;  // float [64 K | 64 V]
+  static constexpr int kOffBar = kOffNorm + 128 * 4;                   // ring 0, 1, S, PV
+  static constexpr int kOffTmem = kOffBar + 4 * 8;
+  static constexpr int kOffRow = kOffTmem + 16;                        // int [128]
+  static constexpr int kBytes = kOffRow + kXRows * 4;
+};
+
+__device__ __forceinline__ void st_v4(uint32_t addr, const uint32_t (&o)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(o[0]), "r"(o[1]),
+               "r"(o[2]), "r"(o[3])
+               : "memory");
+}
+
+template <typename TQ, int BITS>
+__global__ void __launch_bounds__(kXRows, 2)
+    decode_mqtc_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
+                       const int32_t* __restrict__ page_table, int n_pages, int max_pages,
+                       int H, const TQ* __restrict__ Q, int n_q_heads, int n_q,
+                       const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
+                       int n_splits, float* __restrict__ partials, uint32_t* status) {
+  using SM = MqtcSmem<BITS>;
+  constexpr int D = kXD, E = D / 32, NB = E / 4, PS = D + 4;
+  constexpr int CB = code_bytes(D, BITS), BB = block_bytes(D, BITS), W = BITS;
+  constexpr float ALPHA = alpha_of<BITS>();
+  constexpr uint32_t kIdS = tc::idesc_f16(128, 64, false, false);   // scores
+  constexpr uint32_t kIdO = tc::idesc_f16(128, 128, false, true);   // value product
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kOffBar);
+  uint64_t* bar_s = bars + 2;
+  uint64_t* bar_pv = bars + 3;
+  float* nrm = reinterpret_cast<float*>(smem + SM::kOffNorm);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffTmem);
+  int* row_off = reinterpret_cast<int*>(smem + SM::kOffRow);
+  const uint32_t sQh = smem_u32(smem + SM::kOffQh), sQl = smem_u32(smem + SM::kOffQl);
+  const uint32_t sK = smem_u32(smem + SM::kOffK), sV = smem_u32(smem + SM::kOffV);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, s = blockIdx.z;
+  const int G = n_q_heads / H;
+  const int n_rows = n_q * G;
+  const int n_groups = (n_rows + kXRows - 1) / kXRows;
+  const int hk = blockIdx.y / n_groups, rg = blockIdx.y - hk * n_groups;
+  const int row0 = rg * kXRows;
+  const int nh = min(kXRows, n_rows - row0);  // rows handled here
+
+  int len = __ldg(seq_lens + s);
+  if (len > max_pages * kPage) {
+    if (tid == 0 && split == 0 && blockIdx.y == 0) set_status(status, ISOQ_ST_LEN_RANGE);
+    len = max_pages * kPage;
+  }
+  // row r = pair R = row0 + r: query token R / G, head hk * G + R % G, which sits at
+  // position len - n_q + R / G and attends the tokens before and at it
+  {
+    const int R = row0 + tid;
+    row_off[tid] = tid < nh ? (R / G) * n_q_heads + hk * G + R % G : 0;
+  }
+  auto lim_of = [&](int r) { return max(0, min(len, len - n_q + 1 + (row0 + r) / G)); };
+  const int lim_hi = lim_of(nh - 1), lim_lo = lim_of(0);
+  const int my_lim = tid < nh ? lim_of(tid) : lim_hi;
+  const int p_begin = split * pages_per_split;
+  const int p_end = min((lim_hi + kPage - 1) / kPage, p_begin + pages_per_split);
+  float* out_base = partials + ((size_t)s * n_q * n_q_heads) * n_splits * PS + (size_t)split * PS;
+  __syncthreads();
+  if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
+    for (int i = tid; i < nh * PS; i += blockDim.x) {
+      const int r = i / PS, c = i - r * PS;
+      out_base[(size_t)row_off[r] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+    }
+    return;
+  }
+  const int n_my = p_end - p_begin;
+  const int* pt_row = page_table + (size_t)s * max_pages;
+
+  // ---- tensor memory, barriers, the first two pages ------------------------------------
+  if (warp == 0) tc::alloc(tmem_slot, kXCols);
+  auto issue = [&](int k) {  // thread 0
+    const int st = k & 1;
+    const int phys = __ldg(pt_row + p_begin + k);
+    if (phys >= 0 && phys < n_pages) {
+      mbar_expect_tx(bars + st, BB);
+      bulk_copy(smem + SM::kOffRing + st * BB, blocks + ((size_t)phys * H + hk) * BB, BB, bars + st);
+    } else {
+      set_status(status, ISOQ_ST_PAGE_RANGE);
+      mbar_arrive(bars + st);  // complete the phase without data; the page is masked
+    }
+  };
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    issue(0);
+    if (n_my > 1) issue(1);
+  }
+  int issued = min(n_my, 2);  // pages whose copy has been started (CTA-uniform count)
+
+  // ---- a6: rotate the 128 rows' queries into the A tiles (f16 high and low parts) -------
+  {
+    const float* hp = params + (size_t)hk * D * 4;
+    float M[NB][16];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, M[k]);
+    for (int r = warp; r < kXRows; r += 4) {
+      float v[E];
+      if (r < nh) {
+        const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[r]) * D + lane * E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) v[i] = 0.f;
+      }
+      wht_warp<E>(v, lane);
+      float z[E];
+#pragma unroll
+      for (int k = 0; k < NB; ++k) mat_fwd(M[k], v + 4 * k, z + 4 * k);
+      // dims 4 lane .. 4 lane + 3: half of one 16-byte core-matrix row
+      const int k0 = lane * E;
+      const uint32_t off = (k0 >> 3) * 2048 + (r >> 3) * 128 + (r & 7) * 16 + (k0 & 7) * 2;
+      float hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hi[e] = __half2float(__float2half_rn(z[e]));
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sQh + off),
+                   "r"(pack_f16x2(hi[0], hi[1])), "r"(pack_f16x2(hi[2], hi[3]))
+                   : "memory");
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sQl + off),
+                   "r"(pack_f16x2(z[0] - hi[0], z[1] - hi[1])),
+                   "r"(pack_f16x2(z[2] - hi[2], z[3] - hi[3]))
+                   : "memory");
+    }
+  }
+  tc::fence_before();
+  __syncthreads();  // barriers initialised, tensor memory allocated, query tiles written
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);  // this thread's lane
+
+  uint32_t tl0, tl1, th0, th1;
+  level_tables<BITS>(tl0, tl1, th0, th1);
+  const float kf = scale * kLog2e / (ALPHA * (float)D);  // log2 score per (dot * nK)
+
+  // this row's online-softmax state (log2 domain); sigma = its V-norm reference
+  float m2 = -CUDART_INF_F, lsum = 0.f, sigma = 0.f, inv_sigma = 0.f;
+  bool fail = false;
+  int n_s = 0, n_pv = 0;  // score / value-product commits so far (CTA-uniform)
+  int k = 0;
+  // dequantise K_hat (kv = 0) or V_hat (kv = 1) of the page in ring stage st into its tile
+  auto dequant = [&](int st, int kv) {
+    const uint8_t* blk = smem + SM::kOffRing + st * BB;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int u = tid + 128 * hf;
+      const int tk = u & 63, q = u >> 6;  // token, 32-dim group
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(
+                               blk + (kv ? v_codes_off(D, BITS) : 0) + tk * CB) + W * q;
+      uint32_t w[W];
+#pragma unroll
+      for (int i = 0; i < W; ++i) w[i] = wp[i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t o[4];
+        kdeq<BITS>(w, j, tl0, tl1, th0, th1, o);  // dims 32q + 8j .. +7 of token tk
+        const int c = 4 * q + j;
+        const uint32_t addr = kv ? sV + (tk >> 3) * 2048 + c * 128 + (tk & 7) * 16
+                                 : sK + c * 1024 + (tk >> 3) * 128 + (tk & 7) * 16;
+        st_v4(addr, o);
+      }
+    }
+  };
+
+  // Per page k: K_hat(k) -> tile; S(k) issued; V_hat(k) -> tile while S(k) runs; softmax;
+  // O += P' V_hat issued, which runs while the next page's K_hat is dequantised.
+  for (; k < n_my; ++k) {
+    // the K tile is free: S(k-1) completed before its softmax read it
+    bool ok = mbar_wait(bars + (k & 1), (k >> 1) & 1);
+    if (__syncthreads_or(!ok)) {
+      fail = true;
+      break;
+    }
+    dequant(k & 1, 0);
+    fence_proxy_async();  // the generic-proxy tile writes, before the tensor core reads
+    tc::fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc::fence_after();
+      // ---- a7: S = Q~hi . K_hat^T + Q~lo . K_hat^T, 8 k-steps of 16 dims ---------------
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t bd = tc::sdesc(sK + kk * 2048, 1024, 128);
+        tc::mma_ss(tmem + kColS, tc::sdesc(sQh + kk * 4096, 2048, 128), bd, kIdS, kk > 0);
+        tc::mma_ss(tmem + kColS, tc::sdesc(sQl + kk * 4096, 2048, 128), bd, kIdS, 1);
+      }
+      tc::commit(bar_s);
+    }
+    ++n_s;
+    // the V tile, the norms and P' are free once the previous value product has completed
+    ok = k == 0 || mbar_wait(bar_pv, (k - 1) & 1);
+    if (__syncthreads_or(!ok)) {
+      fail = true;
+      break;
+    }
+    dequant(k & 1, 1);
+    {
+      const uint8_t* blk = smem + SM::kOffRing + (k & 1) * BB;
+      if (tid < 64) nrm[tid] = half_at(blk + k_norm_off(D, BITS) + 2 * tid) * kf;
+      else nrm[tid] = half_at(blk + v_norm_off(D, BITS) + 2 * (tid - 64));
+    }
+    fence_proxy_async();
+    __syncthreads();  // norms visible; the ring stage has been read in full
+    if (tid == 0 && k + 2 < n_my) {  // the ring stage of page k takes page k + 2
+      fence_proxy_async();
+      issue(k + 2);
+    }
+    if (k + 2 < n_my) issued = k + 3;
+
+    // ---- a8: this row's online softmax over the page's 64 tokens ----------------------
+    const int pg = p_begin + k;
+    const int phys = __ldg(pt_row + pg);
+    const bool page_ok = phys >= 0 && phys < n_pages;
+    const int tok0 = pg * kPage;
+    const bool full = page_ok && tok0 + kPage <= lim_lo;
+    ok = mbar_wait(bar_s, k & 1);
+    if (__syncthreads_or(!ok)) {
+      fail = true;
+      break;
+    }
+    tc::fence_after();
+    float x[64];
+    {
+      uint32_t sr[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tc::ld32(t_row + kColS + 32 * hh, sr);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[32 * hh + j] = __uint_as_float(sr[j]);
+      }
+    }
+    float tmax = -CUDART_INF_F, vmax = 0.f;
+#pragma unroll
+    for (int j4 = 0; j4 < 64; j4 += 4) {
+      const float4 nk4 = *reinterpret_cast<const float4*>(nrm + j4);
+      const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
+      const float nk[4] = {nk4.x, nk4.y, nk4.z, nk4.w}, nv[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = j4 + e;
+        float sc = x[j] * nk[e];
+        float vv = nv[e];
+        if (!full) {
+          const bool valid = page_ok && tok0 + j < my_lim;
+          sc = valid ? sc : -CUDART_INF_F;
+          vv = valid ? vv : 0.f;
+        }
+        x[j] = sc;
+        tmax = fmaxf(tmax, sc);
+        vmax = fmaxf(vmax, vv);
+      }
+    }
+    // the running maximum and the V-norm reference move only when a score exceeds
+    // m2 + kLazy or a norm exceeds kSigmaSlack sigma; O is then rescaled in place (it is
+    // idle: the last value product completed before this page's tiles were written)
+    float resc = 1.f;
+    bool moved = false;
+    if (tmax > m2 + kLazy) {
+      resc = ex2(m2 - tmax);  // 0 when m2 was -inf
+      lsum *= resc;
+      m2 = tmax;
+      moved = true;
+    }
+    if (vmax > sigma * kSigmaSlack) {
+      resc *= sigma / vmax;  // 0 on the first valid page
+      sigma = vmax;
+      inv_sigma = 1.f / vmax;
+      moved = true;
+    }
+    // tensor-memory loads and stores are warp-collective: a warp rescales when any of its
+    // rows moved (the others with factor 1)
+    if (__any_sync(kFull, moved) && k > 0) {  // before the first product O holds nothing
+      uint32_t ov[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tc::ld32(t_row + kColO + 32 * c, ov);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * resc);
+        tc::st32(t_row + kColO + 32 * c, ov);
+      }
+    }
+    {
+      uint32_t pw[32];
+#pragma unroll
+      for (int j4 = 0; j4 < 64; j4 += 4) {
+        const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
+        const float nv[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float xs = x[j4 + e];
+          const float pe = xs != -CUDART_INF_F ? ex2(xs - m2) : 0.f;
+          lsum += pe;
+          p[e] = pe * (nv[e] * inv_sigma);  // masked tokens have p = 0
+        }
+        pw[j4 / 2] = pack_f16x2(p[0], p[1]);
+        pw[j4 / 2 + 1] = pack_f16x2(p[2], p[3]);
+      }
+      tc::st32(t_row + kColP, pw);
+    }
+    tc::wait_st();
+    tc::fence_before();
+    __syncthreads();  // P' and any rescaled O rows are in tensor memory; S has been read
+    if (tid == 0) {
+      tc::fence_after();
+      // ---- a8: O += P' . V_hat, 4 k-steps of 16 tokens ---------------------------------
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        tc::mma_ts(tmem + kColO, tmem + kColP + 8 * j, tc::sdesc(sV + j * 4096, 2048, 128), kIdO,
+                   (k > 0 || j > 0) ? 1u : 0u);
+      tc::commit(bar_pv);
+    }
+    ++n_pv;
+  }
+
+  if (fail) {
+    // a bounded wait gave up: wait (bounded) for this CTA's page copies and products still
+    // in flight, so its shared and tensor memory are idle before they are released
+    if (tid == 0) {
+      set_status(status, ISOQ_ST_TIMEOUT);
+      for (int kk = k; kk < issued; ++kk) mbar_wait(bars + (kk & 1), (kk >> 1) & 1);
+    }
+    if (n_s > 0) mbar_wait(bar_s, (n_s - 1) & 1);
+    if (n_pv > 0) mbar_wait(bar_pv, (n_pv - 1) & 1);
+  } else {
+    // ---- the chunk's partial result of this row: O sigma / ALPHA, m, l ------------------
+    const bool done = mbar_wait(bar_pv, (n_my - 1) & 1);
+    if (__syncthreads_or(!done)) {
+      if (tid == 0) set_status(status, ISOQ_ST_TIMEOUT);
+    } else {
+      tc::fence_after();
+      float* o = out_base + (size_t)row_off[tid] * n_splits * PS;
+      const float f = sigma / ALPHA;  // O holds sum p |v| ALPHA L / sigma
+      uint32_t ov[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tc::ld32(t_row + kColO + 32 * c, ov);  // warp-collective: every lane loads
+        if (tid < nh) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(o + 32 * c + j) =
+                make_float4(__uint_as_float(ov[j]) * f, __uint_as_float(ov[j + 1]) * f,
+                            __uint_as_float(ov[j + 2]) * f, __uint_as_float(ov[j + 3]) * f);
+        }
+      }
+      if (tid < nh) {
+        o[D] = m2 == -CUDART_INF_F ? -CUDART_INF_F : m2 / kLog2e;  // natural-log units
+        o[D + 1] = lsum;
+      }
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after();
+    tc::dealloc(tmem, kXCols);
+  }
+}
+
+template <typename TQ, int BITS>
+cudaError_t launch_mqtc_t(const DecodeArgs& a, cudaStream_t stream) {
+  using SM = MqtcSmem<BITS>;
+  static unsigned long long attr_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !((attr_set >> dev) & 1ull)) {
+    e = cudaFuncSetAttribute(decode_mqtc_kernel<TQ, BITS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set |= 1ull << dev;
+  }
+  const int G = a.n_q_heads / a.n_kv_heads;
+  dim3 grid(a.n_splits, a.n_kv_heads * ((a.n_q * G + kXRows - 1) / kXRows), a.n_seqs);
+  decode_mqtc_kernel<TQ, BITS><<<grid, kXRows, SM::kBytes, stream>>>(
+      a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
+      static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
+      a.n_splits, a.partials, a.status);
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_mqtc_b(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.q_dtype) {
+    case ISOQ_F32: return launch_mqtc_t<float, BITS>(a, stream);
+    case ISOQ_BF16: return launch_mqtc_t<__nv_bfloat16, BITS>(a, stream);
+    case ISOQ_F16: return launch_mqtc_t<__half, BITS>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_split_mqtc(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.bits) {
+    case 2: return launch_mqtc_b<2>(a, stream);
+    case 3: return launch_mqtc_b<3>(a, stream);
+    case 4: return launch_mqtc_b<4>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace isoq

@@ -74,6 +74,20 @@ int decode_resident_ctas(int d);
 // CTA into shared memory and shared by 64 (query token, head) rows (partials only).
 bool use_shared_mq(const DecodeArgs& a);
 cudaError_t launch_decode_split_mq(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_split_mqtc(const DecodeArgs& a, cudaStream_t stream);
+
+// Rows ((query token, head) pairs of one KV head) per CTA of the attention kernels for a
+// chunk of n_q query tokens and `group` query heads per KV head: the tensor-memory
+// multi-token kernel takes 128 rows, the shared-page mma.sync kernel 64, the per-row
+// kernel 8.  Both multi-token kernels keep 2 CTAs per SM.
+#ifndef ISOQ_MQTC_MIN_ROWS
+#define ISOQ_MQTC_MIN_ROWS 128
+#endif
+inline int attention_rows_per_cta(int d, int n_q, int group) {
+  const long long rows = (long long)n_q * group;
+  if (d != 128 || n_q <= 1 || rows < 16) return 8;
+  return rows >= ISOQ_MQTC_MIN_ROWS ? 128 : 64;
+}
 // Tensor-memory (tcgen05) split kernel, head dimension 128 (partials only).
 cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t stream);
 int decode_tc_resident_ctas();

@@ -25,6 +25,8 @@
 // the layout of the other decode kernels, which the same combine merges.
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
@@ -287,58 +289,65 @@ __global__ void __launch_bounds__(kXRows, 2)
         for (int j = 0; j < 32; ++j) x[32 * hh + j] = __uint_as_float(sr[j]);
       }
     }
-    float tmax = -CUDART_INF_F, vmax = 0.f;
+    // FULL: every token of the page is valid for every row of the CTA (no masking, and the
+    // running maximum is finite once the page's scores are in)
+    auto softmax_page = [&](auto full_c) {
+      constexpr bool FULL = decltype(full_c)::value;
+      float tm[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+      float vm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j4 = 0; j4 < 64; j4 += 4) {
-      const float4 nk4 = *reinterpret_cast<const float4*>(nrm + j4);
-      const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
-      const float nk[4] = {nk4.x, nk4.y, nk4.z, nk4.w}, nv[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
+      for (int j4 = 0; j4 < 64; j4 += 4) {
+        const float4 nk4 = *reinterpret_cast<const float4*>(nrm + j4);
+        const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
+        const float nk[4] = {nk4.x, nk4.y, nk4.z, nk4.w}, nv[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = j4 + e;
-        float sc = x[j] * nk[e];
-        float vv = nv[e];
-        if (!full) {
-          const bool valid = page_ok && tok0 + j < my_lim;
-          sc = valid ? sc : -CUDART_INF_F;
-          vv = valid ? vv : 0.f;
+        for (int e = 0; e < 4; ++e) {
+          const int j = j4 + e;
+          float sc = x[j] * nk[e];
+          float vv = nv[e];
+          if constexpr (!FULL) {
+            const bool valid = page_ok && tok0 + j < my_lim;
+            sc = valid ? sc : -CUDART_INF_F;
+            vv = valid ? vv : 0.f;
+          }
+          x[j] = sc;
+          tm[e] = fmaxf(tm[e], sc);
+          vm[e] = fmaxf(vm[e], vv);
         }
-        x[j] = sc;
-        tmax = fmaxf(tmax, sc);
-        vmax = fmaxf(vmax, vv);
       }
-    }
-    // the running maximum and the V-norm reference move only when a score exceeds
-    // m2 + kLazy or a norm exceeds kSigmaSlack sigma; O is then rescaled in place (it is
-    // idle: the last value product completed before this page's tiles were written)
-    float resc = 1.f;
-    bool moved = false;
-    if (tmax > m2 + kLazy) {
-      resc = ex2(m2 - tmax);  // 0 when m2 was -inf
-      lsum *= resc;
-      m2 = tmax;
-      moved = true;
-    }
-    if (vmax > sigma * kSigmaSlack) {
-      resc *= sigma / vmax;  // 0 on the first valid page
-      sigma = vmax;
-      inv_sigma = 1.f / vmax;
-      moved = true;
-    }
-    // tensor-memory loads and stores are warp-collective: a warp rescales when any of its
-    // rows moved (the others with factor 1)
-    if (__any_sync(kFull, moved) && k > 0) {  // before the first product O holds nothing
-      uint32_t ov[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tc::ld32(t_row + kColO + 32 * c, ov);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * resc);
-        tc::st32(t_row + kColO + 32 * c, ov);
+      const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+      const float vmax = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
+      // the running maximum and the V-norm reference move only when a score exceeds
+      // m2 + kLazy or a norm exceeds kSigmaSlack sigma; O is then rescaled in place (it is
+      // idle: the last value product completed before this page's V tile was written)
+      float resc = 1.f;
+      bool moved = false;
+      if (tmax > m2 + kLazy) {
+        resc = ex2(m2 - tmax);  // 0 when m2 was -inf
+        lsum *= resc;
+        m2 = tmax;
+        moved = true;
       }
-    }
-    {
+      if (vmax > sigma * kSigmaSlack) {
+        resc *= sigma / vmax;  // 0 on the first valid page
+        sigma = vmax;
+        inv_sigma = 1.f / vmax;
+        moved = true;
+      }
+      // tensor-memory loads and stores are warp-collective: a warp rescales when any of its
+      // rows moved (the others with factor 1)
+      if (__any_sync(kFull, moved) && k > 0) {  // before the first product O holds nothing
+        uint32_t ov[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tc::ld32(t_row + kColO + 32 * c, ov);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * resc);
+          tc::st32(t_row + kColO + 32 * c, ov);
+        }
+      }
       uint32_t pw[32];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j4 = 0; j4 < 64; j4 += 4) {
         const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
@@ -347,15 +356,19 @@ __global__ void __launch_bounds__(kXRows, 2)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float xs = x[j4 + e];
-          const float pe = xs != -CUDART_INF_F ? ex2(xs - m2) : 0.f;
-          lsum += pe;
+          float pe = ex2(xs - m2);
+          if constexpr (!FULL) pe = xs != -CUDART_INF_F ? pe : 0.f;  // m2 may still be -inf
+          ls[e] += pe;
           p[e] = pe * (nv[e] * inv_sigma);  // masked tokens have p = 0
         }
         pw[j4 / 2] = pack_f16x2(p[0], p[1]);
         pw[j4 / 2 + 1] = pack_f16x2(p[2], p[3]);
       }
+      lsum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc::st32(t_row + kColP, pw);
-    }
+    };
+    if (full) softmax_page(std::true_type{});
+    else softmax_page(std::false_type{});
     tc::wait_st();
     tc::fence_before();
     __syncthreads();  // P' and any rescaled O rows are in tensor memory; S has been read

@@ -55,7 +55,8 @@ struct MqtcSmem {
   static constexpr int kOffV = 81920;
   static constexpr int kOffRing = 98304;                               // [2][kBB]
   static constexpr int kOffNorm = kOffRing + (2 * kBB + 15) / 16 * 16;  // float [64 K | 64 V]
-  static constexpr int kOffBar = kOffNorm + 128 * 4;                   // ring 0, 1, S, PV
+  static constexpr int kOffRed = kOffNorm + 128 * 4;                   // float [4]
+  static constexpr int kOffBar = kOffRed + 16;                         // ring 0, 1, S, PV
   static constexpr int kOffTmem = kOffBar + 4 * 8;
   static constexpr int kOffRow = kOffTmem + 16;                        // int [128]
   static constexpr int kBytes = kOffRow + kXRows * 4;
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(kXRows, 2)
   uint64_t* bar_s = bars + 2;
   uint64_t* bar_pv = bars + 3;
   float* nrm = reinterpret_cast<float*>(smem + SM::kOffNorm);
+  float* red = reinterpret_cast<float*>(smem + SM::kOffRed);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kOffTmem);
   int* row_off = reinterpret_cast<int*>(smem + SM::kOffRow);
   const uint32_t sQh = smem_u32(smem + SM::kOffQh), sQl = smem_u32(smem + SM::kOffQl);
@@ -193,8 +195,9 @@ __global__ void __launch_bounds__(kXRows, 2)
   level_tables<BITS>(tl0, tl1, th0, th1);
   const float kf = scale * kLog2e / (ALPHA * (float)D);  // log2 score per (dot * nK)
 
-  // this row's online-softmax state (log2 domain); sigma = its V-norm reference
-  float m2 = -CUDART_INF_F, lsum = 0.f, sigma = 0.f, inv_sigma = 0.f;
+  // this row's online-softmax state (log2 domain)
+  float m2 = -CUDART_INF_F, lsum = 0.f;
+  float sigma = 0.f;  // the CTA's V-norm reference (the same in every thread)
   bool fail = false;
   int n_s = 0, n_pv = 0;  // score / value-product commits so far (CTA-uniform)
   int k = 0;
@@ -254,10 +257,32 @@ __global__ void __launch_bounds__(kXRows, 2)
       break;
     }
     dequant(k & 1, 1);
+    const int pg = p_begin + k;
+    const int phys = __ldg(pt_row + pg);
+    const bool page_ok = phys >= 0 && phys < n_pages;
+    const int tok0 = pg * kPage;
+    const bool full = page_ok && tok0 + kPage <= lim_lo;
+    // norms: nrm[j] = |k_j| kf; nrm[64 + j] = |v_j| / sigma', where sigma' is the CTA's
+    // V-norm reference (shared by all rows: it only scales the weights), raised when a
+    // token valid for some row has |v| > kSigmaSlack sigma; computed by warps 2 and 3
     {
       const uint8_t* blk = smem + SM::kOffRing + (k & 1) * BB;
-      if (tid < 64) nrm[tid] = half_at(blk + k_norm_off(D, BITS) + 2 * tid) * kf;
-      else nrm[tid] = half_at(blk + v_norm_off(D, BITS) + 2 * (tid - 64));
+      if (tid < 64) {
+        nrm[tid] = half_at(blk + k_norm_off(D, BITS) + 2 * tid) * kf;
+      } else {
+        const int j = tid - 64;
+        float nv = half_at(blk + v_norm_off(D, BITS) + 2 * j);
+        nv = page_ok && tok0 + j < lim_hi ? nv : 0.f;
+        float pm = nv;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, o));
+        if (lane == 0) red[warp - 2] = pm;
+        asm volatile("bar.sync 1, 64;" ::: "memory");  // warps 2 and 3 only
+        pm = fmaxf(red[0], red[1]);
+        const float sg = pm > sigma * kSigmaSlack ? pm : sigma;
+        nrm[tid] = sg > 0.f ? nv * (1.f / sg) : 0.f;
+        if (tid == 64) red[2] = sg;
+      }
     }
     fence_proxy_async();
     __syncthreads();  // norms visible; the ring stage has been read in full
@@ -266,13 +291,11 @@ __global__ void __launch_bounds__(kXRows, 2)
       issue(k + 2);
     }
     if (k + 2 < n_my) issued = k + 3;
+    const float sigma_new = red[2];
+    const float vr = sigma_new > sigma ? sigma / sigma_new : 1.f;  // 0 on the first valid page
+    sigma = sigma_new;
 
     // ---- a8: this row's online softmax over the page's 64 tokens ----------------------
-    const int pg = p_begin + k;
-    const int phys = __ldg(pt_row + pg);
-    const bool page_ok = phys >= 0 && phys < n_pages;
-    const int tok0 = pg * kPage;
-    const bool full = page_ok && tok0 + kPage <= lim_lo;
     ok = mbar_wait(bar_s, k & 1);
     if (__syncthreads_or(!ok)) {
       fail = true;
@@ -289,50 +312,58 @@ __global__ void __launch_bounds__(kXRows, 2)
         for (int j = 0; j < 32; ++j) x[32 * hh + j] = __uint_as_float(sr[j]);
       }
     }
-    // FULL: every token of the page is valid for every row of the CTA (no masking, and the
-    // running maximum is finite once the page's scores are in)
+    // FULL: every token of the page is valid for every row of the CTA (no masking).  The
+    // exponents a_j = s_j - m2 come from one FMA each; the running maximum m2 moves only
+    // when some a_j > kLazy (or on the row's first scores), and then O is rescaled in
+    // place (it is idle: the last value product completed before this page's V tile was
+    // written).
     auto softmax_page = [&](auto full_c) {
       constexpr bool FULL = decltype(full_c)::value;
-      float tm[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-      float vm[4] = {0.f, 0.f, 0.f, 0.f};
+      float resc = vr;
+      bool moved = vr != 1.f;
+      if (m2 == -CUDART_INF_F) {  // no finite score yet: exponents against this page's max
+        float tm[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-      for (int j4 = 0; j4 < 64; j4 += 4) {
-        const float4 nk4 = *reinterpret_cast<const float4*>(nrm + j4);
-        const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
-        const float nk[4] = {nk4.x, nk4.y, nk4.z, nk4.w}, nv[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = j4 + e;
-          float sc = x[j] * nk[e];
-          float vv = nv[e];
-          if constexpr (!FULL) {
-            const bool valid = page_ok && tok0 + j < my_lim;
-            sc = valid ? sc : -CUDART_INF_F;
-            vv = valid ? vv : 0.f;
-          }
+        for (int j = 0; j < 64; ++j) {
+          float sc = x[j] * nrm[j];
+          if constexpr (!FULL) sc = page_ok && tok0 + j < my_lim ? sc : -CUDART_INF_F;
           x[j] = sc;
-          tm[e] = fmaxf(tm[e], sc);
-          vm[e] = fmaxf(vm[e], vv);
+          tm[j & 3] = fmaxf(tm[j & 3], sc);
         }
-      }
-      const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
-      const float vmax = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
-      // the running maximum and the V-norm reference move only when a score exceeds
-      // m2 + kLazy or a norm exceeds kSigmaSlack sigma; O is then rescaled in place (it is
-      // idle: the last value product completed before this page's V tile was written)
-      float resc = 1.f;
-      bool moved = false;
-      if (tmax > m2 + kLazy) {
-        resc = ex2(m2 - tmax);  // 0 when m2 was -inf
-        lsum *= resc;
-        m2 = tmax;
-        moved = true;
-      }
-      if (vmax > sigma * kSigmaSlack) {
-        resc *= sigma / vmax;  // 0 on the first valid page
-        sigma = vmax;
-        inv_sigma = 1.f / vmax;
-        moved = true;
+        const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+        if (tmax != -CUDART_INF_F) {
+          m2 = tmax;
+          resc = 0.f;  // nothing accumulated yet
+          lsum = 0.f;
+          moved = true;
+        }
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[j] = x[j] - m2;  // -inf - -inf = NaN: masked below
+      } else {
+        float am[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+        for (int j4 = 0; j4 < 64; j4 += 4) {
+          const float4 nk4 = *reinterpret_cast<const float4*>(nrm + j4);
+          const float nk[4] = {nk4.x, nk4.y, nk4.z, nk4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j4 + e;
+            float a = fmaf(x[j], nk[e], -m2);
+            if constexpr (!FULL) a = page_ok && tok0 + j < my_lim ? a : -CUDART_INF_F;
+            x[j] = a;
+            am[e] = fmaxf(am[e], a);
+          }
+        }
+        const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+        if (amax > kLazy) {
+          const float r = ex2(-amax);
+          resc *= r;
+          lsum *= r;
+          m2 += amax;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) x[j] -= amax;
+          moved = true;
+        }
       }
       // tensor-memory loads and stores are warp-collective: a warp rescales when any of its
       // rows moved (the others with factor 1)
@@ -355,11 +386,11 @@ __global__ void __launch_bounds__(kXRows, 2)
         float p[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float xs = x[j4 + e];
-          float pe = ex2(xs - m2);
-          if constexpr (!FULL) pe = xs != -CUDART_INF_F ? pe : 0.f;  // m2 may still be -inf
+          const float a = x[j4 + e];
+          float pe = ex2(a);  // a = -inf: 0
+          if constexpr (!FULL) pe = a == a ? pe : 0.f;  // NaN from a row with no score yet
           ls[e] += pe;
-          p[e] = pe * (nv[e] * inv_sigma);  // masked tokens have p = 0
+          p[e] = pe * nv[e];  // |v| / sigma'; masked tokens have p = 0
         }
         pw[j4 / 2] = pack_f16x2(p[0], p[1]);
         pw[j4 / 2 + 1] = pack_f16x2(p[2], p[3]);

@@ -95,6 +95,9 @@ struct SplitPlan {
 #ifndef ISOQ_DEC_WAVES
 #define ISOQ_DEC_WAVES 4
 #endif
+#ifndef ISOQ_MQ_WAVES  // the same for the multi-token kernels
+#define ISOQ_MQ_WAVES 8
+#endif
 
 // Context chunking for the decode kernel: about ISOQ_DEC_WAVES waves of (chunk, KV head,
 // query-head block, sequence) CTAs at the kernel's resident CTAs per SM, each chunk a whole
@@ -113,7 +116,7 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
   const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group) : 8;
   const long long units =
       (long long)n_seqs * n_kv_heads * (((long long)n_q * group + rows_per_cta - 1) / rows_per_cta);
-  const long long target = (long long)n_sm * ISOQ_DEC_WAVES;
+  const long long target = (long long)n_sm * (shared_mq ? ISOQ_MQ_WAVES : ISOQ_DEC_WAVES);
   long long want = units > 0 ? (target + units - 1) / units : 1;
   const long long cap = (max_pages + min_pages - 1) / min_pages;
   if (want > cap) want = cap;

@@ -111,9 +111,10 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
   const bool tc = !shared_mq && n_q == 1 && isoq::kUseTc128 && d == 128;
   const int n_sm = sm_count() * (shared_mq ? 2 : tc ? isoq::decode_tc_resident_ctas()
                                                     : isoq::decode_resident_ctas(d));
-  const int min_pages = shared_mq ? 4 : tc ? 8 : 16;  // pages per CTA worth a launch
-  const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group) : 8;
+  // pages per CTA worth a launch: the tensor-memory kernel rotates 128 queries per CTA
+  const int min_pages = shared_mq ? (rows_per_cta == 128 ? 16 : 4) : tc ? 8 : 16;
+  const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const long long units =
       (long long)n_seqs * n_kv_heads * (((long long)n_q * group + rows_per_cta - 1) / rows_per_cta);
   const long long target = (long long)n_sm * (shared_mq ? ISOQ_MQ_WAVES : ISOQ_DEC_WAVES);

@@ -207,7 +207,10 @@ __global__ void __launch_bounds__(kXRows, 2)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int u = tid + 128 * hf;
-      const int tk = u & 63, q = u >> 6;  // token, 32-dim group
+      // token, 32-dim group: a warp takes 8 tokens x 4 groups, so its 32-bit code loads
+      // (word 12 tk + 3 q + i) hit 32 distinct banks and each quarter-warp's 16-byte tile
+      // stores 8 distinct bank groups (tk % 8)
+      const int tk = 8 * (u >> 5) + (u & 7), q = (u >> 3) & 3;
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(
                                blk + (kv ? v_codes_off(D, BITS) : 0) + tk * CB) + W * q;
       uint32_t w[W];

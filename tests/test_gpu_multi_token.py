@@ -142,3 +142,55 @@ def test_multi_token_rejects_bad_arguments(run2):
     assert lib.isoq_multi_token_attention(*args(2, need - 16)) == iq.ISOQ_E_WORKSPACE
     assert lib.isoq_multi_token_attention(*args(2, need)) == iq.ISOQ_OK
     torch.cuda.synchronize()
+
+
+# The tensor-memory kernel takes KV heads with >= 128 (query token, head) rows.  These cases
+# reach it with ragged batches (a sequence shorter than the chunk), a partial second row
+# group, fp32 queries, the 2- and 4-bit formats and a context of several chunks.
+@pytest.mark.parametrize("case", ["ragged_G4_nq32", "rows160", "fp32_G4_nq64", "long_20k"])
+def test_multi_token_tensor_memory_kernel(oracle, case):
+    from dataclasses import replace
+    if case == "ragged_G4_nq32":
+        cfg = wl.small_variant(wl.workload(4), n_seqs=3, len_range=(40, 1500))
+        n_q = 32
+    elif case == "rows160":
+        cfg = wl.small_variant(wl.workload(2), length=900)
+        n_q = 20
+    elif case == "fp32_G4_nq64":
+        cfg = wl.workload(1)
+        n_q = 64
+    else:
+        cfg = wl.small_variant(wl.workload(2), length=20000)
+        n_q = 16
+    assert n_q * cfg.n_q_heads // cfg.n_kv_heads >= 128
+    run = Run(cfg)
+    run.prefill()
+    Q = wl.query_chunk(cfg, n_q, device="cuda")
+    lens = list(cfg.decode_lens())
+    if case == "ragged_G4_nq32":
+        lens[0] = 10  # shorter than the chunk: its first 22 query tokens attend nothing
+    out = _multi(run, Q, lens)
+    stats = _compare(_oracle_multi(oracle, run, Q, lens), out)
+    if case == "ragged_G4_nq32":
+        assert torch.all(out[0, :22] == 0)
+    assert iq.isoq_get_status(run.cache) == 0
+    log_record({"case": f"multi_tc_{case}", **stats})
+
+
+@pytest.mark.parametrize("bits,rot", [(2, 0), (4, 1)])
+def test_multi_token_tensor_memory_kernel_formats(oracle, bits, rot):
+    cfg = wl.small_variant(wl.workload(2), length=1100)
+    run = Run(cfg, bits=bits, rot=rot)
+    run.prefill()
+    n_q = 16
+    Q = wl.query_chunk(cfg, n_q, device="cuda")
+    L = cfg.decode_lens()[0]
+    out = _multi(run, Q, [L])
+    pt = run.layout.page_table.numpy()
+    ref = oracle.decode_attention(run.params64(), cfg.d, cfg.n_kv_heads, 64,
+                                  run.cache.blocks.cpu().numpy(), np.repeat(pt[:1], n_q, 0),
+                                  [L - n_q + i + 1 for i in range(n_q)],
+                                  Q[0].float().cpu().numpy().astype(np.float64), cfg.scale,
+                                  bits=bits, rot=rot)
+    stats = _compare(ref[None], out)
+    log_record({"case": f"multi_tc_b{bits}_r{rot}", **stats})

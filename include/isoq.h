@@ -385,6 +385,17 @@ int isoq_reset_status(const isoq_cache* cache, void* stream);
 /* The cudaError_t of the last failing CUDA call in this thread (0 if none). */
 int isoq_last_cuda_error(void);
 
+/* ---- self-test of the bounded waits ------------------------------------------------------
+ * Every wait in the kernels' copy and tensor-core pipelines (on an mbarrier phase) gives up
+ * after a bounded number of polls, reports ISOQ_ST_TIMEOUT in the status word and lets the
+ * kernel finish, so a copy that never lands cannot hang the GPU.  This call exercises that
+ * path with the same wait helper: one kernel of one thread waits `polls` polls on a phase
+ * that nothing completes, sets ISOQ_ST_TIMEOUT in *status (device word) when the wait gives
+ * up, then waits on a phase it has completed itself.  result: device uint32[2] = (the stuck
+ * wait gave up, the completed wait succeeded), 1 for yes.  Asynchronous on `stream`.
+ * Errors: ISOQ_E_ARG (null pointer, polls = 0), ISOQ_E_CUDA. */
+int isoq_selftest_bounded_wait(uint32_t* status, unsigned polls, uint32_t* result, void* stream);
+
 /* A static string describing an ISOQ_* return code. */
 const char* isoq_error_string(int code);
 

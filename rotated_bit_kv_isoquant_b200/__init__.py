@@ -5,7 +5,7 @@ Argument marshalling only: every step of the path runs in the library's CUDA ker
 PyTorch supplies device memory and streams.  The functions carry the C names of
 ``include/isoq.h`` and raise :class:`IsoqError` on a negative return code.  Importing
 this package fails loudly if ``libisoq.so`` has not been built
-(``python -m rotated_bit_kv_isoquant_b200.build``); there is no fallback.
+(``python rotated_bit_kv_isoquant_b200/build.py``); there is no fallback.
 """
 from __future__ import annotations
 
@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libisoq.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libisoq.so is missing at {LIB_PATH}: build it with "
-        "`python -m rotated_bit_kv_isoquant_b200.build` (nvcc, sm_100a). "
+        "`python rotated_bit_kv_isoquant_b200/build.py` (nvcc, sm_100a). "
         "There is no CPU fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -38,6 +38,7 @@ ISOQ_ST_POS_RANGE = 0x2
 ISOQ_ST_PAGE_RANGE = 0x4
 ISOQ_ST_NORM_SAT = 0x8
 ISOQ_ST_LEN_RANGE = 0x10
+ISOQ_ST_TIMEOUT = 0x20
 
 ISOQ_F32, ISOQ_BF16, ISOQ_F16 = 0, 1, 2
 ISOQ_ROT_SO4, ISOQ_ROT_SO2 = 0, 1
@@ -93,6 +94,7 @@ _SIGS = {
     "isoq_get_status": (_i, [_cp, ctypes.POINTER(ctypes.c_uint32)]),
     "isoq_reset_status": (_i, [_cp, _p]),
     "isoq_last_cuda_error": (_i, []),
+    "isoq_selftest_bounded_wait": (_i, [_p, ctypes.c_uint, _p, _p]),
     "isoq_error_string": (ctypes.c_char_p, [_i]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -396,6 +398,19 @@ def isoq_reset_status(cache: PagedCache, stream=None) -> None:
 
 def isoq_last_cuda_error() -> int:
     return int(_lib.isoq_last_cuda_error())
+
+
+def isoq_selftest_bounded_wait(polls: int = 4096, stream=None):
+    """Runs the bounded-wait self-test; returns (status word, stuck wait gave up, completed
+    wait succeeded)."""
+    import torch
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    result = torch.zeros((2,), dtype=torch.int32, device="cuda")
+    _check(_lib.isoq_selftest_bounded_wait(status.data_ptr(), polls, result.data_ptr(),
+                                           _stream_ptr(stream)), "isoq_selftest_bounded_wait")
+    torch.cuda.synchronize()
+    r = result.cpu().tolist()
+    return int(status.item()) & 0xffffffff, bool(r[0]), bool(r[1])
 
 
 def isoq_error_string(code: int) -> str:

@@ -1,6 +1,8 @@
 """Builds libisoq.so in-tree with nvcc for sm_100a (B200).
 
-    python -m rotated_bit_kv_isoquant_b200.build [--force]
+    python rotated_bit_kv_isoquant_b200/build.py [--force]
+
+(run as a script: importing the package itself needs the library)
 
 Each .cu under csrc/ compiles to an object in parallel, then the objects link into
 rotated_bit_kv_isoquant_b200/libisoq.so.  Needs only nvcc (no GPU).

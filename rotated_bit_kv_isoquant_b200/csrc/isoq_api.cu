@@ -95,6 +95,9 @@ struct SplitPlan {
 #ifndef ISOQ_DEC_WAVES
 #define ISOQ_DEC_WAVES 4
 #endif
+#ifndef ISOQ_DEC_MIN_PAGES  // pages per decode CTA worth a launch
+#define ISOQ_DEC_MIN_PAGES 16
+#endif
 #ifndef ISOQ_MQ_WAVES  // the same for the multi-token kernels
 #define ISOQ_MQ_WAVES 8
 #endif
@@ -113,7 +116,7 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
                                                     : isoq::decode_resident_ctas(d));
   const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group) : 8;
   // pages per CTA worth a launch: the tensor-memory kernel rotates 128 queries per CTA
-  const int min_pages = shared_mq ? (rows_per_cta == 128 ? 16 : 4) : tc ? 8 : 16;
+  const int min_pages = shared_mq ? (rows_per_cta == 128 ? 16 : 4) : tc ? 8 : ISOQ_DEC_MIN_PAGES;
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const long long units =
       (long long)n_seqs * n_kv_heads * (((long long)n_q * group + rows_per_cta - 1) / rows_per_cta);

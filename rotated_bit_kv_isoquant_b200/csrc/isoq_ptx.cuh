@@ -64,10 +64,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Polls the phase with the given parity; false if it did not complete within the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+// Polls the phase with the given parity; false if it did not complete within `limit` polls
+// (the kernels use kWaitLimit; a self-test uses a short limit to exercise the give-up path).
+__device__ __forceinline__ bool mbar_wait_n(uint64_t* bar, unsigned parity, unsigned limit) {
   const uint32_t a = smem_u32(bar);
-  for (unsigned i = 0; i < kWaitLimit; ++i) {
+  for (unsigned i = 0; i < limit; ++i) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
@@ -78,6 +79,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
     if (done) return true;
   }
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  return mbar_wait_n(bar, parity, kWaitLimit);
 }
 
 __device__ __forceinline__ void bulk_copy(void* dst, const void* src, unsigned bytes,

@@ -15,11 +15,11 @@ __global__ void bounded_wait_selftest_kernel(uint32_t* status, unsigned polls, u
   ptx::mbar_init(bars, 1);      // never arrived at
   ptx::mbar_init(bars + 1, 1);  // arrived at once below
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  const bool stuck = ptx::mbar_wait_n(bars, 0, polls);
+  const bool gave_up = !ptx::mbar_wait_n(bars, 0, polls);  // false: the phase never completes
   ptx::mbar_arrive(bars + 1);
   const bool done = ptx::mbar_wait_n(bars + 1, 0, polls);
-  if (!stuck) set_status(status, ISOQ_ST_TIMEOUT);
-  result[0] = stuck ? 1u : 0u;
+  if (gave_up) set_status(status, ISOQ_ST_TIMEOUT);  // as a kernel reports a lost page copy
+  result[0] = gave_up ? 1u : 0u;
   result[1] = done ? 1u : 0u;
 }
 

@@ -194,3 +194,29 @@ def test_multi_token_tensor_memory_kernel_formats(oracle, bits, rot):
                                   bits=bits, rot=rot)
     stats = _compare(ref[None], out)
     log_record({"case": f"multi_tc_b{bits}_r{rot}", **stats})
+
+
+@pytest.mark.parametrize("n_q", [1, 4, 16])
+def test_bad_last_page_is_masked_and_reported(oracle, n_q):
+    """A page-table entry outside [0, n_pages) on the last page of a sequence: every kernel
+    (per-row decode, shared-page and tensor-memory multi-token) skips the page's tokens and
+    sets ISOQ_ST_PAGE_RANGE, so each row equals the oracle over the tokens before that page."""
+    cfg = wl.small_variant(wl.workload(2), length=1000)
+    run = Run(cfg)
+    run.prefill()
+    L = cfg.decode_lens()[0]
+    last = (L - 1) // 64
+    good = last * 64  # tokens before the bad page
+    run.cache.page_table[0, last] = -1
+    iq.isoq_reset_status(run.cache)
+    Q = wl.query_chunk(cfg, n_q, device="cuda")
+    out = _multi(run, Q, [L])
+    assert iq.isoq_get_status(run.cache) == iq.ISOQ_ST_PAGE_RANGE
+    pt = run.layout.page_table.numpy()
+    lens_i = [min(L - n_q + i + 1, good) for i in range(n_q)]
+    ref = oracle.decode_attention(run.params64(), cfg.d, cfg.n_kv_heads, 64,
+                                  run.cache.blocks.cpu().numpy(), np.repeat(pt[:1], n_q, 0),
+                                  lens_i, Q[0].float().cpu().numpy().astype(np.float64),
+                                  cfg.scale)
+    stats = _compare(ref[None], out)
+    log_record({"case": f"multi_bad_last_page_nq{n_q}", **stats})

@@ -231,16 +231,16 @@ __global__ void __launch_bounds__(kXRows, 2)
   // Per page k: K_hat(k) -> tile; S(k) issued; V_hat(k) -> tile while S(k) runs; softmax;
   // O += P' V_hat issued, which runs while the next page's K_hat is dequantised.
   for (; k < n_my; ++k) {
-    // the K tile is free: S(k-1) completed before its softmax read it
+    // Three CTA barriers per page; every other hand-off is a thread's own mbarrier wait.
+    // The K tile is free: S(k-1) completed before this thread's softmax read it.
     bool ok = mbar_wait(bars + (k & 1), (k >> 1) & 1);
+    if (ok) dequant(k & 1, 0);
+    fence_proxy_async();  // the generic-proxy tile writes, before the tensor core reads
+    tc::fence_before();
     if (__syncthreads_or(!ok)) {
       fail = true;
       break;
     }
-    dequant(k & 1, 0);
-    fence_proxy_async();  // the generic-proxy tile writes, before the tensor core reads
-    tc::fence_before();
-    __syncthreads();
     if (tid == 0) {
       tc::fence_after();
       // ---- a7: S = Q~hi . K_hat^T + Q~lo . K_hat^T, 8 k-steps of 16 dims ---------------
@@ -253,13 +253,10 @@ __global__ void __launch_bounds__(kXRows, 2)
       tc::commit(bar_s);
     }
     ++n_s;
-    // the V tile, the norms and P' are free once the previous value product has completed
+    // the V tile, P' and O are free once the previous value product has completed (this
+    // thread's own wait); the norms of page k-1 were read before the last barrier
     ok = k == 0 || mbar_wait(bar_pv, (k - 1) & 1);
-    if (__syncthreads_or(!ok)) {
-      fail = true;
-      break;
-    }
-    dequant(k & 1, 1);
+    if (ok) dequant(k & 1, 1);
     const int pg = p_begin + k;
     const int phys = __ldg(pt_row + pg);
     const bool page_ok = phys >= 0 && phys < n_pages;
@@ -288,7 +285,10 @@ __global__ void __launch_bounds__(kXRows, 2)
       }
     }
     fence_proxy_async();
-    __syncthreads();  // norms visible; the ring stage has been read in full
+    if (__syncthreads_or(!ok)) {  // norms visible; the ring stage has been read in full
+      fail = true;
+      break;
+    }
     if (tid == 0 && k + 2 < n_my) {  // the ring stage of page k takes page k + 2
       fence_proxy_async();
       issue(k + 2);
@@ -299,11 +299,8 @@ __global__ void __launch_bounds__(kXRows, 2)
     sigma = sigma_new;
 
     // ---- a8: this row's online softmax over the page's 64 tokens ----------------------
-    ok = mbar_wait(bar_s, k & 1);
-    if (__syncthreads_or(!ok)) {
-      fail = true;
-      break;
-    }
+    ok = __all_sync(kFull, mbar_wait(bar_s, k & 1));  // warp-uniform: collectives below
+    if (ok) {
     tc::fence_after();
     float x[64];
     {
@@ -403,9 +400,13 @@ __global__ void __launch_bounds__(kXRows, 2)
     };
     if (full) softmax_page(std::true_type{});
     else softmax_page(std::false_type{});
+    }
     tc::wait_st();
     tc::fence_before();
-    __syncthreads();  // P' and any rescaled O rows are in tensor memory; S has been read
+    if (__syncthreads_or(!ok)) {  // P' and any rescaled O rows are in TMEM; S has been read
+      fail = true;
+      break;
+    }
     if (tid == 0) {
       tc::fence_after();
       // ---- a8: O += P' . V_hat, 4 k-steps of 16 tokens ---------------------------------

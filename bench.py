@@ -105,7 +105,8 @@ def _tensor_peak():
 
 _KERNEL_SOURCES = {
     "decode": ["isoq_decode_mma.cu", "isoq_decode.cu", "isoq_ptx.cuh", "isoq_common.cuh"],
-    "quantize": ["isoq_quantize.cu", "isoq_common.cuh"],
+    "quantize": ["isoq_quantize_tc.cu", "isoq_quantize.cu", "isoq_codes.cuh", "isoq_tc.cuh",
+                 "isoq_common.cuh"],
 }
 
 

@@ -61,6 +61,9 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
+// d = 128, 3 bits, bf16 / f16 inputs without RoPE: the WHT as a tensor-core product.
+bool use_quantize_tc(const QuantizeArgs& a);
+cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Merge of context-slice states [n_states][n_seqs][n_q_heads][d + 4] into the output.
 cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int n_seqs,

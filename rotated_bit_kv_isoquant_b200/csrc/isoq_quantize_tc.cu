@@ -1,0 +1,380 @@
+// Quantize-append for d = 128, 3-bit codes, bf16 / f16 inputs, with the Walsh-Hadamard
+// transform on the 5th-generation tensor cores.
+//
+// Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
+// Compressed-Space Attention", Abstract: each K/V vector goes through a Walsh-Hadamard
+// transform, then block-diagonal SO(4) rotations, then a 3-bit scalar quantiser.
+//
+// The unnormalised WHT in natural (Sylvester) order is the symmetric matrix
+// H[k][n] = (-1)^popc(k & n).  Its entries are exact in bf16 and f16, and so are the
+// inputs, so the transform of a tile of 128 vectors (128 consecutive tokens of one KV head,
+// K or V) is one 128 x 128 x 128 UMMA (kind::f16, f32 accumulator in tensor memory) with
+// exact products.  The rest runs on the CUDA cores over the accumulator rows: thread pair
+// (r, r + 128) owns vector r, each thread one half of its dims; the pair adds its halves'
+// sums of squares for the norm (|H x|^2 = 128 |x|^2), then each thread applies the head's
+// 4x4 block matrices, decides the codes against the norm-scaled thresholds, packs its two
+// 32-dim groups (24 bytes) and stores them into the paged cache.
+//
+// Pipeline of a CTA over its tiles j: the copies of tile j+2 (cp.async of the 128 rows
+// into the operand layout, and the head's block matrices) and the UMMA of tile j+1 run
+// while the threads work on tile j's accumulator; two accumulators alternate in tensor
+// memory (256 columns) and two operand stages in shared memory.  Every mbarrier wait is
+// bounded; a wait that gives up reports ISOQ_ST_TIMEOUT and the CTA stops after draining
+// what it issued.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include <type_traits>
+
+#include "isoq_codes.cuh"
+#include "isoq_common.cuh"
+#include "isoq_internal.h"
+#include "isoq_ptx.cuh"
+#include "isoq_tc.cuh"
+
+namespace isoq {
+namespace {
+using namespace ptx;
+
+constexpr int kQtD = 128;
+constexpr int kQtRows = 128;                      // vectors per tile = UMMA M
+constexpr int kQtThreads = 256;                   // two threads per vector
+constexpr int kQtTile = kQtRows * kQtD * 2;       // one 16-bit operand tile, 32 KiB
+constexpr int kQtMat = 32 * 16 * 4;               // one head's block matrices, 2 KiB
+constexpr int kOffX = 0;                          // [2] input tiles
+constexpr int kOffH = 2 * kQtTile;                // the Hadamard operand
+constexpr int kOffM = kOffH + kQtTile;            // [3] block-matrix stages
+constexpr int kOffRed = kOffM + 3 * kQtMat;       // [2][128] half sums of squares
+constexpr int kOffBar = kOffRed + 2 * kQtRows * 4;  // 2 mbarriers (UMMA completion)
+constexpr int kOffSlot = kOffBar + 16;            // tensor-memory base address
+constexpr int kQtSmem = kOffSlot + 16;
+constexpr uint32_t kQtCols = 256;                 // two 128-column f32 accumulators
+
+// Byte offset of element (row, k) of a K-major no-swizzle operand tile: core matrices of
+// 8 rows x 16 bytes, 128 bytes apart along k (the descriptor's leading offset) and 2048
+// bytes apart along the rows (its stride offset).
+__host__ __device__ constexpr uint32_t qt_off(int row, int k) {
+  return (uint32_t)((row >> 3) * 2048 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kQtThreads, 2)
+    quantize_tc_kernel(const __grid_constant__ QuantLayers layers, int H, int n_tokens,
+                       const int32_t* __restrict__ seq_ids,
+                       const int32_t* __restrict__ positions) {
+  constexpr int BITS = 3, D = kQtD, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr uint32_t kIdesc = tc::idesc_f16(128, 128, false, false, kBf16);
+  const QuantLayer& L = layers.l[blockIdx.y];  // this launch row's layer
+  const float* __restrict__ mats = L.mats;
+  uint8_t* __restrict__ blocks = L.blocks;
+  const int32_t* __restrict__ page_table = L.page_table;
+  const int n_pages = L.n_pages, max_pages = L.max_pages, n_seqs = L.n_seqs;
+  const uint8_t* __restrict__ Kb = static_cast<const uint8_t*>(L.K);
+  const uint8_t* __restrict__ Vb = static_cast<const uint8_t*>(L.V);
+  uint32_t* status = L.status;
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  float* red = reinterpret_cast<float*>(smem + kOffRed);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffSlot);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, hf = warp >> 2;  // tensor-memory lane quarter, half of the dims
+  const int r = quad * 32 + lane;             // this thread's vector (row) of the tile
+  const int n_chunks = (n_tokens + kQtRows - 1) / kQtRows;
+  const int n_kinds = 2 * H;             // (head, K|V) pairs: rr = 2 head + kind
+  const int n_tiles = n_chunks * n_kinds;  // tile = (128-token chunk, head, K|V), chunk-major
+  const int first = blockIdx.x, stride = gridDim.x;
+  if (first >= n_tiles) return;
+  // this CTA's tiles first, first + stride, ... as (chunk, rr), advanced without division
+  struct Tile {
+    int chunk, rr;
+  };
+  const int step_c = stride / n_kinds, step_r = stride - step_c * n_kinds;
+  auto advance = [&](Tile t) {
+    t.chunk += step_c;
+    t.rr += step_r;
+    if (t.rr >= n_kinds) {
+      t.rr -= n_kinds;
+      ++t.chunk;
+    }
+    return t;
+  };
+  Tile cur{first / n_kinds, first % n_kinds};  // tiles li, li + 1, li + 2
+  Tile nxt = advance(cur), nn = advance(nxt);
+
+  // copies of tile t (local index li) into input stage li & 1 and matrix stage li % 3; a
+  // warp's copy covers 8 rows x 64 bytes, 512 contiguous bytes of the tile.  Rows past the
+  // last token are not copied (their accumulator rows are never used).
+  const int cp_row = 8 * (tid >> 7) + (tid & 7), cp_j = (tid >> 3) & 15;  // + 16 c
+  const uint32_t cp_dst = qt_off(cp_row, 8 * cp_j);
+  const size_t row_bytes = (size_t)H * D * sizeof(T);
+  auto prefetch = [&](Tile t, int li) {
+    if (t.chunk < n_chunks) {
+      const int h = t.rr >> 1;
+      const int t0 = t.chunk * kQtRows;
+      const uint8_t* src = ((t.rr & 1) ? Vb : Kb) + (size_t)(t0 + cp_row) * row_bytes +
+                           (size_t)h * D * sizeof(T) + 16 * cp_j;
+      const uint32_t xs = sbase + kOffX + (li & 1) * kQtTile + cp_dst;
+      const int rows_left = n_tokens - t0 - cp_row;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (16 * c < rows_left) cp_async16(xs + 4096 * c, src + 16 * c * row_bytes);
+      if (tid < kQtMat / 16)
+        cp_async16(sbase + kOffM + (li % 3) * kQtMat + 16 * tid,
+                   reinterpret_cast<const uint8_t*>(mats) + (size_t)h * kQtMat + 16 * tid);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  prefetch(cur, 0);
+  prefetch(nxt, 1);
+
+  // the Hadamard operand (N x K, K-major; symmetric): thread -> row tid / 2, 64 dims
+  {
+    const uint32_t one = kBf16 ? 0x3F80u : 0x3C00u;
+    const int n = tid >> 1;
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) {
+      const int k0 = 64 * (tid & 1) + 8 * kc;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = one | ((__popc(n & (k0 + 2 * e)) & 1u) << 15);
+        const uint32_t hi = one | ((__popc(n & (k0 + 2 * e + 1)) & 1u) << 15);
+        w[e] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(smem + kOffH + qt_off(n, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (tid == 0) {
+    mbar_init(bars + 0, 1);
+    mbar_init(bars + 1, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tc::alloc(tmem_slot, kQtCols);
+
+  auto issue_mma = [&](int li) {  // thread 0: the tile's transform into accumulator li & 1
+    const uint32_t xs = sbase + kOffX + (li & 1) * kQtTile, hs = sbase + kOffH;
+    const uint32_t d = *tmem_slot + (uint32_t)(li & 1) * 128;
+#pragma unroll
+    for (int s = 0; s < D / 16; ++s)
+      tc::mma_ss(d, tc::sdesc(xs + 256 * s, 128, 2048), tc::sdesc(hs + 256 * s, 128, 2048), kIdesc,
+                 s > 0);
+    tc::commit(bars + (li & 1));
+  };
+
+  // sequence, position and page entry of this thread's token, loaded one tile ahead of use
+  int sid = -1, pos = -1, phys = -1;
+  auto load_page = [&](int t) {  // validates (sid, pos) of token t; page entry or -1
+    phys = -1;
+    if (t >= n_tokens) return;
+    if (sid < 0 || sid >= n_seqs) {
+      if (hf == 0) set_status(status, ISOQ_ST_SEQ_RANGE);
+    } else if (pos < 0 || (pos >> 6) >= max_pages) {
+      if (hf == 0) set_status(status, ISOQ_ST_POS_RANGE);
+    } else {
+      phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
+      if (phys < 0 || phys >= n_pages) {
+        if (hf == 0) set_status(status, ISOQ_ST_PAGE_RANGE);
+        phys = -1;
+      }
+    }
+  };
+  {
+    const int t = cur.chunk * kQtRows + r;
+    if (t < n_tokens) {
+      sid = __ldg(seq_ids + t);
+      pos = __ldg(positions + t);
+    }
+    load_page(t);
+  }
+
+  // tile 0's copies, the Hadamard operand and the barriers are visible; first transform
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+  fence_proxy_async();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16);  // this thread's lane
+  if (tid == 0) issue_mma(0);
+
+  bool failed = false, ok = true;  // ok: the last wait for a transform completed
+  int li = 0;
+  for (;; ++li) {
+    if (cur.chunk >= n_chunks) break;
+    const bool has_next = nxt.chunk < n_chunks;
+    // tile li+1's copies landed, tile li-1's accumulator reads are done: transform li+1
+    // (unless a wait gave up anywhere in the CTA)
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    fence_proxy_async();
+    tc::fence_before();
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    if (tid == 0 && has_next) {
+      tc::fence_after();
+      issue_mma(li + 1);
+    }
+    int nsid = -1, npos = -1;
+    if (has_next) {
+      const int tn = nxt.chunk * kQtRows + r;
+      if (tn < n_tokens) {
+        nsid = __ldg(seq_ids + tn);
+        npos = __ldg(positions + tn);
+      }
+    }
+    ok = mbar_wait(bars + (li & 1), (li >> 1) & 1);  // transform li done
+    tc::fence_after();
+    prefetch(nn, li + 2);  // input stage li & 1 is free again
+
+    const int h = cur.rr >> 1, kind = cur.rr & 1;
+    const uint32_t acc = t_row + (uint32_t)(li & 1) * 128 + 64 * hf;  // this thread's 64 dims
+
+    // a1: norm from the transform, |x|^2 = |H x|^2 / 128.  The pair's halves meet in
+    // shared memory behind a barrier of its two warps and are added in a fixed order, so
+    // both threads hold the same value.
+    uint32_t y[64];
+    tc::ld64(acc, y);
+    {
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 64; e += 4) {
+        const float a = __uint_as_float(y[e]), b = __uint_as_float(y[e + 1]);
+        const float cc = __uint_as_float(y[e + 2]), dd = __uint_as_float(y[e + 3]);
+        s0 = fmaf(a, a, s0);
+        s1 = fmaf(b, b, s1);
+        s2 = fmaf(cc, cc, s2);
+        s3 = fmaf(dd, dd, s3);
+      }
+      red[hf * kQtRows + r] = (s0 + s1) + (s2 + s3);
+    }
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");  // warps quad, quad + 4
+    const float n = sqrtf((red[r] + red[kQtRows + r]) * (1.0f / 128.0f));
+
+    // a3 + a4: block matrices and codes of this thread's two 32-dim groups
+    float TB[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      TB[k] = n == 0.f ? CUDART_INF_F : n * pos_threshold_f32(BITS, k) * 0x1p64f;
+    const float4* mh = reinterpret_cast<const float4*>(smem + kOffM + (li % 3) * kQtMat);
+    uint32_t rec[6];
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g = 2 * hf + gg;  // group of the vector
+      uint32_t half[8];
+#pragma unroll
+      for (int bi = 0; bi < 8; ++bi) {
+        const int b = 8 * g + bi;  // block of the vector
+        float W = code_base<BITS>() * 4369.0f;  // sum coef * base over the 4 codes
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 m = mh[4 * b + e];
+          // the chain starts from +0, so z is never -0 (which would code as negative)
+          const uint32_t* yb = y + 32 * gg + 4 * bi;
+          const float z = fmaf(m.w, __uint_as_float(yb[3]),
+                               fmaf(m.z, __uint_as_float(yb[2]),
+                                    fmaf(m.y, __uint_as_float(yb[1]),
+                                         fmaf(m.x, __uint_as_float(yb[0]), 0.0f))));
+          W = add_code<BITS>(W, z, (float)(1 << (4 * e)), TB);
+        }
+        half[bi] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W
+      }
+      uint32_t nib[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[2 * j], half[2 * j + 1]);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
+    }
+
+    if (phys >= 0) {
+      uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
+      const int slot = pos & (kPage - 1);
+      uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB;
+      if (hf == 0) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(rec[0], rec[1], rec[2], rec[3]);
+        *reinterpret_cast<uint2*>(dst + 16) = make_uint2(rec[4], rec[5]);
+        uint16_t nb = __half_as_ushort(__float2half_rn(n));
+        if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
+          nb = 0x7bffu;
+          set_status(status, ISOQ_ST_NORM_SAT);
+        }
+        *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
+                                     2 * slot) = nb;
+      } else {
+        *reinterpret_cast<uint2*>(dst + 24) = make_uint2(rec[0], rec[1]);
+        *reinterpret_cast<uint4*>(dst + 32) = make_uint4(rec[2], rec[3], rec[4], rec[5]);
+      }
+    }
+    if (has_next) {
+      sid = nsid;
+      pos = npos;
+      load_page(nxt.chunk * kQtRows + r);
+    }
+    cur = nxt;
+    nxt = nn;
+    nn = advance(nn);
+  }
+
+  // a wait that gave up (anywhere in the CTA; the loop's end has the last one): report it
+  // and wait (bounded) for the last transform issued before the tensor memory is released
+  if (failed || __syncthreads_or(!ok)) {
+    if (tid == 0) set_status(status, ISOQ_ST_TIMEOUT);
+    const int last = failed ? li : li - 1;
+    if (last >= 0) mbar_wait(bars + (last & 1), (last >> 1) & 1);
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after();
+    tc::dealloc(tmem, kQtCols);
+  }
+}
+
+template <typename T>
+cudaError_t launch_qt(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  static unsigned long long attr_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !((attr_set >> dev) & 1ull)) {
+    e = cudaFuncSetAttribute(quantize_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kQtSmem);
+    if (e != cudaSuccess) return e;
+    attr_set |= 1ull << dev;
+  }
+  const long long tiles = (long long)((a.n_tokens + kQtRows - 1) / kQtRows) * a.n_kv_heads * 2;
+  long long grid = tiles;
+  const long long cap = (long long)n_sm * 2 / a.layers.n;  // one wave of resident CTAs
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  quantize_tc_kernel<T><<<dim3((unsigned)grid, a.layers.n), kQtThreads, kQtSmem, stream>>>(
+      a.layers, a.n_kv_heads, a.n_tokens, a.seq_ids, a.positions);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool use_quantize_tc(const QuantizeArgs& a) {
+  return a.d == kQtD && a.bits == 3 && a.rope == nullptr &&
+         (a.dtype == ISOQ_BF16 || a.dtype == ISOQ_F16);
+}
+
+cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  switch (a.dtype) {
+    case ISOQ_BF16: return launch_qt<__nv_bfloat16>(a, stream, n_sm);
+    case ISOQ_F16: return launch_qt<__half>(a, stream, n_sm);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace isoq

@@ -199,8 +199,47 @@ def test_dtypes(oracle, kv_dtype, q_dtype):
     _log(f"dtype_{kv_dtype}_{q_dtype}_attention", check_attention(oracle, run, Q, out, lens))
 
 
-def test_zero_vector_and_norm_saturation(oracle):
-    cfg, lens = _custom(lens=(70,))
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("n_kv,lens", [(3, (1, 127, 128, 129)), (1, (255, 300)), (8, (513,))])
+def test_quantize_tiles(oracle, dtype, n_kv, lens):
+    """16-bit appends at d = 128 transform 128-token tiles on the tensor cores: lengths around
+    the tile size, an odd head count, several tiles per sequence."""
+    cfg, lens = _custom(n_kv=n_kv, G=2, lens=lens, dtype=dtype)
+    run = _len_run(cfg, lens)
+    run.prefill()
+    seqs = np.concatenate([np.full(n, s) for s, n in enumerate(lens)])
+    pos = np.concatenate([np.arange(n) for n in lens])
+    _log(f"tiles_{dtype}_H{n_kv}_{'-'.join(map(str, lens))}", _codes_all(oracle, run, seqs, pos))
+    assert iq.isoq_get_status(run.cache) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_quantize_tiles_mixed_tokens(oracle, dtype):
+    """One append whose tiles mix sequences and positions in shuffled order."""
+    cfg, lens = _custom(n_kv=2, G=2, lens=(150, 200), dtype=dtype)
+    run = _len_run(cfg, lens)
+    Ks, Vs, sids, poss = [], [], [], []
+    for s, n in enumerate(lens):
+        K, V = wl.kv_tokens(cfg, s, 0, n, device="cuda")
+        Ks.append(K)
+        Vs.append(V)
+        sids.append(torch.full((n,), s, dtype=torch.int32))
+        poss.append(torch.arange(n, dtype=torch.int32))
+    perm = torch.from_numpy(np.random.default_rng(7).permutation(sum(lens)))
+    K = torch.cat(Ks)[perm.cuda()].contiguous()
+    V = torch.cat(Vs)[perm.cuda()].contiguous()
+    sid = torch.cat(sids)[perm].cuda()
+    pos = torch.cat(poss)[perm].cuda()
+    iq.isoq_quantize_append(run.params, run.cache, K, V, sid, pos)
+    seqs = np.concatenate([np.full(n, s) for s, n in enumerate(lens)])
+    p = np.concatenate([np.arange(n) for n in lens])
+    _log(f"tiles_mixed_{dtype}", _codes_all(oracle, run, seqs, p))
+    assert iq.isoq_get_status(run.cache) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_zero_vector_and_norm_saturation(oracle, dtype):
+    cfg, lens = _custom(lens=(70,), dtype=dtype)
     run = _len_run(cfg, lens)
     K, V = wl.kv_tokens(cfg, 0, 0, 70, device="cuda")
     K[3] = 0.0          # zero vectors -> codes 4, norm 0
@@ -217,14 +256,15 @@ def test_zero_vector_and_norm_saturation(oracle):
     assert np.all(kn[7] == 0x7BFF)
     assert iq.isoq_get_status(run.cache) == iq.ISOQ_ST_NORM_SAT
     p64 = run.params64()
-    st = check_codes(oracle, p64, K.cpu().numpy().astype(np.float64), kc, kn, cfg.d)
+    st = check_codes(oracle, p64, K.float().cpu().numpy().astype(np.float64), kc, kn, cfg.d)
     _log("zero_and_saturation", st)
     iq.isoq_reset_status(run.cache)
     assert iq.isoq_get_status(run.cache) == 0
 
 
-def test_out_of_range_writes_are_skipped():
-    cfg, lens = _custom(lens=(64, 64))
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_out_of_range_writes_are_skipped(dtype):
+    cfg, lens = _custom(lens=(64, 64), dtype=dtype)
     run = _len_run(cfg, lens)
     K, V = wl.kv_tokens(cfg, 0, 0, 4, device="cuda")
     before = run.cache.blocks.clone()

@@ -200,10 +200,11 @@ def test_dtypes(oracle, kv_dtype, q_dtype):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("n_kv,lens", [(3, (1, 127, 128, 129)), (1, (255, 300)), (8, (513,))])
+@pytest.mark.parametrize("n_kv,lens", [(3, (1, 127, 128, 129)), (1, (255, 300)), (8, (513,)),
+                                       (8, (1300, 1281)), (5, (2000,))])
 def test_quantize_tiles(oracle, dtype, n_kv, lens):
     """16-bit appends at d = 128 transform 128-token tiles on the tensor cores: lengths around
-    the tile size, an odd head count, several tiles per sequence."""
+    the tile size, an odd head count, several tiles per sequence and per CTA."""
     cfg, lens = _custom(n_kv=n_kv, G=2, lens=lens, dtype=dtype)
     run = _len_run(cfg, lens)
     run.prefill()
@@ -214,9 +215,10 @@ def test_quantize_tiles(oracle, dtype, n_kv, lens):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-def test_quantize_tiles_mixed_tokens(oracle, dtype):
+@pytest.mark.parametrize("n_kv,lens", [(2, (150, 200)), (8, (1500, 1200))])
+def test_quantize_tiles_mixed_tokens(oracle, dtype, n_kv, lens):
     """One append whose tiles mix sequences and positions in shuffled order."""
-    cfg, lens = _custom(n_kv=2, G=2, lens=(150, 200), dtype=dtype)
+    cfg, lens = _custom(n_kv=n_kv, G=2, lens=lens, dtype=dtype)
     run = _len_run(cfg, lens)
     Ks, Vs, sids, poss = [], [], [], []
     for s, n in enumerate(lens):
@@ -233,7 +235,7 @@ def test_quantize_tiles_mixed_tokens(oracle, dtype):
     iq.isoq_quantize_append(run.params, run.cache, K, V, sid, pos)
     seqs = np.concatenate([np.full(n, s) for s, n in enumerate(lens)])
     p = np.concatenate([np.arange(n) for n in lens])
-    _log(f"tiles_mixed_{dtype}", _codes_all(oracle, run, seqs, p))
+    _log(f"tiles_mixed_{dtype}_H{n_kv}", _codes_all(oracle, run, seqs, p))
     assert iq.isoq_get_status(run.cache) == 0
 
 

@@ -263,7 +263,6 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
       // tokens of this lane: tb + 8n + 2t + e (n = 0..3, e = 0, 1).  sv = log2-domain score
       // (-inf when masked), nv = V norm (0 when masked)
       float sv[4][2], nv[4][2];
-      bool grow = false;
       const float sthr = m2 + kLazy, vthr = sigma * kSigmaSlack;
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
@@ -284,18 +283,17 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
           nv[n][0] = v0 ? nv[n][0] : 0.f;
           nv[n][1] = v1 ? nv[n][1] : 0.f;
         }
-        grow |= (fmaxf(sv[n][0], sv[n][1]) > sthr) | (fmaxf(nv[n][0], nv[n][1]) > vthr);
       }
+      // this lane's largest score and V norm of the tile (three-input max instructions)
+      float tmax = fmaxf(fmaxf(fmaxf(sv[0][0], sv[0][1]), fmaxf(sv[1][0], sv[1][1])),
+                         fmaxf(fmaxf(sv[2][0], sv[2][1]), fmaxf(sv[3][0], sv[3][1])));
+      float vmax = fmaxf(fmaxf(fmaxf(nv[0][0], nv[0][1]), fmaxf(nv[1][0], nv[1][1])),
+                         fmaxf(fmaxf(nv[2][0], nv[2][1]), fmaxf(nv[3][0], nv[3][1])));
+      const bool grow = (tmax > sthr) | (vmax > vthr);
       // ---- a8: online softmax.  The running max m2 of head g (shared by the 4 lanes t)
       // and the V-norm reference sigma move only when a score exceeds m2 + 8 or a norm
       // exceeds 16 sigma (first tile included), so the common tile needs no shuffles.
       if (__any_sync(kFull, grow)) {
-        float tmax = -CUDART_INF_F, vmax = 0.f;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          tmax = fmaxf(tmax, fmaxf(sv[n][0], sv[n][1]));
-          vmax = fmaxf(vmax, fmaxf(nv[n][0], nv[n][1]));
-        }
 #pragma unroll
         for (int o = 1; o < 4; o <<= 1) {
           tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, o));

@@ -61,7 +61,7 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_quantize_append(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
-// d = 128, 3 bits, bf16 / f16 inputs without RoPE: the WHT as a tensor-core product.
+// d = 128, bf16 / f16 inputs without RoPE: the WHT as a tensor-core product.
 bool use_quantize_tc(const QuantizeArgs& a);
 cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream, int n_sm);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);

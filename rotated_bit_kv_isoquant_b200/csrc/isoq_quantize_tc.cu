@@ -1,5 +1,5 @@
-// Quantize-append for d = 128, 3-bit codes, bf16 / f16 inputs, with the Walsh-Hadamard
-// transform on the 5th-generation tensor cores.
+// Quantize-append for d = 128 (2-, 3- and 4-bit codes), bf16 / f16 inputs, with the
+// Walsh-Hadamard transform on the 5th-generation tensor cores.
 //
 // Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
 // Compressed-Space Attention", Abstract: each K/V vector goes through a Walsh-Hadamard
@@ -12,8 +12,8 @@
 // exact products.  The rest runs on the CUDA cores over the accumulator rows: thread pair
 // (r, r + 128) owns vector r, each thread one half of its dims; the pair adds its halves'
 // sums of squares for the norm (|H x|^2 = 128 |x|^2), then each thread applies the head's
-// 4x4 block matrices, decides the codes against the norm-scaled thresholds, packs its two
-// 32-dim groups (24 bytes) and stores them into the paged cache.
+// 4x4 block matrices, decides the codes against the norm-scaled thresholds, packs its half
+// of the record (24 bytes at 3 bits) and stores it into the paged cache.
 //
 // Pipeline of a CTA over its tiles j: the copies of tile j+2 (cp.async of the 128 rows
 // into the operand layout, and the head's block matrices) and the UMMA of tile j+1 run
@@ -62,12 +62,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-template <typename T>
+template <typename T, int BITS>
 __global__ void __launch_bounds__(kQtThreads, 2)
     quantize_tc_kernel(const __grid_constant__ QuantLayers layers, int H, int n_tokens,
                        const int32_t* __restrict__ seq_ids,
                        const int32_t* __restrict__ positions) {
-  constexpr int BITS = 3, D = kQtD, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
+  constexpr int D = kQtD, CB = code_bytes(D, BITS), BB = block_bytes(D, BITS);
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdesc = tc::idesc_f16(128, 128, false, false, kBf16);
   const QuantLayer& L = layers.l[blockIdx.y];  // this launch row's layer
@@ -260,48 +260,76 @@ __global__ void __launch_bounds__(kQtThreads, 2)
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");  // warps quad, quad + 4
     const float n = sqrtf((red[r] + red[kQtRows + r]) * (1.0f / 128.0f));
 
-    // a3 + a4: block matrices and codes of this thread's two 32-dim groups
-    float TB[3];
+    // a3 + a4 + a5: block matrices and codes of this thread's 64 dims (16 blocks), summed
+    // into 16-bit half-words (one block at 3 and 4 bits, two at 2 bits) and packed into the
+    // thread's half of the record: bytes [CB/2 hf, CB/2 (hf + 1))
+    constexpr int NT = (1 << (BITS - 1)) - 1;  // positive thresholds
+    constexpr int HPB = BITS == 2 ? 2 : 1;     // blocks per half-word
+    constexpr int NHW = 16 / HPB;              // half-words of the thread
+    float TB[NT];
 #pragma unroll
-    for (int k = 0; k < 3; ++k)
+    for (int k = 0; k < NT; ++k)
       TB[k] = n == 0.f ? CUDART_INF_F : n * pos_threshold_f32(BITS, k) * 0x1p64f;
-    const float4* mh = reinterpret_cast<const float4*>(smem + kOffM + (li % 3) * kQtMat);
-    uint32_t rec[6];
+    const float4* mh = reinterpret_cast<const float4*>(smem + kOffM + (li % 3) * kQtMat) + 64 * hf;
+    uint32_t half[NHW];
 #pragma unroll
-    for (int gg = 0; gg < 2; ++gg) {
-      const int g = 2 * hf + gg;  // group of the vector
-      uint32_t half[8];
+    for (int hw = 0; hw < NHW; ++hw) {
+      float W = code_base<BITS>() * (BITS == 2 ? 21845.0f : 4369.0f);  // sum coef * base
 #pragma unroll
-      for (int bi = 0; bi < 8; ++bi) {
-        const int b = 8 * g + bi;  // block of the vector
-        float W = code_base<BITS>() * 4369.0f;  // sum coef * base over the 4 codes
+      for (int hb = 0; hb < HPB; ++hb) {
+        const int bl = hw * HPB + hb;  // block of the thread
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float4 m = mh[4 * b + e];
+          const float4 m = mh[4 * bl + e];
           // the chain starts from +0, so z is never -0 (which would code as negative)
-          const uint32_t* yb = y + 32 * gg + 4 * bi;
+          const uint32_t* yb = y + 4 * bl;
           const float z = fmaf(m.w, __uint_as_float(yb[3]),
                                fmaf(m.z, __uint_as_float(yb[2]),
                                     fmaf(m.y, __uint_as_float(yb[1]),
                                          fmaf(m.x, __uint_as_float(yb[0]), 0.0f))));
-          W = add_code<BITS>(W, z, (float)(1 << (4 * e)), TB);
+          const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + 4 * hb + e) & 7)))
+                                       : (float)(1 << (4 * e));
+          W = add_code<BITS>(W, z, coef, TB);
         }
-        half[bi] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W
       }
-      uint32_t nib[4];
+      half[hw] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W
+    }
+    constexpr int NR = CB / 8;  // words of the thread's half of the record
+    uint32_t rec[NR];
+    if constexpr (BITS == 3) {
+      // per 32-dim group: nibble words of dims 8j..8j+7, bit 3 from the group's last 8 codes
 #pragma unroll
-      for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[2 * j], half[2 * j + 1]);
+      for (int gg = 0; gg < 2; ++gg) {
+        uint32_t nib[4];
 #pragma unroll
-      for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
+        for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[8 * gg + 2 * j], half[8 * gg + 2 * j + 1]);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < NR; ++j) rec[j] = join_halves(half[2 * j], half[2 * j + 1]);
     }
 
     if (phys >= 0) {
       uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
       const int slot = pos & (kPage - 1);
-      uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB;
+      uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB + (CB / 2) * hf;
+      if constexpr (BITS == 3) {  // 24 bytes at 0 or 24: 16 + 8 or 8 + 16
+        if (hf == 0) {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(rec[0], rec[1], rec[2], rec[3]);
+          *reinterpret_cast<uint2*>(dst + 16) = make_uint2(rec[4], rec[5]);
+        } else {
+          *reinterpret_cast<uint2*>(dst) = make_uint2(rec[0], rec[1]);
+          *reinterpret_cast<uint4*>(dst + 8) = make_uint4(rec[2], rec[3], rec[4], rec[5]);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < NR / 4; ++q)
+          *reinterpret_cast<uint4*>(dst + 16 * q) =
+              make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
+      }
       if (hf == 0) {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(rec[0], rec[1], rec[2], rec[3]);
-        *reinterpret_cast<uint2*>(dst + 16) = make_uint2(rec[4], rec[5]);
         uint16_t nb = __half_as_ushort(__float2half_rn(n));
         if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
           nb = 0x7bffu;
@@ -309,9 +337,6 @@ __global__ void __launch_bounds__(kQtThreads, 2)
         }
         *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
                                      2 * slot) = nb;
-      } else {
-        *reinterpret_cast<uint2*>(dst + 24) = make_uint2(rec[0], rec[1]);
-        *reinterpret_cast<uint4*>(dst + 32) = make_uint4(rec[2], rec[3], rec[4], rec[5]);
       }
     }
     if (has_next) {
@@ -340,14 +365,14 @@ __global__ void __launch_bounds__(kQtThreads, 2)
   }
 }
 
-template <typename T>
+template <typename T, int BITS>
 cudaError_t launch_qt(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   static unsigned long long attr_set = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !((attr_set >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(quantize_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(quantize_tc_kernel<T, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kQtSmem);
     if (e != cudaSuccess) return e;
     attr_set |= 1ull << dev;
@@ -357,7 +382,7 @@ cudaError_t launch_qt(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   const long long cap = (long long)n_sm * 2 / a.layers.n;  // one wave of resident CTAs
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  quantize_tc_kernel<T><<<dim3((unsigned)grid, a.layers.n), kQtThreads, kQtSmem, stream>>>(
+  quantize_tc_kernel<T, BITS><<<dim3((unsigned)grid, a.layers.n), kQtThreads, kQtSmem, stream>>>(
       a.layers, a.n_kv_heads, a.n_tokens, a.seq_ids, a.positions);
   return cudaGetLastError();
 }
@@ -365,14 +390,24 @@ cudaError_t launch_qt(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
 }  // namespace
 
 bool use_quantize_tc(const QuantizeArgs& a) {
-  return a.d == kQtD && a.bits == 3 && a.rope == nullptr &&
+  return a.d == kQtD && a.bits >= 2 && a.bits <= 4 && a.rope == nullptr &&
          (a.dtype == ISOQ_BF16 || a.dtype == ISOQ_F16);
+}
+
+template <typename T>
+cudaError_t launch_qt_b(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
+  switch (a.bits) {
+    case 2: return launch_qt<T, 2>(a, stream, n_sm);
+    case 3: return launch_qt<T, 3>(a, stream, n_sm);
+    case 4: return launch_qt<T, 4>(a, stream, n_sm);
+  }
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_quantize_tc(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   switch (a.dtype) {
-    case ISOQ_BF16: return launch_qt<__nv_bfloat16>(a, stream, n_sm);
-    case ISOQ_F16: return launch_qt<__half>(a, stream, n_sm);
+    case ISOQ_BF16: return launch_qt_b<__nv_bfloat16>(a, stream, n_sm);
+    case ISOQ_F16: return launch_qt_b<__half>(a, stream, n_sm);
   }
   return cudaErrorInvalidValue;
 }

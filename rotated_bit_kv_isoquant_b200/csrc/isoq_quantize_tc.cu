@@ -9,11 +9,11 @@
 // H[k][n] = (-1)^popc(k & n).  Its entries are exact in bf16 and f16, and so are the
 // inputs, so the transform of a tile of 128 vectors (128 consecutive tokens of one KV head,
 // K or V) is one 128 x 128 x 128 UMMA (kind::f16, f32 accumulator in tensor memory) with
-// exact products.  The rest runs on the CUDA cores over the accumulator rows: thread pair
-// (r, r + 128) owns vector r, each thread one half of its dims; the pair adds its halves'
-// sums of squares for the norm (|H x|^2 = 128 |x|^2), then each thread applies the head's
-// 4x4 block matrices, decides the codes against the norm-scaled thresholds, packs its half
-// of the record (24 bytes at 3 bits) and stores it into the paged cache.
+// exact products.  The rest runs on the CUDA cores over the accumulator rows: thread r
+// owns vector r (tensor-memory lane r).  It sums the squares of its row for the norm
+// (|H x|^2 = 128 |x|^2), then, one 64-dim half at a time, applies the head's 4x4 block
+// matrices, decides the codes against the norm-scaled thresholds, packs them and stores
+// that half of the record (24 bytes at 3 bits) into the paged cache.
 //
 // Pipeline of a CTA over its tiles j: the copies of tile j+2 (cp.async of the 128 rows
 // into the operand layout, and the head's block matrices) and the UMMA of tile j+1 run
@@ -39,14 +39,13 @@ using namespace ptx;
 
 constexpr int kQtD = 128;
 constexpr int kQtRows = 128;                      // vectors per tile = UMMA M
-constexpr int kQtThreads = 256;                   // two threads per vector
+constexpr int kQtThreads = 128;                   // one thread per vector (row)
 constexpr int kQtTile = kQtRows * kQtD * 2;       // one 16-bit operand tile, 32 KiB
 constexpr int kQtMat = 32 * 16 * 4;               // one head's block matrices, 2 KiB
 constexpr int kOffX = 0;                          // [2] input tiles
 constexpr int kOffH = 2 * kQtTile;                // the Hadamard operand
 constexpr int kOffM = kOffH + kQtTile;            // [3] block-matrix stages
-constexpr int kOffRed = kOffM + 3 * kQtMat;       // [2][128] half sums of squares
-constexpr int kOffBar = kOffRed + 2 * kQtRows * 4;  // 2 mbarriers (UMMA completion)
+constexpr int kOffBar = kOffM + 3 * kQtMat;       // 2 mbarriers (UMMA completion)
 constexpr int kOffSlot = kOffBar + 16;            // tensor-memory base address
 constexpr int kQtSmem = kOffSlot + 16;
 constexpr uint32_t kQtCols = 256;                 // two 128-column f32 accumulators
@@ -81,13 +80,12 @@ __global__ void __launch_bounds__(kQtThreads, 2)
 
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
-  float* red = reinterpret_cast<float*>(smem + kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffSlot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, hf = warp >> 2;  // tensor-memory lane quarter, half of the dims
-  const int r = quad * 32 + lane;             // this thread's vector (row) of the tile
+  const int quad = warp;           // tensor-memory lane quarter
+  const int r = quad * 32 + lane;  // this thread's vector (row) of the tile
   const int n_chunks = (n_tokens + kQtRows - 1) / kQtRows;
   const int n_kinds = 2 * H;             // (head, K|V) pairs: rr = 2 head + kind
   const int n_tiles = n_chunks * n_kinds;  // tile = (128-token chunk, head, K|V), chunk-major
@@ -113,7 +111,7 @@ __global__ void __launch_bounds__(kQtThreads, 2)
   // copies of tile t (local index li) into input stage li & 1 and matrix stage li % 3; a
   // warp's copy covers 8 rows x 64 bytes, 512 contiguous bytes of the tile.  Rows past the
   // last token are not copied (their accumulator rows are never used).
-  const int cp_row = 8 * (tid >> 7) + (tid & 7), cp_j = (tid >> 3) & 15;  // + 16 c
+  const int cp_row = tid & 7, cp_j = (tid >> 3) & 15;  // + 8 c
   const uint32_t cp_dst = qt_off(cp_row, 8 * cp_j);
   const size_t row_bytes = (size_t)H * D * sizeof(T);
   auto prefetch = [&](Tile t, int li) {
@@ -125,8 +123,8 @@ __global__ void __launch_bounds__(kQtThreads, 2)
       const uint32_t xs = sbase + kOffX + (li & 1) * kQtTile + cp_dst;
       const int rows_left = n_tokens - t0 - cp_row;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (16 * c < rows_left) cp_async16(xs + 4096 * c, src + 16 * c * row_bytes);
+      for (int c = 0; c < 16; ++c)
+        if (8 * c < rows_left) cp_async16(xs + 2048 * c, src + 8 * c * row_bytes);
       if (tid < kQtMat / 16)
         cp_async16(sbase + kOffM + (li % 3) * kQtMat + 16 * tid,
                    reinterpret_cast<const uint8_t*>(mats) + (size_t)h * kQtMat + 16 * tid);
@@ -136,13 +134,13 @@ __global__ void __launch_bounds__(kQtThreads, 2)
   prefetch(cur, 0);
   prefetch(nxt, 1);
 
-  // the Hadamard operand (N x K, K-major; symmetric): thread -> row tid / 2, 64 dims
+  // the Hadamard operand (N x K, K-major; symmetric): thread -> row tid
   {
     const uint32_t one = kBf16 ? 0x3F80u : 0x3C00u;
-    const int n = tid >> 1;
-#pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-      const int k0 = 64 * (tid & 1) + 8 * kc;
+    const int n = tid;
+#pragma unroll 4
+    for (int kc = 0; kc < 16; ++kc) {
+      const int k0 = 8 * kc;
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -176,13 +174,13 @@ __global__ void __launch_bounds__(kQtThreads, 2)
     phys = -1;
     if (t >= n_tokens) return;
     if (sid < 0 || sid >= n_seqs) {
-      if (hf == 0) set_status(status, ISOQ_ST_SEQ_RANGE);
+      set_status(status, ISOQ_ST_SEQ_RANGE);
     } else if (pos < 0 || (pos >> 6) >= max_pages) {
-      if (hf == 0) set_status(status, ISOQ_ST_POS_RANGE);
+      set_status(status, ISOQ_ST_POS_RANGE);
     } else {
       phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
       if (phys < 0 || phys >= n_pages) {
-        if (hf == 0) set_status(status, ISOQ_ST_PAGE_RANGE);
+        set_status(status, ISOQ_ST_PAGE_RANGE);
         phys = -1;
       }
     }
@@ -237,106 +235,112 @@ __global__ void __launch_bounds__(kQtThreads, 2)
     prefetch(nn, li + 2);  // input stage li & 1 is free again
 
     const int h = cur.rr >> 1, kind = cur.rr & 1;
-    const uint32_t acc = t_row + (uint32_t)(li & 1) * 128 + 64 * hf;  // this thread's 64 dims
+    const uint32_t acc = t_row + (uint32_t)(li & 1) * 128;  // this thread's vector
 
-    // a1: norm from the transform, |x|^2 = |H x|^2 / 128.  The pair's halves meet in
-    // shared memory behind a barrier of its two warps and are added in a fixed order, so
-    // both threads hold the same value.
+    // a1: norm from the transform, |x|^2 = |H x|^2 / 128
     uint32_t y[64];
-    tc::ld64(acc, y);
+    float n;
     {
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 64; e += 4) {
-        const float a = __uint_as_float(y[e]), b = __uint_as_float(y[e + 1]);
-        const float cc = __uint_as_float(y[e + 2]), dd = __uint_as_float(y[e + 3]);
-        s0 = fmaf(a, a, s0);
-        s1 = fmaf(b, b, s1);
-        s2 = fmaf(cc, cc, s2);
-        s3 = fmaf(dd, dd, s3);
+      for (int hh = 0; hh < 2; ++hh) {
+        tc::ld64(acc + 64 * hh, y);
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+          const float a = __uint_as_float(y[e]), b = __uint_as_float(y[e + 1]);
+          const float cc = __uint_as_float(y[e + 2]), dd = __uint_as_float(y[e + 3]);
+          s0 = fmaf(a, a, s0);
+          s1 = fmaf(b, b, s1);
+          s2 = fmaf(cc, cc, s2);
+          s3 = fmaf(dd, dd, s3);
+        }
       }
-      red[hf * kQtRows + r] = (s0 + s1) + (s2 + s3);
+      n = sqrtf(((s0 + s1) + (s2 + s3)) * (1.0f / 128.0f));
     }
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");  // warps quad, quad + 4
-    const float n = sqrtf((red[r] + red[kQtRows + r]) * (1.0f / 128.0f));
 
-    // a3 + a4 + a5: block matrices and codes of this thread's 64 dims (16 blocks), summed
-    // into 16-bit half-words (one block at 3 and 4 bits, two at 2 bits) and packed into the
-    // thread's half of the record: bytes [CB/2 hf, CB/2 (hf + 1))
+    // a3 + a4 + a5: per 64-dim half hf of the vector, block matrices and codes of its 16
+    // blocks, summed into 16-bit half-words (one block at 3 and 4 bits, two at 2 bits) and
+    // packed into that half of the record: bytes [CB/2 hf, CB/2 (hf + 1))
     constexpr int NT = (1 << (BITS - 1)) - 1;  // positive thresholds
     constexpr int HPB = BITS == 2 ? 2 : 1;     // blocks per half-word
-    constexpr int NHW = 16 / HPB;              // half-words of the thread
+    constexpr int NHW = 16 / HPB;              // half-words of a half
     float TB[NT];
 #pragma unroll
     for (int k = 0; k < NT; ++k)
       TB[k] = n == 0.f ? CUDART_INF_F : n * pos_threshold_f32(BITS, k) * 0x1p64f;
-    const float4* mh = reinterpret_cast<const float4*>(smem + kOffM + (li % 3) * kQtMat) + 64 * hf;
-    uint32_t half[NHW];
+    // the second half first: the norm pass left its columns in y
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int hf = 1 - pass;
+      if (pass) tc::ld64(acc, y);  // the first half's columns
+      const float4* mh = reinterpret_cast<const float4*>(smem + kOffM + (li % 3) * kQtMat) + 64 * hf;
+      uint32_t half[NHW];
 #pragma unroll
-    for (int hw = 0; hw < NHW; ++hw) {
-      float W = code_base<BITS>() * (BITS == 2 ? 21845.0f : 4369.0f);  // sum coef * base
+      for (int hw = 0; hw < NHW; ++hw) {
+        float W = code_base<BITS>() * (BITS == 2 ? 21845.0f : 4369.0f);  // sum coef * base
 #pragma unroll
-      for (int hb = 0; hb < HPB; ++hb) {
-        const int bl = hw * HPB + hb;  // block of the thread
+        for (int hb = 0; hb < HPB; ++hb) {
+          const int bl = hw * HPB + hb;  // block of the half
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 m = mh[4 * bl + e];
-          // the chain starts from +0, so z is never -0 (which would code as negative)
-          const uint32_t* yb = y + 4 * bl;
-          const float z = fmaf(m.w, __uint_as_float(yb[3]),
-                               fmaf(m.z, __uint_as_float(yb[2]),
-                                    fmaf(m.y, __uint_as_float(yb[1]),
-                                         fmaf(m.x, __uint_as_float(yb[0]), 0.0f))));
-          const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + 4 * hb + e) & 7)))
-                                       : (float)(1 << (4 * e));
-          W = add_code<BITS>(W, z, coef, TB);
+          for (int e = 0; e < 4; ++e) {
+            const float4 m = mh[4 * bl + e];
+            // the chain starts from +0, so z is never -0 (which would code as negative)
+            const uint32_t* yb = y + 4 * bl;
+            const float z = fmaf(m.w, __uint_as_float(yb[3]),
+                                 fmaf(m.z, __uint_as_float(yb[2]),
+                                      fmaf(m.y, __uint_as_float(yb[1]),
+                                           fmaf(m.x, __uint_as_float(yb[0]), 0.0f))));
+            const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + 4 * hb + e) & 7)))
+                                         : (float)(1 << (4 * e));
+            W = add_code<BITS>(W, z, coef, TB);
+          }
         }
+        half[hw] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W
       }
-      half[hw] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W
-    }
-    constexpr int NR = CB / 8;  // words of the thread's half of the record
-    uint32_t rec[NR];
-    if constexpr (BITS == 3) {
-      // per 32-dim group: nibble words of dims 8j..8j+7, bit 3 from the group's last 8 codes
+      constexpr int NR = CB / 8;  // words of half the record
+      uint32_t rec[NR];
+      if constexpr (BITS == 3) {
+        // per 32-dim group: nibble words of dims 8j..8j+7, bit 3 from the group's last 8 codes
 #pragma unroll
-      for (int gg = 0; gg < 2; ++gg) {
-        uint32_t nib[4];
+        for (int gg = 0; gg < 2; ++gg) {
+          uint32_t nib[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[8 * gg + 2 * j], half[8 * gg + 2 * j + 1]);
+          for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[8 * gg + 2 * j], half[8 * gg + 2 * j + 1]);
 #pragma unroll
-        for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < NR; ++j) rec[j] = join_halves(half[2 * j], half[2 * j + 1]);
-    }
-
-    if (phys >= 0) {
-      uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
-      const int slot = pos & (kPage - 1);
-      uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB + (CB / 2) * hf;
-      if constexpr (BITS == 3) {  // 24 bytes at 0 or 24: 16 + 8 or 8 + 16
-        if (hf == 0) {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(rec[0], rec[1], rec[2], rec[3]);
-          *reinterpret_cast<uint2*>(dst + 16) = make_uint2(rec[4], rec[5]);
-        } else {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(rec[0], rec[1]);
-          *reinterpret_cast<uint4*>(dst + 8) = make_uint4(rec[2], rec[3], rec[4], rec[5]);
+          for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < NR / 4; ++q)
-          *reinterpret_cast<uint4*>(dst + 16 * q) =
-              make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
+        for (int j = 0; j < NR; ++j) rec[j] = join_halves(half[2 * j], half[2 * j + 1]);
       }
-      if (hf == 0) {
-        uint16_t nb = __half_as_ushort(__float2half_rn(n));
-        if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
-          nb = 0x7bffu;
-          set_status(status, ISOQ_ST_NORM_SAT);
+
+      if (phys >= 0) {
+        uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
+        const int slot = pos & (kPage - 1);
+        uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB + (CB / 2) * hf;
+        if constexpr (BITS == 3) {  // 24 bytes at 0 or 24: 16 + 8 or 8 + 16
+          if (hf == 0) {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(rec[0], rec[1], rec[2], rec[3]);
+            *reinterpret_cast<uint2*>(dst + 16) = make_uint2(rec[4], rec[5]);
+          } else {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(rec[0], rec[1]);
+            *reinterpret_cast<uint4*>(dst + 8) = make_uint4(rec[2], rec[3], rec[4], rec[5]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < NR / 4; ++q)
+            *reinterpret_cast<uint4*>(dst + 16 * q) =
+                make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
         }
-        *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
-                                     2 * slot) = nb;
+        if (hf == 0) {
+          uint16_t nb = __half_as_ushort(__float2half_rn(n));
+          if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
+            nb = 0x7bffu;
+            set_status(status, ISOQ_ST_NORM_SAT);
+          }
+          *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
+                                       2 * slot) = nb;
+        }
       }
     }
     if (has_next) {

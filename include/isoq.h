@@ -199,8 +199,8 @@ size_t isoq_block_bytes(int d, int page_size);
  * binary16 norm are written to slot positions[t] % 64 of page
  * page_table[seq_ids[t]][positions[t] / 64].
  *
- * K, V: device [n_tokens][n_kv_heads][d] contiguous, element type `dtype` (ISOQ_F32,
- * ISOQ_BF16 or ISOQ_F16).  seq_ids, positions: device int32 [n_tokens].
+ * K, V: device [n_tokens][n_kv_heads][d] contiguous, 16-byte aligned (ISOQ_E_ARG
+ * otherwise), element type `dtype` (ISOQ_F32, ISOQ_BF16 or ISOQ_F16).  seq_ids, positions: device int32 [n_tokens].
  * n_tokens == 0 is a no-op.  Arithmetic is binary32; the code decision compares
  * sqrt(d) z_i against n t_j with no division.
  * Errors: ISOQ_E_ARG (null pointers, n_tokens < 0, unknown dtype), ISOQ_E_DIM (cache d or

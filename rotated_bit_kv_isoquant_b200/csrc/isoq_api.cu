@@ -325,7 +325,9 @@ int quantize_common(const isoq_params* const* params, const isoq_cache* const* c
   if (n_tokens == 0) return ISOQ_OK;
   if (!seq_ids || !positions) return ISOQ_E_ARG;
   for (int i = 0; i < n_layers; ++i) {
-    if (!K[i] || !V[i]) return ISOQ_E_ARG;
+    // the kernels copy whole vectors in 16-byte pieces
+    if (!K[i] || !V[i] || ((uintptr_t)K[i] & 15u) != 0 || ((uintptr_t)V[i] & 15u) != 0)
+      return ISOQ_E_ARG;
     const int rc = check_device(params[i]);
     if (rc) return rc;
   }

@@ -337,6 +337,17 @@ def test_error_codes():
     with pytest.raises(iq.IsoqError) as e:
         iq.isoq_make_params(0, 96, 2)
     assert e.value.code == iq.ISOQ_E_DIM
+    # K, V must start on a 16-byte boundary (rejected before any launch; cache untouched)
+    K, V = wl.kv_tokens(cfg, 0, 0, 3, device="cuda")
+    flat = torch.empty(K.numel() + 8, dtype=K.dtype, device="cuda")
+    Kmis = flat[1:1 + K.numel()].view(K.shape)
+    Kmis.copy_(K)
+    before = run.cache.blocks.clone()
+    with pytest.raises(iq.IsoqError) as e:
+        iq.isoq_quantize_append(run.params, run.cache, Kmis, V, sl[:1].repeat(3) * 0,
+                                torch.arange(3, dtype=torch.int32, device="cuda"))
+    assert e.value.code == iq.ISOQ_E_ARG
+    assert torch.equal(run.cache.blocks, before)
     lib = iq.raw_lib()
     import ctypes
     assert lib.isoq_decode_attention(run.params.handle, ctypes.byref(run.cache.c), None, 0, 1,

@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
         }
       }
     };
-#pragma unroll 1
+#pragma unroll
     for (int tb = 0; tb < kPage; tb += 32) {
       if (full) tile(tb, std::true_type{});
       else tile(tb, std::false_type{});

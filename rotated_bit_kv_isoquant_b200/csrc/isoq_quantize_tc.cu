@@ -57,6 +57,18 @@ __host__ __device__ constexpr uint32_t qt_off(int row, int k) {
   return (uint32_t)((row >> 3) * 2048 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
 }
 
+// Packed pair of binary32 FMAs (one instruction, the same rounding per lane as fmaf).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("{\n .reg .b64 pa, pb, pc;\n mov.b64 pa, {%1, %2};\n mov.b64 pb, {%3, %4};\n"
+      " mov.b64 pc, {%5, %6};\n fma.rn.f32x2 %0, pa, pb, pc;\n}"
+      : "=l"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  float2 o;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+  return o;
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -241,21 +253,19 @@ __global__ void __launch_bounds__(kQtThreads, 2)
     uint32_t y[64];
     float n;
     {
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      float2 s01 = make_float2(0.f, 0.f), s23 = make_float2(0.f, 0.f);  // four partial sums
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         tc::ld64(acc + 64 * hh, y);
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
-          const float a = __uint_as_float(y[e]), b = __uint_as_float(y[e + 1]);
-          const float cc = __uint_as_float(y[e + 2]), dd = __uint_as_float(y[e + 3]);
-          s0 = fmaf(a, a, s0);
-          s1 = fmaf(b, b, s1);
-          s2 = fmaf(cc, cc, s2);
-          s3 = fmaf(dd, dd, s3);
+          const float2 ab = make_float2(__uint_as_float(y[e]), __uint_as_float(y[e + 1]));
+          const float2 cd = make_float2(__uint_as_float(y[e + 2]), __uint_as_float(y[e + 3]));
+          s01 = fma2(ab, ab, s01);
+          s23 = fma2(cd, cd, s23);
         }
       }
-      n = sqrtf(((s0 + s1) + (s2 + s3)) * (1.0f / 128.0f));
+      n = sqrtf(((s01.x + s01.y) + (s23.x + s23.y)) * (1.0f / 128.0f));
     }
 
     // a3 + a4 + a5: per 64-dim half hf of the vector, block matrices and codes of its 16
@@ -284,12 +294,15 @@ __global__ void __launch_bounds__(kQtThreads, 2)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float4 m = mh[4 * bl + e];
-            // the chain starts from +0, so z is never -0 (which would code as negative)
+            // row e of the block as two packed FMA chains (dims 0, 2 and 1, 3) from +0, so z
+            // is never -0 (which would code as negative)
             const uint32_t* yb = y + 4 * bl;
-            const float z = fmaf(m.w, __uint_as_float(yb[3]),
-                                 fmaf(m.z, __uint_as_float(yb[2]),
-                                      fmaf(m.y, __uint_as_float(yb[1]),
-                                           fmaf(m.x, __uint_as_float(yb[0]), 0.0f))));
+            float2 p = fma2(make_float2(m.x, m.y),
+                            make_float2(__uint_as_float(yb[0]), __uint_as_float(yb[1])),
+                            make_float2(0.f, 0.f));
+            p = fma2(make_float2(m.z, m.w),
+                     make_float2(__uint_as_float(yb[2]), __uint_as_float(yb[3])), p);
+            const float z = p.x + p.y;
             const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + 4 * hb + e) & 7)))
                                          : (float)(1 << (4 * e));
             W = add_code<BITS>(W, z, coef, TB);

@@ -108,8 +108,16 @@ class ContextParallelDecoder:
 
     def __call__(self, Q, local_lens, out, scale: float, stream=None):
         """Q [n_seqs][n_q_heads][d] (same on every rank), local_lens int32 [n_seqs] (this
-        rank's slice lengths); writes the attention over the whole contexts to out."""
-        self.local_state(Q, local_lens, scale, stream)
-        states = gather_states(self.state, self.group)
-        isoq_decode_merge_states(self.params, states, out, stream)
+        rank's slice lengths); writes the attention over the whole contexts to out.
+
+        All three steps run on `stream` (default: the current stream).  The all-gather is
+        issued with that stream current, so torch.distributed orders it after the
+        partial-state kernel and the merge after the all-gather; a stream other than the
+        current one therefore needs no extra synchronisation by the caller."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.state.device)
+        with torch.cuda.stream(s):
+            self.local_state(Q, local_lens, scale, s)
+            states = gather_states(self.state, self.group)
+            isoq_decode_merge_states(self.params, states, out, s)
         return out

@@ -111,12 +111,10 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
   // the multi-token kernels (64 or 128 rows per CTA, 2 CTAs per SM) when a chunk gives a
   // KV head at least 16 rows; else the per-row kernel (8 rows per CTA)
   const bool shared_mq = d == 128 && n_q > 1 && (long long)n_q * group >= 16;
-  const bool tc = !shared_mq && n_q == 1 && isoq::kUseTc128 && d == 128;
-  const int n_sm = sm_count() * (shared_mq ? 2 : tc ? isoq::decode_tc_resident_ctas()
-                                                    : isoq::decode_resident_ctas(d));
+  const int n_sm = sm_count() * (shared_mq ? 2 : isoq::decode_resident_ctas(d));
   const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group) : 8;
   // pages per CTA worth a launch: the tensor-memory kernel rotates 128 queries per CTA
-  const int min_pages = shared_mq ? (rows_per_cta == 128 ? 16 : 4) : tc ? 8 : ISOQ_DEC_MIN_PAGES;
+  const int min_pages = shared_mq ? (rows_per_cta == 128 ? 16 : 4) : ISOQ_DEC_MIN_PAGES;
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
   const long long units =
       (long long)n_seqs * n_kv_heads * (((long long)n_q * group + rows_per_cta - 1) / rows_per_cta);
@@ -449,7 +447,7 @@ bool rows_fit(int n_q, int n_q_heads, int n_kv_heads) {
 
 // Shared by the decode entry points: validation, the split plan, then the split kernel and
 // the combine into either the output rows (out) or merged states (state).
-int decode_common(const isoq_params* params, const isoq_cache* cache, const void* Q,
+int decode_common_impl(const isoq_params* params, const isoq_cache* cache, const void* Q,
                   int q_dtype, int n_seqs, int n_q, int n_q_heads, const int32_t* seq_lens,
                   int max_seq_len, float* out, float* state, float scale, void* workspace,
                   size_t workspace_bytes, void* stream) {
@@ -496,6 +494,26 @@ int decode_common(const isoq_params* params, const isoq_cache* cache, const void
   return e == cudaSuccess ? ISOQ_OK : cuda_fail(e);
 }
 
+}  // namespace
+
+namespace isoq {
+int decode_run(const isoq_params* params, const isoq_cache* cache, const void* Q, int q_dtype,
+               int n_seqs, int n_q, int n_q_heads, const int32_t* seq_lens, int max_seq_len,
+               float* out, float* state, float scale, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  return decode_common_impl(params, cache, Q, q_dtype, n_seqs, n_q, n_q_heads, seq_lens,
+                            max_seq_len, out, state, scale, workspace, workspace_bytes, stream);
+}
+}  // namespace isoq
+
+namespace {
+inline int decode_common(const isoq_params* params, const isoq_cache* cache, const void* Q,
+                         int q_dtype, int n_seqs, int n_q, int n_q_heads, const int32_t* seq_lens,
+                         int max_seq_len, float* out, float* state, float scale, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return decode_common_impl(params, cache, Q, q_dtype, n_seqs, n_q, n_q_heads, seq_lens,
+                            max_seq_len, out, state, scale, workspace, workspace_bytes, stream);
+}
 }  // namespace
 
 extern "C" {

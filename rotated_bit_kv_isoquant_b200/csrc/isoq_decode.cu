@@ -136,9 +136,8 @@ __global__ void __launch_bounds__(128)
 
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
-  cudaError_t e = use_shared_mq(a)                                    ? launch_decode_split_mq(a, stream)
-                  : (kUseTc128 && D == 128 && a.n_q == 1 && a.bits == 3) ? launch_decode_split_tc(a, stream)
-                                                                          : launch_decode_split_mma(a, stream);
+  cudaError_t e = use_shared_mq(a) ? launch_decode_split_mq(a, stream)
+                                   : launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
   const int rows = a.n_q * a.n_q_heads;
   dim3 grid(rows, a.n_seqs);

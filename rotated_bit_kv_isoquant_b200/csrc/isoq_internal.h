@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 struct isoq_params;
+struct isoq_cache;
 
 namespace isoq {
 
@@ -91,17 +92,6 @@ inline int attention_rows_per_cta(int d, int n_q, int group) {
   if (d != 128 || n_q <= 1 || rows < 16) return 8;
   return rows >= ISOQ_MQTC_MIN_ROWS ? 128 : 64;
 }
-// Tensor-memory (tcgen05) split kernel, head dimension 128 (partials only).
-cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t stream);
-int decode_tc_resident_ctas();
-
-// The decode uses the mma.sync kernel; building with ISOQ_DECODE_TC selects the tcgen05
-// kernel for d = 128 instead (parity-equivalent, measured slower: see the design notes).
-#ifdef ISOQ_DECODE_TC
-constexpr bool kUseTc128 = true;
-#else
-constexpr bool kUseTc128 = false;
-#endif
 
 // Accessors of the opaque parameter handle (defined in isoq_api.cu).
 const float* params_device_mats(const struct ::isoq_params* p);  // [H][d/4][4][4]
@@ -109,6 +99,12 @@ int params_bits(const struct ::isoq_params* p);
 int params_device(const struct ::isoq_params* p);
 // Records e as the thread's last CUDA error and returns ISOQ_E_CUDA.
 int record_cuda_error(cudaError_t e);
+// The decode entry points' shared body (defined in isoq_api.cu): argument checks, the
+// split plan, the split kernel and the combine, with the split partials in `workspace`.
+int decode_run(const struct ::isoq_params* params, const ::isoq_cache* cache, const void* Q,
+               int q_dtype, int n_seqs, int n_q, int n_q_heads, const int32_t* seq_lens,
+               int max_seq_len, float* out, float* state, float scale, void* workspace,
+               size_t workspace_bytes, void* stream);
 
 // Partial-result stride (floats) of one (sequence, head, split): acc[d], m, l, 2 pad.
 inline int partial_stride(int d) { return d + 4; }

@@ -19,7 +19,6 @@
 //   * the first call on a device looks up the array's device address there
 //     (cudaGetSymbolAddress), so make that first call before any stream capture.
 #include <cuda_runtime.h>
-#include <math.h>
 
 #include <mutex>
 
@@ -55,8 +54,6 @@ float* scratch_address(int device, cudaError_t* err) {
   return addr[device];
 }
 
-bool valid_dtype(int t) { return t == ISOQ_F32 || t == ISOQ_BF16 || t == ISOQ_F16; }
-
 }  // namespace
 
 extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const isoq_cache* cache,
@@ -64,33 +61,11 @@ extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const is
                                              int n_q_heads, const int32_t* seq_lens,
                                              int max_seq_len, float* out, float scale,
                                              void* stream) {
-  if (!params || !cache || !cache->blocks || !cache->page_table) return ISOQ_E_ARG;
-  int pd = 0, ph = 0;
-  isoq_params_shape(params, &pd, &ph);
-  if (cache->page_size != ISOQ_PAGE_SIZE || (cache->d != 128 && cache->d != 256))
-    return ISOQ_E_DIM;
-  if (cache->d != pd || cache->n_kv_heads != ph) return ISOQ_E_DIM;
-  if ((cache->bits == 0 ? 3 : cache->bits) != isoq::params_bits(params)) return ISOQ_E_DIM;
-  if (cache->n_pages < 0 || cache->max_pages_per_seq < 1 || cache->n_seqs < 1 ||
-      cache->n_kv_heads < 1)
-    return ISOQ_E_ARG;
-  if (n_seqs < 0 || n_q_heads < 0 || max_seq_len < 0 || !valid_dtype(q_dtype)) return ISOQ_E_ARG;
-  if (!(scale == scale) || isinf(scale)) return ISOQ_E_ARG;
-  if (n_q_heads % cache->n_kv_heads || n_q_heads / cache->n_kv_heads > 16) return ISOQ_E_GQA;
-  if (n_seqs > cache->n_seqs) return ISOQ_E_ARG;
-  if (n_seqs == 0 || n_q_heads == 0) return ISOQ_OK;
-  if (!Q || !seq_lens || !out) return ISOQ_E_ARG;
-
-  // Same context chunking as isoq_decode_attention; reject what does not fit the array.
-  const size_t need = isoq_decode_workspace_bytes(n_seqs, n_q_heads, cache->n_kv_heads,
-                                                  cache->d, max_seq_len);
-  if (need == 0 || need > (size_t)ISOQ_NOALLOC_SCRATCH_BYTES) return ISOQ_E_WORKSPACE;
-  const int n_splits =
-      isoq_decode_num_splits(n_seqs, n_q_heads, cache->n_kv_heads, cache->d, max_seq_len);
-  if (n_splits < 1) return n_splits < 0 ? n_splits : ISOQ_E_ARG;
-  const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
-  const int pages_per_split = (max_pages + n_splits - 1) / n_splits;
-
+  if (!params) return ISOQ_E_ARG;
+  // The array's address is looked up with the parameters' device current (the address is
+  // per device); the decode then runs exactly as isoq_decode_attention does -- same checks,
+  // same split plan, same kernels -- with the array as its workspace, and refuses a plan
+  // whose partials do not fit the array (ISOQ_E_WORKSPACE, nothing launched).
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -101,28 +76,7 @@ extern "C" int isoq_decode_attention_noalloc(const isoq_params* params, const is
   if (dev != isoq::params_device(params)) return ISOQ_E_DEVICE;
   float* scratch = scratch_address(dev, &e);
   if (!scratch) return isoq::record_cuda_error(e);
-
-  isoq::DecodeArgs a{};
-  a.params = isoq::params_device_mats(params);
-  a.bits = isoq::params_bits(params);
-  a.blocks = cache->blocks;
-  a.page_table = cache->page_table;
-  a.n_pages = cache->n_pages;
-  a.max_pages = cache->max_pages_per_seq;
-  a.n_kv_heads = cache->n_kv_heads;
-  a.d = cache->d;
-  a.Q = Q;
-  a.q_dtype = q_dtype;
-  a.n_seqs = n_seqs;
-  a.n_q_heads = n_q_heads;
-  a.n_q = 1;
-  a.seq_lens = seq_lens;
-  a.scale = scale;
-  a.n_splits = n_splits;
-  a.pages_per_split = pages_per_split;
-  a.partials = scratch;
-  a.out = out;
-  a.status = cache->status;
-  e = isoq::launch_decode(a, (cudaStream_t)stream);
-  return e == cudaSuccess ? ISOQ_OK : isoq::record_cuda_error(e);
+  return isoq::decode_run(params, cache, Q, q_dtype, n_seqs, 1, n_q_heads, seq_lens, max_seq_len,
+                          out, nullptr, scale, scratch, (size_t)ISOQ_NOALLOC_SCRATCH_BYTES,
+                          stream);
 }

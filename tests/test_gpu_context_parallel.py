@@ -136,3 +136,36 @@ def test_cp_decoder_over_a_one_rank_nccl_group(oracle, run2):
         check_attention(oracle, run2, Q, out, lens)
     finally:
         dist.destroy_process_group()
+
+
+def test_cp_decoder_on_a_side_stream(oracle, run2):
+    """The decoder given a stream other than the current one: the partial state, the
+    all-gather (NCCL, a group of one GPU) and the merge all run in order on that stream,
+    and the result equals the one on the current stream bitwise."""
+    import torch.distributed as dist
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1)
+    try:
+        Q = wl.queries(run2.cfg, device="cuda")
+        lens = run2.cfg.decode_lens()
+        sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        dec = ContextParallelDecoder(run2.params, run2.cache, Q.shape[0], Q.shape[1], max(lens))
+        ref = torch.empty((Q.shape[0], Q.shape[1], run2.cfg.d), dtype=torch.float32,
+                          device="cuda")
+        dec(Q, sl, ref, run2.cfg.scale)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        out = torch.full_like(ref, float("nan"))
+        dec.state.fill_(float("nan"))
+        junk = torch.empty((1 << 26,), device="cuda")
+        side.wait_stream(torch.cuda.current_stream())
+        # a long kernel on the side stream first, so a merge that ran ahead of the
+        # partial state or the gather would read stale data
+        with torch.cuda.stream(side):
+            junk.normal_()
+        dec(Q, sl, out, run2.cfg.scale, stream=side)
+        side.synchronize()
+        assert torch.equal(out, ref)
+        check_attention(oracle, run2, Q, out, lens)
+    finally:
+        dist.destroy_process_group()

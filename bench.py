@@ -34,6 +34,11 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0    # B200 HBM3e specification (context for the measured copy peak)
+# the headline metric, printed identically by both arms
+METRIC = "packed-KV decode attention GB/s (% of B200 HBM peak); quantize Mvec/s"
+# what the decode's contraction computes in (operands and accumulator)
+DECODE_DTYPE = "f16 operands (query as an f16 high+low pair), f32 accumulate"
 
 
 def _args():
@@ -45,7 +50,10 @@ def _args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="steps of the end-to-end timing (default: --steps)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload measurements of the other configurations")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the multi-token and context-parallel measurements")
     ap.add_argument("--chunk", type=int, default=16,
@@ -219,14 +227,16 @@ def oracle_sample(cfg, tokens: int = 4096, units: int = 1):
             "pairs": H * cfg.group, "tokens": tokens, "units": H}
 
 
-def cpu_baseline(cfg, budget_s: float = 12.0):
-    """Oracle decode GB/s (and quantize Mvec/s) on a bounded sample sized to ~budget_s."""
+def cpu_baseline(cfg, budget_s: float = 12.0, single_core_s: float = 3.0):
+    """Oracle decode GB/s (and quantize Mvec/s) on a bounded sample sized to ~budget_s on all
+    of the host's cores, and on one core with a sample sized to ~single_core_s."""
+    import oracle
     probe = oracle_sample(cfg, tokens=1024, units=1)
     per_tok = (probe["quant_s"] + probe["decode_s"]) / 1024
     tokens = int(max(1024, min(cfg.decode_lens()[0], budget_s / max(per_tok, 1e-9))))
     tokens = (tokens // 64) * 64
     r = oracle_sample(cfg, tokens=tokens, units=1)
-    return {
+    res = {
         "value": r["packed_bytes"] / r["decode_s"] / 1e9, "unit": "GB/s",
         "cores": min(r["threads"], r["pairs"]), "kind": "oracle",
         "quantize_mvec_s": r["vectors"] / r["quant_s"] / 1e6,
@@ -235,6 +245,21 @@ def cpu_baseline(cfg, budget_s: float = 12.0):
                    f"heads: oracle quantize ({r['vectors']} vectors) then decode "
                    f"({r['packed_bytes']} packed bytes)"),
     }
+    if single_core_s > 0:
+        threads = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            p1 = oracle_sample(cfg, tokens=256, units=1)
+            per1 = (p1["quant_s"] + p1["decode_s"]) / 256
+            t1 = int(max(256, min(cfg.decode_lens()[0], single_core_s / max(per1, 1e-9))))
+            r1 = oracle_sample(cfg, tokens=(t1 // 64) * 64 or 64, units=1)
+        finally:
+            oracle.set_num_threads(threads)
+        res["single_core"] = {
+            "value": r1["packed_bytes"] / r1["decode_s"] / 1e9, "unit": "GB/s", "cores": 1,
+            "quantize_mvec_s": r1["vectors"] / r1["quant_s"] / 1e6,
+            "sample": f"sequence 0, first {r1['tokens']} tokens, 1 KV head"}
+    return res
 
 
 def run_reference(args, cfg):
@@ -253,7 +278,7 @@ def run_reference(args, cfg):
     sample = (f"per step: sequence 0, first {tokens} tokens, 1 KV head x {rr['pairs']} query "
               f"heads; oracle quantize then decode")
     line = {
-        "impl": "reference", "metric": "packed-KV decode attention GB/s", "value": value,
+        "impl": "reference", "metric": METRIC, "value": value,
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": (dec + qt) / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -401,31 +426,33 @@ def run_ours(args, cfg):
             decode()
             hout.copy_(out, non_blocking=True)
 
+        e2e_steps = args.e2e_steps or args.steps
         e2e_step()
         torch.cuda.synchronize()
         a, b = ev(), ev()
         barrier()
         torch.cuda.synchronize()
         a.record(stream)
-        for _ in range(args.e2e_steps):
+        for _ in range(e2e_steps):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
         e_ms = rank_max(a.elapsed_time(b))
-        e2e = {"value": weak_scaling_rate(packed, args.e2e_steps, world, e_ms) / 1e9,
+        e2e = {"value": weak_scaling_rate(packed, e2e_steps, world, e_ms) / 1e9,
                "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
+               "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps,
                "what": "packed-KV bytes decoded per step / step time with the step's K, V and "
                        "Q copied from pinned host memory, quantize-append, decode and the "
                        "output copied back"}
 
     line = {
-        "metric": "packed-KV decode attention GB/s (% of B200 HBM peak); quantize Mvec/s",
+        "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": DECODE_DTYPE, "data": "synthetic",
+        "hbm_frac_of_spec": dec_gbs_1 / SPEC_HBM_GBS,
         "config": _config(cfg),
         "quantize": {"value": qval, "unit": "Mvec/s", "ms_per_step": q_ms / args.steps,
                      "roofline": {"bound": "hbm", "achieved": q_gbs_1, "peak": peak,
@@ -454,6 +481,14 @@ def run_ours(args, cfg):
                                              rank_max, peak, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
+    if not args.no_configs and not args.seqs:
+        line["configs"] = _bench_configs(
+            args, cfg, {"decode_GBps": dec_gbs_1, "decode_ms": dec_launch_ms,
+                        "quantize_Mvec_s": qval / world, "quantize_frac": q_gbs_1 / peak,
+                        "packed_bytes": packed, "vectors": n_vec,
+                        "oracle": line.get("cpu_baseline")},
+            flush, stream, rank_max, peak, peak_kind, dev,
+            oracle_ok=(rank == 0 and world == 1 and not args.no_cpu_baseline))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -629,6 +664,85 @@ def _bench_context_parallel(args, cfg, params, cache, layout, lens, Q, flush, st
     return {"value": gbs, "unit": "GB/s", "scaling": "strong", "ms_per_call": ms,
             "n_gpus": world, "state_bytes_per_rank": int(dec.state.numel() * 4),
             "roofline_frac_per_gpu": gbs / world / peak, "peak_kind": peak_kind}
+
+
+def _bench_configs(args, head_cfg, head, flush, stream, rank_max, peak, peak_kind, dev,
+                   oracle_ok: bool):
+    """Every workload of the configuration list on this GPU: the prefill quantised in its
+    chunked calls (Mvec/s), the appended tokens, one decode step of every sequence (mean of
+    10 calls, L2 flushed before each), the fraction of the measured and of the specified
+    HBM peak, and the oracle on a bounded sample of the same workload.  The headline
+    workload's numbers are the main measurement's."""
+    import torch
+
+    import rotated_bit_kv_isoquant_b200 as iq
+    import workloads as wl
+    res = {}
+    for idx in range(1, len(wl.WORKLOADS) + 1):
+        cfg = wl.workload(idx)
+        lens = cfg.decode_lens()
+        packed = sum(lens) * cfg.n_kv_heads * 2 * (3 * cfg.d // 8 + 2)
+        in_b = 4 if cfg.in_dtype == torch.float32 else 2
+        vec_bytes = cfg.d * in_b + 3 * cfg.d // 8 + 2
+        if idx == head_cfg.idx:
+            r = {"decode_GBps": head["decode_GBps"], "decode_ms": head["decode_ms"],
+                 "quantize_Mvec_s": head["quantize_Mvec_s"],
+                 "quantize_frac_measured": head["quantize_frac"],
+                 "packed_bytes": head["packed_bytes"], "quantize_vectors": head["vectors"],
+                 "oracle": head["oracle"], "source": "the main measurement"}
+        else:
+            params = iq.isoq_make_params(wl.PARAM_SEED, cfg.d, cfg.n_kv_heads)
+            layout = wl.page_layout(cfg)
+            cache = iq.PagedCache(cfg.d, cfg.n_kv_heads, layout.n_pages, layout.page_table,
+                                  device=dev)
+            q_ms, n_vec = 0.0, 0
+            for s, start, count in wl.prefill_calls(cfg):
+                K, V = wl.kv_tokens(cfg, s, start, count, device=dev)
+                sid = torch.full((count,), s, dtype=torch.int32, device=dev)
+                pos = torch.arange(start, start + count, dtype=torch.int32, device=dev)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                iq.isoq_quantize_append(params, cache, K, V, sid, pos, stream=stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+                q_ms += a.elapsed_time(b)
+                n_vec += 2 * cfg.n_kv_heads * count
+                del K, V
+            app = wl.append_kv(cfg, device=dev)
+            app_us = None
+            if app[0].shape[0]:
+                fn_app = lambda: iq.isoq_quantize_append(params, cache, *app, stream=stream)
+                app_us = rank_max(_time_calls(fn_app, flush, stream, iters=10)) * 1e3
+            Q = wl.queries(cfg, device=dev)
+            sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+            out = torch.empty((cfg.n_seqs, cfg.n_q_heads, cfg.d), dtype=torch.float32, device=dev)
+            nb = iq.isoq_decode_workspace_bytes(cfg.n_seqs, cfg.n_q_heads, cfg.n_kv_heads,
+                                                cfg.d, max(lens))
+            ws = torch.empty((max(nb, 16),), dtype=torch.uint8, device=dev)
+            fn = lambda: iq.isoq_decode_attention(params, cache, Q, sl, max(lens), out,
+                                                  cfg.scale, ws, stream=stream)
+            d_ms = rank_max(_time_calls(fn, flush, stream, iters=10, warmup=3))
+            assert iq.isoq_get_status(cache) == 0, f"status bits set on workload {idx}"
+            q_ms = rank_max(q_ms)
+            r = {"decode_GBps": packed / (d_ms / 1e3) / 1e9, "decode_ms": d_ms,
+                 "quantize_Mvec_s": n_vec / (q_ms / 1e3) / 1e6,
+                 "quantize_frac_measured": n_vec * vec_bytes / (q_ms / 1e3) / 1e9 / peak,
+                 "packed_bytes": packed, "quantize_vectors": n_vec,
+                 "decode_splits": iq.isoq_decode_num_splits(cfg.n_seqs, cfg.n_q_heads,
+                                                            cfg.n_kv_heads, cfg.d, max(lens))}
+            if app_us is not None:
+                r["append_us"] = app_us
+                r["append_vectors"] = 2 * cfg.n_kv_heads * app[0].shape[0]
+            r["oracle"] = cpu_baseline(cfg, budget_s=2.5, single_core_s=1.5) if oracle_ok else None
+            del cache, params, Q, out, ws
+            torch.cuda.empty_cache()
+        r["decode_frac_measured"] = r["decode_GBps"] / peak
+        r["decode_frac_spec"] = r["decode_GBps"] / SPEC_HBM_GBS
+        r["context"] = max(lens)
+        r["target_applies"] = max(lens) >= 32768     # >= 0.70 of the HBM peak at 32k+ contexts
+        res[cfg.name] = r
+    res["peak"] = {"measured_GBps": peak, "kind": peak_kind, "spec_GBps": SPEC_HBM_GBS}
+    return res
 
 
 def main():

@@ -61,6 +61,8 @@ def _declare(L):
     L.ref_threshold.restype = _d
     L.ref_threshold.argtypes = [_i]
     L.ref_num_threads.restype = _i
+    L.ref_set_num_threads.restype = None
+    L.ref_set_num_threads.argtypes = [_i]
     L.ref_splitmix64_next.restype = ctypes.c_uint64
     L.ref_splitmix64_next.argtypes = [_p]
     L.ref_normal.restype = _d
@@ -170,6 +172,11 @@ def thresholds(bits: int = 3) -> np.ndarray:
 
 def num_threads() -> int:
     return int(lib().ref_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops from now on (timing only)."""
+    lib().ref_set_num_threads(int(n))
 
 
 # ------------------------------------------------------------------------------------

@@ -82,6 +82,16 @@ int ref_num_threads(void) {
 #endif
 }
 
+/* Thread count of the parallel loops that follow (timing only: every loop's iterations
+ * are independent, so the results do not depend on it). */
+void ref_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------------ */
 /* Random rotation parameters.                                                      */
 /* SplitMix64: G. Steele, D. Lea, C. Flood, "Fast splittable pseudorandom number   */

@@ -99,10 +99,17 @@ def test_config4_batched_paged(oracle):
     sv = check_codes(oracle, p64, V.float().cpu().numpy().astype(np.float64), vc, vn, cfg.d)
     _log("cfg4_codes_appended", {k: sk[k] + sv[k] for k in sk})
     Q, out = run.decode()
-    sel = [(int(s), int(h)) for s, h in zip(rng.integers(0, cfg.n_seqs, 16),
-                                            rng.integers(0, cfg.n_q_heads, 16))]
-    sel += [(int(np.argmax(cfg.decode_lens())), 0), (int(np.argmin(cfg.decode_lens())), 31)]
-    _log("cfg4_attention_sampled", check_attention(oracle, run, Q, out, cfg.decode_lens(), sel))
+    # every KV head (and so every head's rotation parameters) for the shortest, the longest
+    # and a dozen random sequences; the query head inside the group varies
+    lens = cfg.decode_lens()
+    seqs4 = [int(np.argmin(lens)), int(np.argmax(lens))]
+    seqs4 += [int(x) for x in rng.choice([i for i in range(cfg.n_seqs) if i not in seqs4], 12,
+                                         replace=False)]
+    sel = [(s, kv * cfg.group + (s + kv) % cfg.group) for s in seqs4
+           for kv in range(cfg.n_kv_heads)]
+    stats = check_attention(oracle, run, Q, out, lens, sel)
+    assert stats["pairs"] == 14 * cfg.n_kv_heads
+    _log("cfg4_attention_every_kv_head", stats)
     assert iq.isoq_get_status(run.cache) == 0
 
 
@@ -114,8 +121,12 @@ def test_config5_long_context(oracle):
     seqs, p = _sample_tokens(cfg, 64, rng)
     _log("cfg5_codes_sampled", _codes_all(oracle, run, seqs, p))
     Q, out = run.decode()
-    sel = [(s, h) for s in range(cfg.n_seqs) for h in (0, 37)]
-    _log("cfg5_attention_sampled", check_attention(oracle, run, Q, out, cfg.decode_lens(), sel))
+    # one query head of every KV head, for every sequence (the head inside the group varies)
+    sel = [(s, kv * cfg.group + (s + kv) % cfg.group) for s in range(cfg.n_seqs)
+           for kv in range(cfg.n_kv_heads)]
+    stats = check_attention(oracle, run, Q, out, cfg.decode_lens(), sel)
+    assert stats["pairs"] == cfg.n_seqs * cfg.n_kv_heads
+    _log("cfg5_attention_every_kv_head", stats)
     assert torch.isfinite(out).all()
     assert iq.isoq_get_status(run.cache) == 0
 

@@ -143,6 +143,12 @@ def _declare(L):
     L.ref_quantize_rows_v.argtypes = [_i, _i, _p, _i, _i, _p, _i, _p, _p, _p]
     L.ref_unpack_codes_batch_v.restype = None
     L.ref_unpack_codes_batch_v.argtypes = [_i, _p, _i, ctypes.c_long, _p]
+    L.ref_v_put_codes.restype = None
+    L.ref_v_put_codes.argtypes = [_i, _i, _i, _p, _i, _p]
+    L.ref_v_get_codes.restype = None
+    L.ref_v_get_codes.argtypes = [_i, _i, _i, _p, _i, _p]
+    L.ref_v_region_records.restype = None
+    L.ref_v_region_records.argtypes = [_i, _i, _i, _p, _p]
 
 
 def _ptr(a: np.ndarray):
@@ -330,6 +336,34 @@ def unpack_codes(packed, d: int, bits: int = 3) -> np.ndarray:
     codes = np.zeros(d, dtype=np.uint8)
     lib().ref_unpack_codes_v(bits, _ptr(packed), d, _ptr(codes))
     return codes
+
+
+def v_put_codes(region, slot: int, codes, bits: int = 3, page: int = 64) -> None:
+    """Write one slot's V codes into a page's V region (uint8, modified in place): the 3-bit
+    V tile layout, or the slot's record at 2 and 4 bits."""
+    assert region.dtype == np.uint8 and region.flags.c_contiguous
+    codes = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    lib().ref_v_put_codes(bits, codes.shape[0], page, _ptr(region), int(slot), _ptr(codes))
+
+
+def v_get_codes(region, slot: int, d: int, bits: int = 3, page: int = 64) -> np.ndarray:
+    region = np.ascontiguousarray(np.asarray(region, dtype=np.uint8))
+    codes = np.zeros(d, np.uint8)
+    lib().ref_v_get_codes(bits, d, page, _ptr(region), int(slot), _ptr(codes))
+    return codes
+
+
+def v_region_records(regions, d: int, bits: int = 3, page: int = 64) -> np.ndarray:
+    """V regions [..., page * bits*d/8] -> per-slot records [..., page, bits*d/8] in the
+    record packing of pack_codes."""
+    regions = np.ascontiguousarray(np.asarray(regions, dtype=np.uint8))
+    cb = bits * d // 8
+    lead = regions.shape[:-1]
+    flat = regions.reshape(-1, page * cb)
+    out = np.zeros((flat.shape[0], page, cb), np.uint8)
+    for i in range(flat.shape[0]):
+        lib().ref_v_region_records(bits, d, page, _ptr(flat[i]), _ptr(out[i]))
+    return out.reshape(lead + (page, cb))
 
 
 def block_bytes(d: int, page: int = 64, bits: int = 3) -> int:

@@ -464,7 +464,9 @@ void ref_unpack_codes(const uint8_t *in, int d, uint8_t *codes) { ref_unpack_cod
 /* ------------------------------------------------------------------------------ */
 /* Paged cache: blocks[page][kv_head] of block_bytes; a block holds, for 64 (page)  */
 /* token slots: K codes [P][cb] | K norms [P] binary16 | V codes | V norms, with     */
-/* cb = bits * d / 8 code bytes per vector.                                          */
+/* cb = bits * d / 8 code bytes per vector.  K codes are one record per slot (the    */
+/* packing above).  V codes: one record per slot at 2 and 4 bits; at 3 bits the V    */
+/* tile layout below.                                                                */
 /* ------------------------------------------------------------------------------ */
 static size_t cbytes(int bits, int d) { return (size_t)bits * d / 8; }
 
@@ -473,11 +475,104 @@ size_t ref_block_bytes(int d, int page) { return ref_block_bytes_v(3, d, page); 
 
 static size_t k_codes_off(size_t cb, int page, int slot) { (void)page; return (size_t)slot * cb; }
 static size_t k_norm_off(size_t cb, int page, int slot) { return (size_t)page * cb + 2 * (size_t)slot; }
-static size_t v_codes_off(size_t cb, int page, int slot) {
-  return (size_t)page * (cb + 2) + (size_t)slot * cb;
-}
+static size_t v_region_off(size_t cb, int page) { return (size_t)page * (cb + 2); }
 static size_t v_norm_off(size_t cb, int page, int slot) {
   return (size_t)page * (cb + 2) + (size_t)page * cb + 2 * (size_t)slot;
+}
+
+/* ------------------------------------------------------------------------------ */
+/* 3-bit V tile layout (this build's format; the pages fix none).  The V region of  */
+/* a page is 4 blocks of 16 token slots, 6 d bytes each.  Inside block B the 16     */
+/* slots form 4 quads: quad t (0..3) = slots 16B + 2t + {0, 1, 8, 9}, its member j   */
+/* (0..3) being slot 16B + 2t + (j & 1) + 8 (j >> 1).  Dims form units of 8          */
+/* (unit u = dims 8u .. 8u+7).  The 12-byte group of (quad t, unit u) sits at byte   */
+/* ((u >> 1) * 8 + 2 t + (u & 1)) * 12 of the block and holds three little-endian   */
+/* words W0, W1, W2:                                                                 */
+/*   bits 4n .. 4n+2 of W_b hold the code of member (n & 3), dim 8u + 2b + (n >> 2)   */
+/*   (nibbles 0-3: dim 8u+2b of the four members; nibbles 4-7: dim 8u+2b+1);        */
+/*   bit 4n + 3 of W_b holds bit (2 - b) of the code of member (n & 3),               */
+/*   dim 8u + 6 + (n >> 2).                                                          */
+/* So each 16-bit half of a word is four members' codes of one dim: a decoder can    */
+/* turn it into the values of four tokens of one dimension with byte permutes.       */
+/* ------------------------------------------------------------------------------ */
+static void v3_locate(int d, int slot, int dim, size_t *group, int *nib, int *spare) {
+  int B = slot >> 4, r = slot & 15;
+  int t = (r >> 1) & 3, j = (r & 1) | ((r >> 3) << 1);
+  int u = dim >> 3, e = dim & 7;
+  *group = (size_t)B * 6 * d + (size_t)(((u >> 1) * 8 + 2 * t + (u & 1)) * 12);
+  *spare = e >= 6;
+  *nib = *spare ? j + 4 * (e - 6) : j + 4 * (e & 1);
+  if (!*spare) *group += 4 * (size_t)(e >> 1); /* word b = e / 2 */
+}
+
+static void put_bit(uint8_t *base, size_t byte, int bit, int v) {
+  if (v) base[byte] |= (uint8_t)(1u << bit);
+  else base[byte] &= (uint8_t)~(1u << bit);
+}
+
+static int get_bit(const uint8_t *base, size_t byte, int bit) { return (base[byte] >> bit) & 1; }
+
+/* The codes of one slot into / out of a V region (3 bits: the tile layout; 2 and 4 bits:
+ * the slot's record). */
+void ref_v_put_codes(int bits, int d, int page, uint8_t *region, int slot, const uint8_t *codes) {
+  if (bits != 3) {
+    ref_pack_codes_v(bits, codes, d, region + (size_t)slot * cbytes(bits, d));
+    return;
+  }
+  (void)page;
+  for (int i = 0; i < d; i++) {
+    size_t g;
+    int n, sp;
+    v3_locate(d, slot, i, &g, &n, &sp);
+    unsigned c = codes[i] & 7u;
+    if (!sp) {
+      for (int k = 0; k < 3; k++) {
+        size_t bit = 4 * (size_t)n + k;
+        put_bit(region, g + bit / 8, (int)(bit % 8), (c >> k) & 1);
+      }
+    } else {
+      for (int b = 0; b < 3; b++) {
+        size_t bit = 4 * (size_t)n + 3;
+        put_bit(region, g + 4 * (size_t)b + bit / 8, (int)(bit % 8), (c >> (2 - b)) & 1);
+      }
+    }
+  }
+}
+
+void ref_v_get_codes(int bits, int d, int page, const uint8_t *region, int slot, uint8_t *codes) {
+  if (bits != 3) {
+    ref_unpack_codes_v(bits, region + (size_t)slot * cbytes(bits, d), d, codes);
+    return;
+  }
+  (void)page;
+  for (int i = 0; i < d; i++) {
+    size_t g;
+    int n, sp;
+    v3_locate(d, slot, i, &g, &n, &sp);
+    unsigned c = 0;
+    if (!sp) {
+      for (int k = 0; k < 3; k++) {
+        size_t bit = 4 * (size_t)n + k;
+        c |= (unsigned)get_bit(region, g + bit / 8, (int)(bit % 8)) << k;
+      }
+    } else {
+      for (int b = 0; b < 3; b++) {
+        size_t bit = 4 * (size_t)n + 3;
+        c |= (unsigned)get_bit(region, g + 4 * (size_t)b + bit / 8, (int)(bit % 8)) << (2 - b);
+      }
+    }
+    codes[i] = (uint8_t)c;
+  }
+}
+
+/* A page's V region as per-slot records in the K record packing (tests compare GPU and
+ * oracle codes record by record): records [page][cb]. */
+void ref_v_region_records(int bits, int d, int page, const uint8_t *region, uint8_t *records) {
+  uint8_t codes[1024];
+  for (int s = 0; s < page; s++) {
+    ref_v_get_codes(bits, d, page, region, s, codes);
+    ref_pack_codes_v(bits, codes, d, records + (size_t)s * cbytes(bits, d));
+  }
 }
 
 /* Quantise n_tokens tokens of K and V ([n_tokens][n_kv_heads][d], fp64) into the paged
@@ -503,8 +598,10 @@ int ref_quantize_append_v(int bits, int rot, const double *params, int d, int n_
         const double *x = (kv == 0 ? K : V) + ((size_t)t * n_kv_heads + h) * d;
         uint16_t n16;
         overflow += ref_quantize_vector_v(bits, rot, ph, x, d, codes, &n16, NULL);
-        uint8_t *dst = blk + (kv == 0 ? k_codes_off(cb, page, slot) : v_codes_off(cb, page, slot));
-        ref_pack_codes_v(bits, codes, d, dst);
+        if (kv == 0)
+          ref_pack_codes_v(bits, codes, d, blk + k_codes_off(cb, page, slot));
+        else
+          ref_v_put_codes(bits, d, page, blk + v_region_off(cb, page), slot, codes);
         uint8_t *nd = blk + (kv == 0 ? k_norm_off(cb, page, slot) : v_norm_off(cb, page, slot));
         nd[0] = (uint8_t)(n16 & 0xff);
         nd[1] = (uint8_t)(n16 >> 8);
@@ -523,14 +620,26 @@ int ref_quantize_append(const double *params, int d, int n_kv_heads, int page,
 }
 
 /* Dequantised vector in the rotated space: (stored norm / sqrt(d)) * level[code]. */
-static void dequant_rotated(int bits, const uint8_t *packed, const uint8_t *norm_bytes, int d,
-                            double *out) {
-  uint8_t codes[1024];
-  ref_unpack_codes_v(bits, packed, d, codes);
+static void dequant_codes(int bits, const uint8_t *codes, const uint8_t *norm_bytes, int d,
+                          double *out) {
   uint16_t n16 = (uint16_t)(norm_bytes[0] | (norm_bytes[1] << 8));
   double s = ref_fp16_value(n16) / sqrt((double)d);
   const double *L = levels_of(bits);
   for (int i = 0; i < d; i++) out[i] = s * L[codes[i]];
+}
+
+/* Slot `slot` of a block: K (kind 0) or V (kind 1) dequantised in the rotated space. */
+static void dequant_slot(int bits, int d, int page, const uint8_t *blk, int slot, int kind,
+                         double *out) {
+  size_t cb = cbytes(bits, d);
+  uint8_t codes[1024];
+  if (kind == 0) {
+    ref_unpack_codes_v(bits, blk + k_codes_off(cb, page, slot), d, codes);
+    dequant_codes(bits, codes, blk + k_norm_off(cb, page, slot), d, out);
+  } else {
+    ref_v_get_codes(bits, d, page, blk + v_region_off(cb, page), slot, codes);
+    dequant_codes(bits, codes, blk + v_norm_off(cb, page, slot), d, out);
+  }
 }
 
 /* Materialise one cached vector back in the input space (K-hat or V-hat): inverse
@@ -539,13 +648,10 @@ static void dequant_rotated(int bits, const uint8_t *packed, const uint8_t *norm
 void ref_dequantize_slot_v(int bits, int rot, const double *params, int d, int n_kv_heads,
                            int page, const uint8_t *blocks, int phys_page, int kv_head, int slot,
                            int kind, double *out) {
-  size_t bb = ref_block_bytes_v(bits, d, page), cb = cbytes(bits, d);
+  size_t bb = ref_block_bytes_v(bits, d, page);
   const uint8_t *blk = blocks + ((size_t)phys_page * n_kv_heads + kv_head) * bb;
   double zr[1024];
-  if (kind == 0)
-    dequant_rotated(bits, blk + k_codes_off(cb, page, slot), blk + k_norm_off(cb, page, slot), d, zr);
-  else
-    dequant_rotated(bits, blk + v_codes_off(cb, page, slot), blk + v_norm_off(cb, page, slot), d, zr);
+  dequant_slot(bits, d, page, blk, slot, kind, zr);
   ref_unrotate_v(rot, params + (size_t)kv_head * ref_params_per_head(rot, d), zr, out, d);
 }
 
@@ -572,7 +678,7 @@ void ref_decode_attention_v(int bits, int rot, const double *params, int d, int 
                             const int32_t *seq_lens, const double *Q, double scale, double *out,
                             const int32_t *sel, int n_sel) {
   int G = n_q_heads / n_kv_heads;
-  size_t bb = ref_block_bytes_v(bits, d, page), cb = cbytes(bits, d);
+  size_t bb = ref_block_bytes_v(bits, d, page);
   int pph = ref_params_per_head(rot, d);
   int total = sel ? n_sel : n_seqs * n_q_heads;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -594,8 +700,7 @@ void ref_decode_attention_v(int bits, int rot, const double *params, int d, int 
     for (int t = 0; t < len; t++) {
       int phys = page_table[(size_t)s * max_pages_per_seq + t / page];
       const uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + kvh) * bb;
-      dequant_rotated(bits, blk + k_codes_off(cb, page, t % page),
-                      blk + k_norm_off(cb, page, t % page), d, kt);
+      dequant_slot(bits, d, page, blk, t % page, 0, kt);
       double dot = 0.0;
       for (int i = 0; i < d; i++) dot += qt[i] * kt[i];
       sc[t] = scale * dot;
@@ -610,8 +715,7 @@ void ref_decode_attention_v(int bits, int rot, const double *params, int d, int 
       l += p;
       int phys = page_table[(size_t)s * max_pages_per_seq + t / page];
       const uint8_t *blk = blocks + ((size_t)phys * n_kv_heads + kvh) * bb;
-      dequant_rotated(bits, blk + v_codes_off(cb, page, t % page),
-                      blk + v_norm_off(cb, page, t % page), d, vt);
+      dequant_slot(bits, d, page, blk, t % page, 1, vt);
       for (int i = 0; i < d; i++) ot[i] += p * vt[i];
     }
     for (int i = 0; i < d; i++) ot[i] /= l;

@@ -92,12 +92,21 @@ def gather_records(cache: iq.PagedCache, page_table: torch.Tensor, seqs, positio
         return cache.blocks[phys[:, None, None], hh[None, :, None], col[:, None, :]]
 
     kc = take(slot[:, None] * cb + ar)
-    vc = take(v_codes_off + slot[:, None] * cb + ar)
+    if bits == 3:
+        # 3-bit V codes use the V tile layout: fetch the V regions of the pages involved
+        # and let the oracle turn them into per-slot records
+        import oracle
+        uniq, inv = torch.unique(phys, return_inverse=True)
+        reg = cache.blocks[uniq][:, :, v_codes_off:v_codes_off + 64 * cb]
+        rec = oracle.v_region_records(reg.cpu().numpy(), d, bits=bits)   # [U][H][64][cb]
+        vc = rec[inv.cpu().numpy()[:, None], np.arange(H)[None, :], slot.cpu().numpy()[:, None]]
+    else:
+        vc = take(v_codes_off + slot[:, None] * cb + ar).cpu().numpy()
     two = torch.arange(2, device=dev)
     kn = take(k_norm_off + 2 * slot[:, None] + two)
     vn = take(v_norm_off + 2 * slot[:, None] + two)
     to16 = lambda t: t.cpu().numpy().copy().view(np.uint16)[..., 0]
-    return kc.cpu().numpy(), to16(kn), vc.cpu().numpy(), to16(vn)
+    return kc.cpu().numpy(), to16(kn), vc, to16(vn)
 
 
 def check_codes(oracle, params64, X, gpu_codes_packed, gpu_norms, d, bits: int = 3, rot: int = 0):

@@ -153,13 +153,23 @@ size_t isoq_block_bytes_v(int d, int bits, int page_size);
  *
  * blocks: device uint8 [n_pages][n_kv_heads][isoq_block_bytes(d, 64)].  One block holds
  * one KV head of one 64-token page:
- *     K codes [64][3d/8] | K norms [64] binary16 | V codes [64][3d/8] | V norms [64] binary16
+ *     K codes [64][3d/8] | K norms [64] binary16 | V codes (64 * 3d/8 bytes) | V norms [64]
  * (6400 bytes at d = 128, 12544 at d = 256; both multiples of 16).
  *
- * Codes of one vector (3 bits each, 3d/8 bytes): d/32 groups of 12 bytes; group g covers
+ * K codes of one slot (3 bits each, 3d/8 bytes): d/32 groups of 12 bytes; group g covers
  * dims 32g..32g+31 and is three little-endian 32-bit words w0, w1, w2:
  *     dim 32g + 8j + k (j = 0,1,2; k = 0..7): the code is bits 4k..4k+2 of w_j;
  *     dim 32g + 24 + k (k = 0..7): bit (2 - b) of the code is bit 4k+3 of w_b.
+ * 3-bit V codes of a page ("V tile layout"): 4 blocks of 16 slots, 6d bytes each.  In
+ * block B, quad t (0..3) is the slots 16B + 2t + {0, 1, 8, 9}, member j of the quad being
+ * slot 16B + 2t + (j & 1) + 8 (j >> 1); unit u is dims 8u..8u+7.  The 12-byte group of
+ * (quad t, unit u) starts at byte ((u >> 1) * 8 + 2t + (u & 1)) * 12 of the block and is
+ * three little-endian words W0, W1, W2:
+ *     bits 4n..4n+2 of W_b: the code of member n & 3 at dim 8u + 2b + (n >> 2);
+ *     bit 4n+3 of W_b: bit (2 - b) of the code of member n & 3 at dim 8u + 6 + (n >> 2)
+ * (n = 0..7).  Each 16-bit half of a word is thus four tokens' codes of one dim, the
+ * operand shape of the decode's value product.  At 2 and 4 bits V codes are one record
+ * per slot, like K.
  * A code c in 0..7 indexes the ascending levels
  *     L = {-2.1520, -1.3440, -0.7560, -0.2451, 0.2451, 0.7560, 1.3440, 2.1520}
  * (the 8-level Lloyd-Max quantiser for N(0,1), J. Max 1960), and stands for the rotated

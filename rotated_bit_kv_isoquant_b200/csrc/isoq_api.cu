@@ -111,8 +111,9 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
   // the multi-token kernels (64 or 128 rows per CTA, 2 CTAs per SM) when a chunk gives a
   // KV head at least 16 rows; else the per-row kernel (8 rows per CTA)
   const bool shared_mq = d == 128 && n_q > 1 && (long long)n_q * group >= 16;
-  const int n_sm = sm_count() * (shared_mq ? 2 : isoq::decode_resident_ctas(d));
-  const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group) : 8;
+  const int n_sm = sm_count() * (shared_mq ? 2 : isoq::decode_i8_resident_ctas(d));
+  const int rows_per_cta = shared_mq ? isoq::attention_rows_per_cta(d, n_q, group)
+                                     : isoq::decode_rows_per_block(d, n_q, group);
   // pages per CTA worth a launch: the tensor-memory kernel rotates 128 queries per CTA
   const int min_pages = shared_mq ? (rows_per_cta == 128 ? 16 : 4) : ISOQ_DEC_MIN_PAGES;
   const int max_pages = max_seq_len > 0 ? (max_seq_len + ISOQ_PAGE_SIZE - 1) / ISOQ_PAGE_SIZE : 1;
@@ -125,6 +126,7 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
   if (want < 1) want = 1;
   int pps = (int)((max_pages + want - 1) / want);
   if (pps < 1) pps = 1;
+  if (pps > isoq::kMaxPagesPerSplit) pps = isoq::kMaxPagesPerSplit;
   int n_splits = (max_pages + pps - 1) / pps;
   return SplitPlan{n_splits, pps};
 }

@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(128)
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = use_shared_mq(a) ? launch_decode_split_mq(a, stream)
+                  : a.bits == 3    ? launch_decode_split_i8(a, stream)
                                    : launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
   const int rows = a.n_q * a.n_q_heads;

@@ -1,0 +1,664 @@
+// Decode attention on the packed 3-bit cache with 8-bit integer tensor-core products
+// (split-K partials).
+//
+// Method: "RotaryQuant: Fitting 120B MoE Models on Consumer Hardware via Fused
+// Compressed-Space Attention", Abstract: attention is computed directly on the packed
+// 3-bit codes and full-precision K/V are never rebuilt.  With R orthogonal,
+// q.k_hat = (R q).(R k_hat), so the rows' queries are rotated once per CTA and the scores
+// and the value sum run on codebook levels in the rotated space.
+//
+// Scores in exact integer arithmetic.  The levels are 4-decimal numbers, so 10000 L[c] is
+// an exact 16-bit integer, split into two signed bytes kh * 256 + kl.  Each thread turns a
+// 16-bit half of a packed word (four 3-bit codes) into four such bytes with one byte
+// permute against an 8-entry table of the levels' high bytes and one against their low
+// bytes: two permutes per four keys, the operand of an int8 mma.sync as it is.  The
+// rotated query of a row is scaled to a 24-bit integer (8e6 / max|q~|) and split into
+// three balanced signed bytes d2 d1 d0, so a score is
+//   2^24 d2.kh + 2^16 (d2.kl + d1.kh) + 2^8 (d1.kl + d0.kh)   (+ d0.kl, below 2^-23 of it)
+// from s8 x s8 -> s32 products that are exact; the query's rounding (relative 1e-7) is
+// the only error before the binary32 softmax.
+// Values in f16.  The value weights P' = p nV / sigma (lazily rescaled running maximum and
+// V-norm reference) span many binades, which a fixed-point operand would cut short, so the
+// value product keeps f16 operands with f32 accumulators: V_hat^T from byte permutes of
+// f16 level bytes (ALPHA times the levels, < 2e-5 relative error), P' as f16.
+//
+// Work: one CTA of 4 warps per (context chunk, KV head, block of RB rows, sequence); a
+// row is a (query token, query head) pair.  Each warp streams its own pages of the chunk
+// through a private ring of shared-memory stages filled by 1-D bulk copies (one page
+// block per copy, completion on an mbarrier, every wait bounded).  Per 32-token tile:
+//   scores  C[16 x 8 tokens] = A[16 x 32 dims] . K_hat^T, m16n8k32 s8, 4 tiles of 8 tokens:
+//           RB = 8: A = [d2; d1] against kh and kl, [d0; 0] against kh (3 mma per k-step);
+//           RB = 4: A = [d2; d1; d0; 0] against kh, [d2; d1; 0; 0] against kl (2 mma).
+//           Lane t of a quad owns 32-dim group t of every token (the k order inside a
+//           k-step is a permutation of the dims, the query digits follow it).
+//   online softmax per row, rescaled only when a running maximum grows (lazy), so the
+//           common tile needs no shuffles
+//   values  O^T[16 dims x 8 rows] += V_hat^T[16 x 16 tokens] . P'^T, m16n8k16 f16 per
+//           16-token block: the score tile's columns 2t, 2t+1 of two 8-token tiles are
+//           exactly the k slots 2t, 2t+1, 2t+8, 2t+9 of the value product, and the V tile
+//           layout stores those four tokens' codes of one dim as the four nibbles of a
+//           16-bit half-word: two level-byte lookups and two interleaves give the A
+//           registers of two k slots each, with no cross-token merging.
+#include <math_constants.h>
+
+#include <type_traits>
+
+#include "isoq_common.cuh"
+#include "isoq_internal.h"
+#include "isoq_ptx.cuh"
+#include "isoq_vtile.cuh"
+
+namespace isoq {
+using namespace ptx;
+namespace {
+
+constexpr float kQMax = 8.0e6f;       // |24-bit query integer| bound (digits stay in s8)
+constexpr float kLevelScale = 1.0e4f; // integer levels: 10000 L[c]
+
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Integer level 10000 L[c] = kh * 256 + kl with kl in [-128, 127], kh = floor((v + 128) / 256).
+__host__ __device__ constexpr int ilevel(int c) {
+  return c == 0 ? -21520 : c == 1 ? -13440 : c == 2 ? -7560 : c == 3 ? -2451
+       : c == 4 ? 2451 : c == 5 ? 7560 : c == 6 ? 13440 : 21520;
+}
+__host__ __device__ constexpr int ilevel_hi(int c) {
+  return (ilevel(c) + 128 >= 0) ? (ilevel(c) + 128) / 256 : -((-(ilevel(c) + 128) + 255) / 256);
+}
+__host__ __device__ constexpr int ilevel_lo(int c) { return ilevel(c) - 256 * ilevel_hi(c); }
+__host__ __device__ constexpr uint32_t level_bytes(bool hi, int c0) {
+  uint32_t w = 0;
+  for (int k = 0; k < 4; ++k)
+    w |= (uint32_t)((hi ? ilevel_hi(c0 + k) : ilevel_lo(c0 + k)) & 0xff) << (8 * k);
+  return w;
+}
+static_assert(ilevel_hi(2) * 256 + ilevel_lo(2) == -7560 && ilevel_lo(1) == -128 &&
+                  ilevel_lo(6) == -128 && ilevel_hi(7) == 84 && ilevel_lo(7) == 16,
+              "integer level split");
+constexpr uint32_t kTH0 = level_bytes(true, 0), kTH1 = level_bytes(true, 4);
+constexpr uint32_t kTL0 = level_bytes(false, 0), kTL1 = level_bytes(false, 4);
+
+// Balanced base-256 digits of a 24-bit integer: q = d2 * 65536 + d1 * 256 + d0.
+__device__ __forceinline__ void digits3(int q, int& d2, int& d1, int& d0) {
+  d0 = ((q + 128) & 255) - 128;
+  const int r = (q - d0) >> 8;
+  d1 = ((r + 128) & 255) - 128;
+  d2 = (r - d1) >> 8;
+}
+
+__device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 255) | ((uint32_t)(b & 255) << 8) | ((uint32_t)(c & 255) << 16) |
+         ((uint32_t)(d & 255) << 24);
+}
+
+// Shared memory: [kWarps][NST] page stages, the mbarriers, the score mma's A fragments
+// (A1: 4 words per k-step and lane, 16-byte aligned; RB = 8 also A2: 2 words, 8-byte
+// aligned), per-row score factors, output row indices.  The stage area is reused for the
+// final merge.
+template <int D, int NST, int RB>
+struct I8Smem {
+  static constexpr int kStageBytes = block_bytes(D, 3);
+  static constexpr int kRing = kWarps * NST * kStageBytes;
+  static constexpr int kBarOff = kRing;
+  static constexpr int kAOff = kBarOff + kWarps * NST * 8;             // uint4 [D/32][32]
+  static constexpr int kA2Off = kAOff + (D / 32) * 32 * 16;            // uint2 [D/32][32]
+  static constexpr int kKfOff = kA2Off + (RB == 8 ? (D / 32) * 32 * 8 : 0);  // float [8]
+  static constexpr int kRowOff = kKfOff + 8 * 4;                      // int [8]
+  static constexpr int kBytes = kRowOff + 8 * 4;
+  static constexpr int kMergeBytes = kWarps * 8 * (D + 4) * 4;
+  static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
+  static_assert(kAOff % 16 == 0 && kA2Off % 8 == 0, "A fragments must be aligned");
+};
+
+template <int D>
+constexpr int i8_min_blocks() { return D == 128 ? 3 : 2; }
+
+// MQ: chunks of several query tokens per sequence with causal limits; the decode (one
+// query token, every row attending the whole context) is compiled without them.
+template <int D, int NST, int RB, typename TQ, bool MQ>
+__global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
+    decode_i8_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
+                     const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
+                     const TQ* __restrict__ Q, int n_q_heads, int n_q,
+                     const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
+                     int n_splits, float* __restrict__ partials, uint32_t* status) {
+  using SM = I8Smem<D, NST, RB>;
+  constexpr int E = D / 32;           // elements per lane in the warp WHT layout
+  constexpr int NB = E / 4;
+  constexpr int CB = code_bytes(D, 3);
+  constexpr int BB = block_bytes(D, 3);
+  constexpr int NG = D / 128;         // 32-dim groups per lane and token (groups t, t + 4)
+  constexpr int NU = D / 128;         // unit pairs per lane in the V tile (g, g + 8)
+  constexpr int MT = 8 * NU;          // m-tiles of the value product
+  constexpr int PS = D + 4;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
+  uint32_t* afr = reinterpret_cast<uint32_t*>(smem + SM::kAOff);    // [D/32][32][4]
+  uint32_t* afr2 = reinterpret_cast<uint32_t*>(smem + SM::kA2Off);  // [D/32][32][2] (RB = 8)
+  float* kf_row = reinterpret_cast<float*>(smem + SM::kKfOff);
+  int* row_off = reinterpret_cast<int*>(smem + SM::kRowOff);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int split = blockIdx.x, s = blockIdx.z;
+  // The CTA's RB rows are (query token i, query head) pairs of KV head hk: row r is pair
+  // R = RB rb + r of the group's n_q * G pairs, i = R / G, head hk * G + R % G.  Query
+  // token i of a sequence of len tokens sits at position len - n_q + i and attends the
+  // tokens before and at it (n_q = 1: the decode, every row attends the whole context).
+  if constexpr (!MQ) n_q = 1;
+  const int G = n_q_heads / H;
+  const int n_rows = n_q * G;
+  const int nrb = (n_rows + RB - 1) / RB;
+  const int hk = blockIdx.y / nrb, rb = blockIdx.y - hk * nrb;
+  const int nh = min(RB, n_rows - rb * RB);      // rows handled here
+  const int rg = RB == 8 ? g : (g & 3);           // this lane's score row
+  auto row_token = [&](int r) { return (rb * RB + r) / G; };
+  auto row_index = [&](int r) {                   // row of the sequence's output / partials
+    const int R = rb * RB + r;
+    return (R / G) * n_q_heads + hk * G + R % G;
+  };
+
+  int len = __ldg(seq_lens + s);
+  if (len > max_pages * kPage) {
+    if (tid == 0 && split == 0 && blockIdx.y == 0) set_status(status, ISOQ_ST_LEN_RANGE);
+    len = max_pages * kPage;
+  }
+  // causal limits: lim(r) = len - n_q + 1 + i(r), clamped to [0, len]
+  const int lim_lo = MQ ? max(0, min(len, len - n_q + 1 + row_token(0))) : len;
+  const int lim_hi = MQ ? max(0, min(len, len - n_q + 1 + row_token(nh - 1))) : len;
+  const int lim_g = MQ && rg < nh ? max(0, min(len, len - n_q + 1 + row_token(rg))) : lim_hi;
+  const int p_begin = split * pages_per_split;
+  const int p_end = min((lim_hi + kPage - 1) / kPage, p_begin + pages_per_split);
+
+  float* out_base = partials + ((size_t)s * n_q * n_q_heads) * n_splits * PS + (size_t)split * PS;
+  if (tid < RB) row_off[tid] = tid < nh ? row_index(tid) : 0;
+  __syncthreads();
+  if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
+    for (int i = tid; i < nh * PS; i += blockDim.x) {
+      const int h = i / PS, c = i - h * PS;
+      out_base[(size_t)row_off[h] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+    }
+    return;
+  }
+
+  // ---- barriers, then prefetch the first pages of every warp --------------------------
+  uint64_t* mybar = bars + warp * NST;
+  uint8_t* myring = smem + warp * NST * BB;
+  if (lane == 0) {
+    for (int i = 0; i < NST; ++i) mbar_init(mybar + i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const int* pt_row = page_table + (size_t)s * max_pages;
+  // page k of this warp = p_begin + warp + kWarps * k
+  const int n_my = (p_end - p_begin - warp + kWarps - 1) / kWarps;  // may be <= 0
+  auto issue = [&](int k) {  // lane 0 only
+    const int pg = p_begin + warp + kWarps * k;
+    const int st = k % NST;
+    const int phys = __ldg(pt_row + pg);
+    if (phys >= 0 && phys < n_pages) {
+      mbar_expect_tx(mybar + st, BB);
+      bulk_copy(myring + st * BB, blocks + ((size_t)phys * H + hk) * BB, BB, mybar + st);
+    } else {
+      set_status(status, ISOQ_ST_PAGE_RANGE);
+      mbar_arrive(mybar + st);  // complete the phase without data; tokens are masked
+    }
+  };
+  if (lane == 0)
+    for (int k = 0; k < NST && k < n_my; ++k) issue(k);
+  int issued = min(NST, max(n_my, 0));  // warp-uniform count of copies issued
+
+  // ---- a6: rotate the CTA's queries (unnormalised WHT + SO(4)), scale each row to a
+  // 24-bit integer and store its balanced digits as the score mma's A fragments.  k-step
+  // kb, lane (g', t') covers dims base..base+7, base = 32 (t' + 4 (kb / 4)) + 8 (kb % 4):
+  // bytes 0-3 of a0/a1 are dims base..base+3, of a2/a3 dims base+4..base+7.
+  {
+    const float* hp = params + (size_t)hk * D * 4;  // this head's block matrices
+    float pq[NB][16];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, pq[k]);
+    for (int r = warp; r < RB; r += kWarps) {
+      float v[E];
+      if (r < nh) {
+        const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[r]) * D + lane * E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) v[i] = 0.f;
+      }
+      wht_warp<E>(v, lane);
+      float z[E];
+#pragma unroll
+      for (int k = 0; k < NB; ++k) mat_fwd(pq[k], v + 4 * k, z + 4 * k);
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(z[i]));
+      amax = warp_max(amax);
+      const float S = amax > 0.f ? kQMax / amax : 0.f;
+      // log2 score per (integer score / 2^16 * nK): the unnormalised WHT makes z = sqrt(d)
+      // q~ and K_hat = (nK / sqrt(d)) L, so q~.K_hat = nK (score / (S 10000)) / d
+      if (lane == 0)
+        kf_row[r] = S > 0.f ? scale * kLog2e * 65536.0f / (kLevelScale * (float)D * S) : 0.f;
+      // this lane's E dims: lane * E .. + E-1 = E/4 runs of 4 dims (one A register each)
+#pragma unroll
+      for (int k = 0; k < NB; ++k) {
+        const int base = lane * E + 4 * k;  // dims base..base+3
+        int d2[4], d1[4], d0[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) digits3(__float2int_rn(z[4 * k + e] * S), d2[e], d1[e], d0[e]);
+        const uint32_t w2 = pack_s8x4(d2[0], d2[1], d2[2], d2[3]);
+        const uint32_t w1 = pack_s8x4(d1[0], d1[1], d1[2], d1[3]);
+        const uint32_t w0 = pack_s8x4(d0[0], d0[1], d0[2], d0[3]);
+        // base = 32 q + 8 u + 4 hf: group q -> lane t' = q % 4, k-step 4 (q / 4) + u; hf
+        // selects a0/a1 (dims +0..3) or a2/a3 (dims +4..7)
+        const int q = base >> 5, u = (base >> 3) & 3, hf = (base >> 2) & 1;
+        const int kb = 4 * (q >> 2) + u, tq = q & 3;
+        if constexpr (RB == 8) {
+          // lane (g' = r, t' = tq): A1 = (d2, d1, d2+4, d1+4), A2 = (d0, d0+4)
+          uint32_t* f = afr + (kb * 32 + 4 * r + tq) * 4;
+          f[2 * hf] = w2;
+          f[2 * hf + 1] = w1;
+          afr2[(kb * 32 + 4 * r + tq) * 2 + hf] = w0;
+        } else {
+          // rows 0-3: d2 of rows r, 4-7: d1, 8-11: d0 (12-15 zero): lanes g' = r and r + 4
+          uint32_t* fa = afr + (kb * 32 + 4 * r + tq) * 4;        // g' = r
+          uint32_t* fb = afr + (kb * 32 + 4 * (r + 4) + tq) * 4;  // g' = r + 4
+          fa[2 * hf] = w2;      // row r
+          fa[2 * hf + 1] = w0;  // row r + 8
+          fb[2 * hf] = w1;      // row r + 4
+          fb[2 * hf + 1] = 0u;  // row r + 12
+        }
+      }
+    }
+    if constexpr (RB == 4) {  // rows nh..3 of lanes g' >= 4 are written above (r < RB)
+    }
+  }
+  __syncthreads();
+
+  const float kf = kf_row[rg];
+  // level byte tables of the value product (f16 of ALPHA times the levels)
+  uint32_t tl0, tl1, th0, th1;
+  level_tables<3>(tl0, tl1, th0, th1);
+  constexpr float ALPHA = alpha_of<3>();
+
+  // Softmax state of row rg (the score rows of this lane); the value accumulator columns
+  // of this lane are rows 2t, 2t+1 (RB = 4: columns 4-7 unused), whose rescale factors come
+  // from lanes 8t and 8t + 4.
+  float m2 = -CUDART_INF_F;  // running max of the log2 scores of row rg
+  float lsum = 0.f;          // this lane's share of sum p of row rg
+  float sigma = 0.f;         // V-norm reference (warp-uniform)
+  float inv_sigma = 0.f;
+  float acc[MT][4];
+#pragma unroll
+  for (int i = 0; i < MT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+  bool timed_out = false;
+  int k = 0;
+  for (; k < n_my; ++k) {
+    const int st = k % NST;
+    if (!mbar_wait(mybar + st, (k / NST) & 1)) {
+      timed_out = true;
+      break;
+    }
+    const uint8_t* blk = myring + st * BB;
+    const int pg = p_begin + warp + kWarps * k;
+    const int phys = __ldg(pt_row + pg);
+    const bool page_ok = phys >= 0 && phys < n_pages;
+    const int tok0 = pg * kPage;
+
+    // a page whose 64 tokens are all valid takes the tile body without masking
+    const bool full = page_ok && tok0 + kPage <= lim_lo;
+    auto tile = [&](const int tb, auto full_c) {
+      constexpr bool FULL = decltype(full_c)::value;
+      // ---- a7: scores of 4 tiles of 8 tokens; B = K_hat^T of token tb + 8n + g ----------
+      float sv[4][2];  // log2-domain scores of tokens tb + 8n + 2t + c (row rg)
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        int C1[4] = {0, 0, 0, 0}, C2[4] = {0, 0, 0, 0};
+        [[maybe_unused]] int C3[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int gq = 0; gq < NG; ++gq) {
+          const uint32_t* p =
+              reinterpret_cast<const uint32_t*>(blk + (tb + 8 * n + g) * CB) + 3 * (t + 4 * gq);
+          const uint32_t w0 = p[0], w1 = p[1], w2 = p[2];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int kb = 4 * gq + u;
+            const uint32_t S = u == 0 ? (w0 & 0x77777777u)
+                             : u == 1 ? (w1 & 0x77777777u)
+                             : u == 2 ? (w2 & 0x77777777u)
+                                      : spare_codes(w0, w1, w2);
+            const uint32_t S2 = S >> 16;
+            const uint32_t bh0 = prmt(kTH0, kTH1, S), bh1 = prmt(kTH0, kTH1, S2);
+            const uint32_t bl0 = prmt(kTL0, kTL1, S), bl1 = prmt(kTL0, kTL1, S2);
+            if constexpr (RB == 8) {
+              const uint4 A1 = *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4);
+              const uint2 A2 = *reinterpret_cast<const uint2*>(afr2 + (kb * 32 + lane) * 2);
+              mma_s8(C1, A1.x, A1.y, A1.z, A1.w, bh0, bh1);
+              mma_s8(C2, A1.x, A1.y, A1.z, A1.w, bl0, bl1);
+              mma_s8(C3, A2.x, 0u, A2.y, 0u, bh0, bh1);
+            } else {
+              const uint4 A1 = *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4);
+              mma_s8(C1, A1.x, A1.y, A1.z, A1.w, bh0, bh1);
+              mma_s8(C2, A1.x, 0u, A1.z, 0u, bl0, bl1);
+            }
+          }
+        }
+        // tokens tb + 8n + 2t + c: raw = (integer score) / 2^16
+        const int tk = tb + 8 * n + 2 * t;
+        const float2 nk2 = __half22float2(
+            *reinterpret_cast<const __half2*>(blk + k_norm_off(D, 3) + 2 * tk));
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float raw;
+          if constexpr (RB == 8) {
+            const int Z = C1[c] * 256 + (C2[c] + C1[2 + c]);
+            const int Y = C2[2 + c] + C3[c];
+            raw = fmaf((float)Y, 1.0f / 256.0f, (float)Z);
+          } else {
+            // lanes g < 4: d2.kh, d0.kh (row g + 8), d2.kl; lanes g >= 4: d1.kh, d1.kl
+            const bool top = g < 4;
+            const int hi = top ? C1[c] * 256 + C2[c] : C1[c];
+            const int lo = top ? C1[2 + c] : C2[c];
+            const float part = fmaf((float)lo, 1.0f / 256.0f, (float)hi);
+            raw = part + __shfl_xor_sync(kFull, part, 16);
+          }
+          sv[n][c] = raw * ((c ? nk2.y : nk2.x) * kf);
+        }
+      }
+
+      // norms of this lane's V tokens (the same 8 tokens) and the masks
+      float nv[4][2];
+      const float sthr = m2 + kLazy, vthr = sigma * kSigmaSlack;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        const int tk = tb + 8 * n + 2 * t;
+        const float2 nv2 = __half22float2(
+            *reinterpret_cast<const __half2*>(blk + v_norm_off(D, 3) + 2 * tk));
+        nv[n][0] = nv2.x;
+        nv[n][1] = nv2.y;
+        if constexpr (!FULL) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const bool vld = page_ok && (tok0 + tk + c) < lim_hi;
+            sv[n][c] = vld && (!MQ || (tok0 + tk + c) < lim_g) ? sv[n][c] : -CUDART_INF_F;
+            nv[n][c] = vld ? nv[n][c] : 0.f;
+          }
+        }
+      }
+      // this lane's largest score and V norm of the tile (three-input max instructions)
+      float tmax = fmaxf(fmaxf(fmaxf(sv[0][0], sv[0][1]), fmaxf(sv[1][0], sv[1][1])),
+                         fmaxf(fmaxf(sv[2][0], sv[2][1]), fmaxf(sv[3][0], sv[3][1])));
+      float vmax = fmaxf(fmaxf(fmaxf(nv[0][0], nv[0][1]), fmaxf(nv[1][0], nv[1][1])),
+                         fmaxf(fmaxf(nv[2][0], nv[2][1]), fmaxf(nv[3][0], nv[3][1])));
+      const bool grow = (tmax > sthr) | (vmax > vthr);
+      // ---- a8: online softmax.  The running max m2 of a row (shared by the 4 lanes t)
+      // and the V-norm reference sigma move only when a score exceeds m2 + 8 or a norm
+      // exceeds 16 sigma (first tile included), so the common tile needs no shuffles.
+      if (__any_sync(kFull, grow)) {
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, o));
+          vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
+        }
+        float resc = 1.f;
+        if (tmax > sthr) {
+          resc = ex2(m2 - tmax);  // 0 when m2 was -inf
+          lsum *= resc;
+          m2 = tmax;
+        }
+        float vr = 1.f;
+        if (vmax > vthr) {   // warp-uniform
+          vr = sigma / vmax;  // 0 on the first valid tile
+          sigma = vmax;
+          inv_sigma = 1.f / vmax;
+        }
+        // columns 2t, 2t+1 are rows 2t, 2t+1 (RB = 4: rows 2t & 3, unused for t >= 2)
+        const float r0 = __shfl_sync(kFull, resc, 4 * ((2 * t) % RB)) * vr;
+        const float r1 = __shfl_sync(kFull, resc, 4 * ((2 * t + 1) % RB)) * vr;
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          acc[i][0] *= r0;
+          acc[i][1] *= r1;
+          acc[i][2] *= r0;
+          acc[i][3] *= r1;
+        }
+      }
+      // P'^T B fragments of the value mma: 16-token block jb = score tiles 2jb, 2jb+1;
+      // b0 = tile 2jb's tokens 2t, 2t+1, b1 = tile 2jb+1's, column = row g (RB = 4: rows
+      // 4-7 are zero)
+      uint32_t pb[2][2];
+      const bool col_live = RB == 8 || g < 4;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        float p0 = ex2(sv[n][0] - m2), p1 = ex2(sv[n][1] - m2);
+        if constexpr (!FULL) {  // a masked token while m2 is still -inf: -inf - -inf
+          p0 = sv[n][0] != -CUDART_INF_F ? p0 : 0.f;
+          p1 = sv[n][1] != -CUDART_INF_F ? p1 : 0.f;
+        }
+        lsum += p0 + p1;
+        const uint32_t w = pack_f16x2(p0 * (nv[n][0] * inv_sigma), p1 * (nv[n][1] * inv_sigma));
+        pb[n >> 1][n & 1] = col_live ? w : 0u;
+      }
+
+      // ---- a8: V accumulation, A = V_hat^T (rows = dims, k = the block's tokens) --------
+      const uint8_t* vbase = blk + v_codes_off(D, 3) + (tb >> 4) * 6 * D;
+#pragma unroll
+      for (int up = 0; up < NU; ++up) {
+#pragma unroll
+        for (int jb = 0; jb < 2; ++jb) {
+          // this lane's 24 bytes of the 16-token block: units 2 (g + 8 up), +1 of quad t
+          uint32_t W[6];
+          const uint2* src = reinterpret_cast<const uint2*>(
+              vbase + jb * 6 * D + vt_group_off(D, 0, t, 2 * (g + 8 * up)));
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const uint2 w = src[i];
+            W[2 * i] = w.x;
+            W[2 * i + 1] = w.y;
+          }
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {      // unit 2 (g + 8 up) + p
+            const uint32_t* w = W + 3 * p;
+            const uint32_t Sp = spare_codes(w[0], w[1], w[2]);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {    // words 0..2, then the spare unit
+              const int mt = 8 * up + 4 * p + b;
+              const uint32_t S = b < 3 ? (w[b] & 0x77777777u) : Sp;
+              // low half: dim 8u + 2b of members 0-3 (row g); high half: dim + 1 (row g+8)
+              const uint32_t Sh = S >> 16;
+              const uint32_t le = prmt(tl0, tl1, S), he = prmt(th0, th1, S);
+              const uint32_t lo = prmt(tl0, tl1, Sh), ho = prmt(th0, th1, Sh);
+              mma16816(acc[mt], prmt(le, he, 0x5140u), prmt(lo, ho, 0x5140u),
+                       prmt(le, he, 0x7362u), prmt(lo, ho, 0x7362u), pb[jb][0], pb[jb][1]);
+            }
+          }
+        }
+      }
+    };
+#pragma unroll
+    for (int tb = 0; tb < kPage; tb += 32) {
+      if (full) tile(tb, std::true_type{});
+      else tile(tb, std::false_type{});
+    }
+    __syncwarp();
+    // stage st is consumed: refill it with page k + NST
+    if (k + NST < n_my) {
+      if (lane == 0) {
+        fence_proxy_async();
+        issue(k + NST);
+      }
+      ++issued;
+    }
+  }
+
+  if (timed_out) {
+    if (lane == 0) set_status(status, ISOQ_ST_TIMEOUT);
+    // copies k .. issued-1 may still be in flight: wait for them (bounded) before the
+    // CTA's shared memory can be reused or released
+    for (int kk = k; kk < issued; ++kk)
+      if (!mbar_wait(mybar + (kk % NST), (kk / NST) & 1)) break;
+  }
+
+  // ---- merge the 4 warps' states in shared memory, write the chunk's partials ---------
+  // row rg's sum p over the lanes t (RB = 4: lanes g and g + 4 hold the same row)
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
+  __syncthreads();  // all warps done with their rings
+  float* mb = reinterpret_cast<float*>(smem);  // [kWarps][8 rows][D + 4]
+  {
+    // acc_true = acc * sigma / ALPHA (times 1 / exp2(m2) in the log2 frame).  Lane (g, t):
+    // m-tile mt = 8 up + 4 p + b, rows g / g + 8 = dims 8u + 2b / + 1 with u = 2 (g + 8 up)
+    // + p (b = 3: the spare unit, dims 8u + 6, 8u + 7); columns 2t, 2t+1 = rows
+    const float f = sigma / ALPHA;
+    if (2 * t < RB) {
+#pragma unroll
+      for (int up = 0; up < NU; ++up)
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int mt = 8 * up + 4 * p + b;
+            const int d0 = 8 * (2 * (g + 8 * up) + p) + 2 * b;
+            float* r0 = mb + (warp * 8 + 2 * t) * PS;
+            float* r1 = mb + (warp * 8 + 2 * t + 1) * PS;
+            r0[d0] = acc[mt][0] * f;
+            r1[d0] = acc[mt][1] * f;
+            r0[d0 + 1] = acc[mt][2] * f;
+            r1[d0 + 1] = acc[mt][3] * f;
+          }
+    }
+    if (t == 0 && g < RB) {
+      float* r = mb + (warp * 8 + g) * PS;
+      r[D] = m2;
+      r[D + 1] = lsum;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < nh * (D + 1); i += blockDim.x) {
+    const int h = i / (D + 1), c = i - h * (D + 1);
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mb[(w * 8 + h) * PS + D]);
+    float v = 0.f;
+    if (M != -CUDART_INF_F) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = mb[(w * 8 + h) * PS + D];
+        if (mw == -CUDART_INF_F) continue;
+        const float sc = ex2(mw - M);
+        v += sc * mb[(w * 8 + h) * PS + (c == D ? D + 1 : c)];
+      }
+    }
+    float* o = out_base + (size_t)row_off[h] * n_splits * PS;
+    if (c < D) o[c] = v;
+    else {
+      o[D] = M == -CUDART_INF_F ? -CUDART_INF_F : M / kLog2e;  // natural-log units
+      o[D + 1] = v;
+    }
+  }
+}
+
+template <int D, int NST, int RB, typename TQ, bool MQ>
+cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream) {
+  using SM = I8Smem<D, NST, RB>;
+  // the dynamic shared-memory opt-in is per function and per device
+  static unsigned long long attr_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !((attr_set >> dev) & 1ull)) {
+    e = cudaFuncSetAttribute(decode_i8_kernel<D, NST, RB, TQ, MQ>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set |= 1ull << dev;
+  }
+  const int G = a.n_q_heads / a.n_kv_heads;
+  dim3 grid(a.n_splits, a.n_kv_heads * ((a.n_q * G + RB - 1) / RB), a.n_seqs);
+  decode_i8_kernel<D, NST, RB, TQ, MQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
+      a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
+      static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
+      a.n_splits, a.partials, a.status);
+  return cudaGetLastError();
+}
+
+template <int D, int NST, int RB>
+cudaError_t launch_i8_rb(const DecodeArgs& a, cudaStream_t stream) {
+  const bool mq = a.n_q > 1;
+  switch (a.q_dtype) {
+    case ISOQ_F32:
+      return mq ? launch_i8_t<D, NST, RB, float, true>(a, stream)
+                : launch_i8_t<D, NST, RB, float, false>(a, stream);
+    case ISOQ_BF16:
+      return mq ? launch_i8_t<D, NST, RB, __nv_bfloat16, true>(a, stream)
+                : launch_i8_t<D, NST, RB, __nv_bfloat16, false>(a, stream);
+    case ISOQ_F16:
+      return mq ? launch_i8_t<D, NST, RB, __half, true>(a, stream)
+                : launch_i8_t<D, NST, RB, __half, false>(a, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+#ifndef ISOQ_I8_NST128
+#define ISOQ_I8_NST128 2
+#endif
+#ifndef ISOQ_I8_NST256
+#define ISOQ_I8_NST256 2
+#endif
+
+cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.bits != 3) return cudaErrorInvalidValue;
+  const int rb = decode_rows_per_block(a.d, a.n_q, a.n_q_heads / a.n_kv_heads);
+  if (a.d == 128)
+    return rb == 8 ? launch_i8_rb<128, ISOQ_I8_NST128, 8>(a, stream)
+                   : launch_i8_rb<128, ISOQ_I8_NST128, 4>(a, stream);
+  if (a.d == 256) return launch_i8_rb<256, ISOQ_I8_NST256, 4>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+// Resident CTAs per SM of the decode kernel for head dimension d on the current device
+// (cached per device; 2 when it cannot be queried).
+int decode_i8_resident_ctas(int d) {
+  static int cache[64][2] = {{0}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 2;
+  }
+  const int di = d == 256 ? 1 : 0;
+  if (!cache[dev][di]) {
+    int n = 0;
+    cudaError_t e;
+    if (d == 256) {
+      using SM = I8Smem<256, ISOQ_I8_NST256, 4>;
+      auto k = decode_i8_kernel<256, ISOQ_I8_NST256, 4, __nv_bfloat16, false>;
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+      if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kWarps * 32, SM::kBytes);
+    } else {
+      using SM = I8Smem<128, ISOQ_I8_NST128, 8>;
+      auto k = decode_i8_kernel<128, ISOQ_I8_NST128, 8, __nv_bfloat16, false>;
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+      if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kWarps * 32, SM::kBytes);
+    }
+    if (e != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 2;
+    }
+    cache[dev][di] = n;
+  }
+  return cache[dev][di];
+}
+
+}  // namespace isoq

@@ -501,7 +501,7 @@ cudaError_t launch_decode_mma_b(const DecodeArgs& a, cudaStream_t stream) {
 
 template <int D, int NST>
 cudaError_t launch_decode_mma_d(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.bits == 3) return launch_decode_mma_b<D, NST, 3>(a, stream);
+  // 3-bit caches use the V tile layout and the integer kernel (isoq_decode_i8.cu)
   if constexpr (D == 128) {  // the 2- and 4-bit variants exist at d = 128
     if (a.bits == 2) return launch_decode_mma_b<D, NST, 2>(a, stream);
     if (a.bits == 4) return launch_decode_mma_b<D, NST, 4>(a, stream);
@@ -536,19 +536,15 @@ int decode_resident_ctas(int d) {
     int n = 0;
     cudaError_t e;
     if (d == 256) {
-      using SM = MmaSmem<256, ISOQ_DEC_NST256>;
-      e = cudaFuncSetAttribute(decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false, 3>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
-      if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, decode_mma_kernel<256, ISOQ_DEC_NST256, __nv_bfloat16, false, 3>, kWarps * 32, SM::kBytes);
+      n = 2;  // the 2- and 4-bit formats exist at d = 128 only
+      e = cudaSuccess;
     } else {
-      using SM = MmaSmem<128, ISOQ_DEC_NST128>;
-      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false, 3>,
+      using SM = MmaSmem<128, ISOQ_DEC_NST128, 4>;
+      e = cudaFuncSetAttribute(decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false, 4>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false, 3>, kWarps * 32, SM::kBytes);
+            &n, decode_mma_kernel<128, ISOQ_DEC_NST128, __nv_bfloat16, false, 4>, kWarps * 32, SM::kBytes);
     }
     if (e != cudaSuccess || n < 1) {
       cudaGetLastError();

@@ -25,6 +25,7 @@
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
+#include "isoq_vtile.cuh"
 
 namespace isoq {
 using namespace ptx;
@@ -207,12 +208,27 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
       const int tk = u >> 2, q = u & 3;
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
+        const uint32_t base = (kv ? sV : sK);
+        if (BITS == 3 && kv == 1) {
+          // V tile layout: unit u = (block, quad, 8-dim unit) group of four tokens
+          const int B = u >> 6, t4 = (u >> 4) & 3, un = u & 15;
+          const uint32_t* wp = reinterpret_cast<const uint32_t*>(
+              blk + v_codes_off(D, BITS) + vt_group_off(D, B, t4, un));
+          uint32_t o[4][4];
+          vdeq_group(wp[0], wp[1], wp[2], tl0, tl1, th0, th1, o);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             base + tile_off(vt_member_slot(B, t4, j), un)),
+                         "r"(o[j][0]), "r"(o[j][1]), "r"(o[j][2]), "r"(o[j][3])
+                         : "memory");
+          continue;
+        }
         const uint32_t* wp = reinterpret_cast<const uint32_t*>(blk + (kv ? v_codes_off(D, BITS) : 0) +
                                                              tk * CB) + W * q;
         uint32_t w[W];
 #pragma unroll
         for (int i = 0; i < W; ++i) w[i] = wp[i];
-        const uint32_t base = (kv ? sV : sK);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t o[4];

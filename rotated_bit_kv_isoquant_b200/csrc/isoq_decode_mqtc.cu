@@ -30,6 +30,7 @@
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
+#include "isoq_vtile.cuh"
 #include "isoq_tc.cuh"
 
 namespace isoq {
@@ -207,6 +208,20 @@ __global__ void __launch_bounds__(kXRows, 2)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int u = tid + 128 * hf;
+      if (BITS == 3 && kv == 1) {
+        // V tile layout: u = (block, quad, 8-dim unit) group of four tokens
+        const int B = u >> 6, t4 = (u >> 4) & 3, un = u & 15;
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(
+            blk + v_codes_off(D, BITS) + vt_group_off(D, B, t4, un));
+        uint32_t o[4][4];
+        vdeq_group(wp[0], wp[1], wp[2], tl0, tl1, th0, th1, o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int tkj = vt_member_slot(B, t4, j);
+          st_v4(sV + (tkj >> 3) * 2048 + un * 128 + (tkj & 7) * 16, o[j]);
+        }
+        continue;
+      }
       // token, 32-dim group: a warp takes 8 tokens x 4 groups, so its 32-bit code loads
       // (word 12 tk + 3 q + i) hit 32 distinct banks and each quarter-warp's 16-byte tile
       // stores 8 distinct bank groups (tk % 8)

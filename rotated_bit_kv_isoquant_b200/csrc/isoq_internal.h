@@ -70,10 +70,23 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int n_seqs,
                                 int n_q_heads, int n_states, const float* states, float* out,
                                 cudaStream_t stream);
-// Tensor-core split kernel (partials only); the combine runs separately.
+// Tensor-core split kernel (partials only); the combine runs separately.  The 2- and
+// 4-bit formats (f16 operands).
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
 // Resident CTAs per SM of that kernel for head dimension d on the current device.
 int decode_resident_ctas(int d);
+// The 3-bit split kernel on 8-bit integer tensor-core products (partials only).
+cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream);
+int decode_i8_resident_ctas(int d);
+// Rows ((query token, head) pairs of one KV head) per CTA of the 3-bit split kernel: 4
+// when a KV head has at most 4 rows (the query digits of all of them then fit the 16 rows
+// of one mma) or d = 256 (register budget), else 8.
+inline int decode_rows_per_block(int d, int n_q, int group) {
+  return (d == 256 || (long long)n_q * group <= 4) ? 4 : 8;
+}
+// Pages per context chunk at most: a warp of the 3-bit kernel then sums at most 32768
+// tokens into its s32 value accumulators (|per-token term| < 2^16, far from overflow).
+constexpr int kMaxPagesPerSplit = 2048;
 // Multi-token chunks with many rows per KV head (d = 128): the page dequantised once per
 // CTA into shared memory and shared by 64 (query token, head) rows (partials only).
 bool use_shared_mq(const DecodeArgs& a);

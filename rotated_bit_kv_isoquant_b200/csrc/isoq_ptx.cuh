@@ -232,6 +232,33 @@ __device__ __forceinline__ void vdeq(uint32_t Sa, uint32_t Sb, int part, uint32_
   }
 }
 
+// 3-bit V tile layout: the group (W0, W1, W2) of one unit (8 dims) of four member tokens
+// -> o[j][i] = f16x2 (dims 2i, 2i+1 of the unit) of member j, the values ALPHA * level.
+// The low / high 16 bits of a word are one dim of the four members: one lookup of the
+// level's low bytes and one of its high bytes give that dim of all four, then permutes
+// regroup them per token.
+__device__ __forceinline__ void vdeq_group(uint32_t W0, uint32_t W1, uint32_t W2, uint32_t tl0,
+                                           uint32_t tl1, uint32_t th0, uint32_t th1,
+                                           uint32_t (&o)[4][4]) {
+  const uint32_t Sp = spare_codes(W0, W1, W2);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t S = i == 0 ? (W0 & 0x77777777u)
+                     : i == 1 ? (W1 & 0x77777777u)
+                     : i == 2 ? (W2 & 0x77777777u)
+                              : Sp;
+    const uint32_t Sh = S >> 16;
+    const uint32_t le = prmt(tl0, tl1, S), he = prmt(th0, th1, S);    // dim 2i, members 0-3
+    const uint32_t lo = prmt(tl0, tl1, Sh), ho = prmt(th0, th1, Sh);  // dim 2i + 1
+    const uint32_t A01 = prmt(le, he, 0x5140u), A23 = prmt(le, he, 0x7362u);
+    const uint32_t B01 = prmt(lo, ho, 0x5140u), B23 = prmt(lo, ho, 0x7362u);
+    o[0][i] = prmt(A01, B01, 0x5410u);
+    o[1][i] = prmt(A01, B01, 0x7632u);
+    o[2][i] = prmt(A23, B23, 0x5410u);
+    o[3][i] = prmt(A23, B23, 0x7632u);
+  }
+}
+
 __device__ __forceinline__ float half_at(const uint8_t* p) {
   return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
 }

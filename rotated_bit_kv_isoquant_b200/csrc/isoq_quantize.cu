@@ -19,6 +19,7 @@
 #include "isoq_codes.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
+#include "isoq_vtile.cuh"
 
 namespace isoq {
 
@@ -198,9 +199,31 @@ __global__ void __launch_bounds__(256)
           const int src_lane = (E == 4) ? (8 * (m / 3) + 2 * (m % 3)) : (4 * (m / 3) + (m % 3));
           q4[r4] = __shfl_sync(kFull, word, src_lane);
         }
-        uint8_t* dst = blk + (kv == 0 ? 0 : v_codes_off(D)) + slot * CB;
-        if (lane < CB / 16)
-          *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+        if (kv == 0) {
+          uint8_t* dst = blk + slot * CB;
+          if (lane < CB / 16)
+            *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+        } else {
+          // V in the tile layout: the unit word of unit u (dims 8u..8u+7) is lane u's
+          // nibble word (8 dims per lane), or lanes 2u, 2u+1 joined (4 dims per lane); the
+          // token's bits of that unit's group are set in place
+          const uint32_t pair = E == 4 ? __shfl_xor_sync(kFull, nib, 1) : 0u;
+          const bool owner = E == 8 || (lane & 1) == 0;
+          const int u = E == 8 ? lane : lane >> 1;
+          if (owner) {
+            const uint32_t U = E == 8 ? nib : (nib | (pair << 16));
+            int B, t, j;
+            vt_slot(slot, B, t, j);
+            uint32_t W[3], mask;
+            vt_member_words(U, j, W, mask);
+            uint32_t* g = reinterpret_cast<uint32_t*>(blk + v_codes_off(D) + vt_group_off(D, B, t, u));
+#pragma unroll
+            for (int w = 0; w < 3; ++w) {
+              atomicAnd(g + w, ~mask);
+              atomicOr(g + w, W[w]);
+            }
+          }
+        }
 
         if (lane == 0) {
           uint16_t nb = __half_as_ushort(__float2half_rn(n[kv]));
@@ -226,6 +249,7 @@ __global__ void __launch_bounds__(256)
 // The next task's vector, sequence and position are fetched while the current one is
 // processed; the page-table entry is loaded before the arithmetic and used after it.
 constexpr int kTpvThreads = 128;
+constexpr int kTpvStage = 20;  // words per thread of the 3-bit V unit-word stage (16 + pad)
 #ifndef ISOQ_TPV_MINB
 #define ISOQ_TPV_MINB 3
 #endif
@@ -255,6 +279,10 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
   constexpr int VB = D * (int)sizeof(T), VS = VB + 16;
   extern __shared__ __align__(16) float smats[];
   uint8_t* slot_mem = reinterpret_cast<uint8_t*>(smats + H * (D / 4) * 16) + threadIdx.x * VS;
+  // 3-bit V: the unit words of this thread's vector, for the warp's V tile store
+  uint32_t* stage = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(smats + H * (D / 4) * 16) +
+                                                kTpvThreads * VS) +
+                    threadIdx.x * kTpvStage;
 
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
@@ -328,23 +356,27 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     }
     const int sid = nsid, pos = npos;
     prefetch(task + stride);
-    if (t >= n_tokens) continue;
+    // a lane without a valid token still runs the arithmetic (on whatever its slot holds)
+    // and stores nothing: every lane takes part in the warp's 3-bit V store
+    bool valid = t < n_tokens;
     // the page-table entry is loaded here and first used by the stores at the end
-    uint32_t bad = 0;
     int phys = -1;
-    if (sid < 0 || sid >= n_seqs) {
-      bad = ISOQ_ST_SEQ_RANGE;
-    } else if (pos < 0 || (pos >> 6) >= max_pages || (ROPE && pos >= rope_max_pos)) {
-      bad = ISOQ_ST_POS_RANGE;
-    } else {
-      phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
-    }
-    if (bad) {
-      set_status(status, bad);
-      continue;
+    if (valid) {
+      uint32_t bad = 0;
+      if (sid < 0 || sid >= n_seqs) {
+        bad = ISOQ_ST_SEQ_RANGE;
+      } else if (pos < 0 || (pos >> 6) >= max_pages || (ROPE && pos >= rope_max_pos)) {
+        bad = ISOQ_ST_POS_RANGE;
+      } else {
+        phys = __ldg(page_table + (size_t)sid * max_pages + (pos >> 6));
+      }
+      if (bad) {
+        set_status(status, bad);
+        valid = false;
+      }
     }
 
-    if (ROPE && kind == 0) {  // RoPE of K at its position: dims (i, i + D/2)
+    if (ROPE && kind == 0 && valid) {  // RoPE of K at its position: dims (i, i + D/2)
       const float4* tab = reinterpret_cast<const float4*>(rope + (size_t)pos * D);
 #pragma unroll
       for (int i = 0; i < D / 4; ++i) {
@@ -426,27 +458,46 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
 #pragma unroll
         for (int j = 0; j < 3; ++j) rec[3 * g + j] = nib[4 * g + j] | ((N3 << (j + 1)) & 0x88888888u);
       }
+      if (kind == 1) {  // V: the unit words, for the V tile layout
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q)
+          *reinterpret_cast<uint4*>(stage + 4 * q) =
+              make_uint4(nib[4 * q], nib[4 * q + 1], nib[4 * q + 2], nib[4 * q + 3]);
+      }
     } else {
 #pragma unroll
       for (int j = 0; j < CB / 4; ++j) rec[j] = join_halves(half[2 * j], half[2 * j + 1]);
     }
-    if (phys < 0 || phys >= n_pages) {
+    if (valid && (phys < 0 || phys >= n_pages)) {
       set_status(status, ISOQ_ST_PAGE_RANGE);
-      continue;
+      valid = false;
     }
-    uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
-    const int slot = pos & (kPage - 1);
-    uint4* dst = reinterpret_cast<uint4*>(blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB);
+    if (!valid) phys = -1;
+    if (valid) {
+      uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
+      const int slot = pos & (kPage - 1);
+      if (BITS != 3 || kind == 0) {
+        uint4* dst =
+            reinterpret_cast<uint4*>(blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB);
 #pragma unroll
-    for (int q = 0; q < CB / 16; ++q)
-      dst[q] = make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
-    uint16_t nb = __half_as_ushort(__float2half_rn(n));
-    if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
-      nb = 0x7bffu;
-      set_status(status, ISOQ_ST_NORM_SAT);
+        for (int q = 0; q < CB / 16; ++q)
+          dst[q] = make_uint4(rec[4 * q], rec[4 * q + 1], rec[4 * q + 2], rec[4 * q + 3]);
+      }
+      uint16_t nb = __half_as_ushort(__float2half_rn(n));
+      if ((nb & 0x7fffu) == 0x7c00u) {  // overflowed binary16
+        nb = 0x7bffu;
+        set_status(status, ISOQ_ST_NORM_SAT);
+      }
+      *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
+                                   2 * slot) = nb;
     }
-    *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
-                                 2 * slot) = nb;
+    if constexpr (BITS == 3) {
+      if (kind == 1) {  // warp-uniform: the task is the warp's
+        __syncwarp();
+        vt_store_warp<D, kTpvStage>(stage - lane * kTpvStage, lane, sid, pos, phys, blocks, H, h);
+        __syncwarp();  // the stage is rewritten by the next task
+      }
+    }
   }
 }
 
@@ -466,7 +517,8 @@ static cudaError_t launch_t(const QuantizeArgs& a, cudaStream_t stream, int n_sm
 template <typename T, int BITS, bool ROPE>
 static cudaError_t launch_tpv(const QuantizeArgs& a, cudaStream_t stream, int n_sm) {
   const size_t smem = (size_t)a.n_kv_heads * 32 * 16 * sizeof(float) +
-                      (size_t)kTpvThreads * (128 * sizeof(T) + 16);
+                      (size_t)kTpvThreads * (128 * sizeof(T) + 16) +
+                      (size_t)kTpvThreads * kTpvStage * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(quantize_tpv_kernel<T, BITS, ROPE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

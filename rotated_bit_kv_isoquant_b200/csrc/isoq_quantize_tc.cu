@@ -32,6 +32,7 @@
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
 #include "isoq_tc.cuh"
+#include "isoq_vtile.cuh"
 
 namespace isoq {
 namespace {
@@ -47,7 +48,9 @@ constexpr int kOffH = 2 * kQtTile;                // the Hadamard operand
 constexpr int kOffM = kOffH + kQtTile;            // [3] block-matrix stages
 constexpr int kOffBar = kOffM + 3 * kQtMat;       // 2 mbarriers (UMMA completion)
 constexpr int kOffSlot = kOffBar + 16;            // tensor-memory base address
-constexpr int kQtSmem = kOffSlot + 16;
+constexpr int kStageWords = 20;                   // per thread: 16 unit words (+4 pad)
+constexpr int kOffStage = kOffSlot + 16;          // [128 threads][20] 3-bit V unit words
+constexpr int kQtSmem = kOffStage + kQtThreads * kStageWords * 4;
 constexpr uint32_t kQtCols = 256;                 // two 128-column f32 accumulators
 
 // Byte offset of element (row, k) of a K-major no-swizzle operand tile: core matrices of
@@ -96,6 +99,7 @@ __global__ void __launch_bounds__(kQtThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffSlot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t* stage = reinterpret_cast<uint32_t*>(smem + kOffStage) + tid * kStageWords;
   const int quad = warp;           // tensor-memory lane quarter
   const int r = quad * 32 + lane;  // this thread's vector (row) of the tile
   const int n_chunks = (n_tokens + kQtRows - 1) / kQtRows;
@@ -321,6 +325,9 @@ __global__ void __launch_bounds__(kQtThreads, 2)
           for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[8 * gg + 2 * j], half[8 * gg + 2 * j + 1]);
 #pragma unroll
           for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
+          if (kind == 1)  // V: the unit words 8 hf + 4 gg .. +3, for the V tile layout
+            *reinterpret_cast<uint4*>(stage + 8 * hf + 4 * gg) =
+                make_uint4(nib[0], nib[1], nib[2], nib[3]);
         }
       } else {
 #pragma unroll
@@ -331,7 +338,9 @@ __global__ void __launch_bounds__(kQtThreads, 2)
         uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
         const int slot = pos & (kPage - 1);
         uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB + (CB / 2) * hf;
-        if constexpr (BITS == 3) {  // 24 bytes at 0 or 24: 16 + 8 or 8 + 16
+        if (BITS == 3 && kind == 1) {
+          // V at 3 bits: written after both halves, in the V tile layout
+        } else if constexpr (BITS == 3) {  // 24 bytes at 0 or 24: 16 + 8 or 8 + 16
           if (hf == 0) {
             *reinterpret_cast<uint4*>(dst) = make_uint4(rec[0], rec[1], rec[2], rec[3]);
             *reinterpret_cast<uint2*>(dst + 16) = make_uint2(rec[4], rec[5]);
@@ -354,6 +363,12 @@ __global__ void __launch_bounds__(kQtThreads, 2)
           *reinterpret_cast<uint16_t*>(blk + (kind == 0 ? k_norm_off(D, BITS) : v_norm_off(D, BITS)) +
                                        2 * slot) = nb;
         }
+      }
+    }
+    if constexpr (BITS == 3) {
+      if (kind == 1) {  // CTA-uniform
+        __syncwarp();
+        vt_store_warp<kQtD, kStageWords>(stage - lane * kStageWords, lane, sid, pos, phys, blocks, H, h);
       }
     }
     if (has_next) {

@@ -93,7 +93,11 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_rejects_requests_larger_than_its_array():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    d, n_kv, n_seqs, G = 256, 8, 64, 16
+    d, n_kv, G = 256, 8, 16
+    n_seqs = 64   # more sequences until one decode's partials exceed the array
+    while iq.isoq_decode_workspace_bytes(n_seqs, n_kv * G, n_kv, d, 4096) <= \
+            iq.ISOQ_NOALLOC_SCRATCH_BYTES:
+        n_seqs *= 2
     params = iq.isoq_make_params(0, d, n_kv)
     cache = iq.PagedCache(d, n_kv, 1, torch.zeros((n_seqs, 1), dtype=torch.int32))
     need = iq.isoq_decode_workspace_bytes(n_seqs, n_kv * G, n_kv, d, 4096)

@@ -50,6 +50,7 @@
 
 namespace isoq {
 using namespace ptx;
+int decode_i8_sms();
 namespace {
 
 constexpr float kQMax = 8.0e6f;       // |24-bit query integer| bound (digits stay in s8)
@@ -62,6 +63,22 @@ __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, ui
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The same with a zero accumulator (c = a . b): no zeroing of c beforehand.
+__device__ __forceinline__ void mma_s8_first(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {0,0,0,0};"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool FIRST>
+__device__ __forceinline__ void mma_s8_acc(int (&c)[4], uint4 a, uint32_t b0, uint32_t b1) {
+  if constexpr (FIRST) mma_s8_first(c, a.x, a.y, a.z, a.w, b0, b1);
+  else mma_s8(c, a.x, a.y, a.z, a.w, b0, b1);
 }
 
 // Integer level 10000 L[c] = kh * 256 + kl with kl in [-128, 127], kh = floor((v + 128) / 256).
@@ -98,38 +115,54 @@ __device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
          ((uint32_t)(d & 255) << 24);
 }
 
-// Shared memory: [kWarps][NST] page stages, the mbarriers, the score mma's A fragments
-// (A1: 4 words per k-step and lane, 16-byte aligned; RB = 8 also A2: 2 words, 8-byte
-// aligned), per-row score factors, output row indices.  The stage area is reused for the
-// final merge.
-template <int D, int NST, int RB>
+// Shared memory: [NW warps][NST] page stages, the mbarriers, the score mma's A fragments
+// (A1 and A2, 4 words per k-step and lane; A2 holds its zero rows explicitly, so each is
+// one 16-byte load straight into the mma's register quad), per-row score factors, output
+// row indices.  The stage area is reused for the final merge.
+template <int D, int NST, int RB, int NW>
 struct I8Smem {
   static constexpr int kStageBytes = block_bytes(D, 3);
-  static constexpr int kRing = kWarps * NST * kStageBytes;
+  static constexpr int kRing = NW * NST * kStageBytes;
   static constexpr int kBarOff = kRing;
-  static constexpr int kAOff = kBarOff + kWarps * NST * 8;             // uint4 [D/32][32]
-  static constexpr int kA2Off = kAOff + (D / 32) * 32 * 16;            // uint2 [D/32][32]
-  static constexpr int kKfOff = kA2Off + (RB == 8 ? (D / 32) * 32 * 8 : 0);  // float [8]
+  static constexpr int kAOff = kBarOff + NW * NST * 8;                 // uint4 [D/32][32]
+  static constexpr int kA2Off = kAOff + (D / 32) * 32 * 16;            // uint4 [D/32][32]
+  static constexpr int kKfOff = kA2Off + (D / 32) * 32 * 16;           // float [8]
   static constexpr int kRowOff = kKfOff + 8 * 4;                      // int [8]
   static constexpr int kBytes = kRowOff + 8 * 4;
-  static constexpr int kMergeBytes = kWarps * 8 * (D + 4) * 4;
+  static constexpr int kMergeBytes = NW * 8 * (D + 4) * 4;
   static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
-  static_assert(kAOff % 16 == 0 && kA2Off % 8 == 0, "A fragments must be aligned");
+  static_assert(kAOff % 16 == 0 && kA2Off % 16 == 0, "A fragments must be aligned");
 };
 
+#ifndef ISOQ_I8_MINB128
+#define ISOQ_I8_MINB128 4
+#endif
+#ifndef ISOQ_I8_NT  // 8-token score tiles per load of the query fragments (1, 2 or 4)
+#define ISOQ_I8_NT 4
+#endif
+constexpr int kI8NT = ISOQ_I8_NT;
+static_assert(4 % kI8NT == 0, "score tiles per fragment load");
+
+// CTAs per SM the register budget is set for: 4-warp CTAs as many as fit (d = 128: 4, d =
+// 256: 2); the wide CTAs of small grids (one per SM) get the same per-thread budget.
 template <int D>
-constexpr int i8_min_blocks() { return D == 128 ? 3 : 2; }
+constexpr int i8_min_blocks(int nw) { return nw == 4 ? (D == 128 ? ISOQ_I8_MINB128 : 2) : 1; }
+
 
 // MQ: chunks of several query tokens per sequence with causal limits; the decode (one
 // query token, every row attending the whole context) is compiled without them.
-template <int D, int NST, int RB, typename TQ, bool MQ>
-__global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
+// NW: warps per CTA.  4 normally (several CTAs per SM); a grid with fewer CTAs than the
+// GPU holds gives each CTA more warps (16 at d = 128, 8 at d = 256), so that the pages of
+// a chunk are in flight at once instead of one after another per warp, at the cost of one
+// query rotation and one merge per CTA as before.
+template <int D, int NST, int RB, typename TQ, bool MQ, int NW>
+__global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
     decode_i8_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
                      const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                      const TQ* __restrict__ Q, int n_q_heads, int n_q,
                      const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
                      int n_splits, float* __restrict__ partials, uint32_t* status) {
-  using SM = I8Smem<D, NST, RB>;
+  using SM = I8Smem<D, NST, RB, NW>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
   constexpr int CB = code_bytes(D, 3);
@@ -141,7 +174,7 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint32_t* afr = reinterpret_cast<uint32_t*>(smem + SM::kAOff);    // [D/32][32][4]
-  uint32_t* afr2 = reinterpret_cast<uint32_t*>(smem + SM::kA2Off);  // [D/32][32][2] (RB = 8)
+  uint32_t* afr2 = reinterpret_cast<uint32_t*>(smem + SM::kA2Off);  // [D/32][32][4]
   float* kf_row = reinterpret_cast<float*>(smem + SM::kKfOff);
   int* row_off = reinterpret_cast<int*>(smem + SM::kRowOff);
 
@@ -197,10 +230,10 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
   }
   __syncwarp();
   const int* pt_row = page_table + (size_t)s * max_pages;
-  // page k of this warp = p_begin + warp + kWarps * k
-  const int n_my = (p_end - p_begin - warp + kWarps - 1) / kWarps;  // may be <= 0
+  // page k of this warp = p_begin + warp + NW * k
+  const int n_my = (p_end - p_begin - warp + NW - 1) / NW;  // may be <= 0
   auto issue = [&](int k) {  // lane 0 only
-    const int pg = p_begin + warp + kWarps * k;
+    const int pg = p_begin + warp + NW * k;
     const int st = k % NST;
     const int phys = __ldg(pt_row + pg);
     if (phys >= 0 && phys < n_pages) {
@@ -224,7 +257,7 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
     float pq[NB][16];
 #pragma unroll
     for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, pq[k]);
-    for (int r = warp; r < RB; r += kWarps) {
+    for (int r = warp; r < RB; r += NW) {
       float v[E];
       if (r < nh) {
         const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[r]) * D + lane * E;
@@ -266,15 +299,24 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
           uint32_t* f = afr + (kb * 32 + 4 * r + tq) * 4;
           f[2 * hf] = w2;
           f[2 * hf + 1] = w1;
-          afr2[(kb * 32 + 4 * r + tq) * 2 + hf] = w0;
+          uint32_t* f2 = afr2 + (kb * 32 + 4 * r + tq) * 4;  // A2 = [d0; 0]
+          f2[2 * hf] = w0;
+          f2[2 * hf + 1] = 0u;
         } else {
-          // rows 0-3: d2 of rows r, 4-7: d1, 8-11: d0 (12-15 zero): lanes g' = r and r + 4
-          uint32_t* fa = afr + (kb * 32 + 4 * r + tq) * 4;        // g' = r
-          uint32_t* fb = afr + (kb * 32 + 4 * (r + 4) + tq) * 4;  // g' = r + 4
+          // A1: rows 0-3: d2 of rows r, 4-7: d1, 8-11: d0 (12-15 zero); A2: the same
+          // without d0.  Lanes g' = r and r + 4.
+          uint32_t* fa = afr + (kb * 32 + 4 * r + tq) * 4;         // g' = r
+          uint32_t* fb = afr + (kb * 32 + 4 * (r + 4) + tq) * 4;   // g' = r + 4
+          uint32_t* ga = afr2 + (kb * 32 + 4 * r + tq) * 4;
+          uint32_t* gb = afr2 + (kb * 32 + 4 * (r + 4) + tq) * 4;
           fa[2 * hf] = w2;      // row r
           fa[2 * hf + 1] = w0;  // row r + 8
           fb[2 * hf] = w1;      // row r + 4
           fb[2 * hf + 1] = 0u;  // row r + 12
+          ga[2 * hf] = w2;
+          ga[2 * hf + 1] = 0u;
+          gb[2 * hf] = w1;
+          gb[2 * hf + 1] = 0u;
         }
       }
     }
@@ -284,9 +326,15 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
   __syncthreads();
 
   const float kf = kf_row[rg];
-  // level byte tables of the value product (f16 of ALPHA times the levels)
+  // level byte tables: the scores' integer level bytes and the value product's f16 level
+  // bytes (ALPHA times the levels).  They are constants, but opaque to the compiler here:
+  // otherwise it rebuilds a table word with a move before every byte permute instead of
+  // keeping the eight words in registers.
   uint32_t tl0, tl1, th0, th1;
   level_tables<3>(tl0, tl1, th0, th1);
+  uint32_t kh0 = kTH0, kh1 = kTH1, kl0 = kTL0, kl1 = kTL1;
+  asm volatile("" : "+r"(tl0), "+r"(tl1), "+r"(th0), "+r"(th1));
+  asm volatile("" : "+r"(kh0), "+r"(kh1), "+r"(kl0), "+r"(kl1));
   constexpr float ALPHA = alpha_of<3>();
 
   // Softmax state of row rg (the score rows of this lane); the value accumulator columns
@@ -309,7 +357,7 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
       break;
     }
     const uint8_t* blk = myring + st * BB;
-    const int pg = p_begin + warp + kWarps * k;
+    const int pg = p_begin + warp + NW * k;
     const int phys = __ldg(pt_row + pg);
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
@@ -319,59 +367,77 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
     auto tile = [&](const int tb, auto full_c) {
       constexpr bool FULL = decltype(full_c)::value;
       // ---- a7: scores of 4 tiles of 8 tokens; B = K_hat^T of token tb + 8n + g ----------
+      // NT tiles at a time share each load of the query fragments
       float sv[4][2];  // log2-domain scores of tokens tb + 8n + 2t + c (row rg)
 #pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        int C1[4] = {0, 0, 0, 0}, C2[4] = {0, 0, 0, 0};
-        [[maybe_unused]] int C3[4] = {0, 0, 0, 0};
+      for (int n0 = 0; n0 < 4; n0 += kI8NT) {
+        int C1[kI8NT][4], C2[kI8NT][4];
+        [[maybe_unused]] int C3[kI8NT][4];
 #pragma unroll
         for (int gq = 0; gq < NG; ++gq) {
-          const uint32_t* p =
-              reinterpret_cast<const uint32_t*>(blk + (tb + 8 * n + g) * CB) + 3 * (t + 4 * gq);
-          const uint32_t w0 = p[0], w1 = p[1], w2 = p[2];
+          uint32_t w[kI8NT][3];
+#pragma unroll
+          for (int nn = 0; nn < kI8NT; ++nn) {
+            const uint32_t* p = reinterpret_cast<const uint32_t*>(
+                                    blk + (tb + 8 * (n0 + nn) + g) * CB) + 3 * (t + 4 * gq);
+            w[nn][0] = p[0];
+            w[nn][1] = p[1];
+            w[nn][2] = p[2];
+          }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int kb = 4 * gq + u;
-            const uint32_t S = u == 0 ? (w0 & 0x77777777u)
-                             : u == 1 ? (w1 & 0x77777777u)
-                             : u == 2 ? (w2 & 0x77777777u)
-                                      : spare_codes(w0, w1, w2);
-            const uint32_t S2 = S >> 16;
-            const uint32_t bh0 = prmt(kTH0, kTH1, S), bh1 = prmt(kTH0, kTH1, S2);
-            const uint32_t bl0 = prmt(kTL0, kTL1, S), bl1 = prmt(kTL0, kTL1, S2);
-            if constexpr (RB == 8) {
-              const uint4 A1 = *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4);
-              const uint2 A2 = *reinterpret_cast<const uint2*>(afr2 + (kb * 32 + lane) * 2);
-              mma_s8(C1, A1.x, A1.y, A1.z, A1.w, bh0, bh1);
-              mma_s8(C2, A1.x, A1.y, A1.z, A1.w, bl0, bl1);
-              mma_s8(C3, A2.x, 0u, A2.y, 0u, bh0, bh1);
-            } else {
-              const uint4 A1 = *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4);
-              mma_s8(C1, A1.x, A1.y, A1.z, A1.w, bh0, bh1);
-              mma_s8(C2, A1.x, 0u, A1.z, 0u, bl0, bl1);
+            const uint4 A1 = *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4);
+            const uint4 A2 = *reinterpret_cast<const uint4*>(afr2 + (kb * 32 + lane) * 4);
+#pragma unroll
+            for (int nn = 0; nn < kI8NT; ++nn) {
+              const uint32_t S = u == 0 ? (w[nn][0] & 0x77777777u)
+                               : u == 1 ? (w[nn][1] & 0x77777777u)
+                               : u == 2 ? (w[nn][2] & 0x77777777u)
+                                        : spare_codes(w[nn][0], w[nn][1], w[nn][2]);
+              const uint32_t S2 = S >> 16;
+              const uint32_t bh0 = prmt(kh0, kh1, S), bh1 = prmt(kh0, kh1, S2);
+              const uint32_t bl0 = prmt(kl0, kl1, S), bl1 = prmt(kl0, kl1, S2);
+              // the first k-step starts the accumulators from zero
+              auto step = [&](auto first) {
+                constexpr bool F = decltype(first)::value;
+                mma_s8_acc<F>(C1[nn], A1, bh0, bh1);
+                if constexpr (RB == 8) {
+                  mma_s8_acc<F>(C2[nn], A1, bl0, bl1);
+                  mma_s8_acc<F>(C3[nn], A2, bh0, bh1);
+                } else {
+                  mma_s8_acc<F>(C2[nn], A2, bl0, bl1);
+                }
+              };
+              if (gq == 0 && u == 0) step(std::true_type{});
+              else step(std::false_type{});
             }
           }
         }
         // tokens tb + 8n + 2t + c: raw = (integer score) / 2^16
-        const int tk = tb + 8 * n + 2 * t;
-        const float2 nk2 = __half22float2(
-            *reinterpret_cast<const __half2*>(blk + k_norm_off(D, 3) + 2 * tk));
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float raw;
-          if constexpr (RB == 8) {
-            const int Z = C1[c] * 256 + (C2[c] + C1[2 + c]);
-            const int Y = C2[2 + c] + C3[c];
-            raw = fmaf((float)Y, 1.0f / 256.0f, (float)Z);
-          } else {
-            // lanes g < 4: d2.kh, d0.kh (row g + 8), d2.kl; lanes g >= 4: d1.kh, d1.kl
-            const bool top = g < 4;
-            const int hi = top ? C1[c] * 256 + C2[c] : C1[c];
-            const int lo = top ? C1[2 + c] : C2[c];
-            const float part = fmaf((float)lo, 1.0f / 256.0f, (float)hi);
-            raw = part + __shfl_xor_sync(kFull, part, 16);
+        for (int nn = 0; nn < kI8NT; ++nn) {
+          const int n = n0 + nn;
+          const int tk = tb + 8 * n + 2 * t;
+          const float2 nk2 = __half22float2(
+              *reinterpret_cast<const __half2*>(blk + k_norm_off(D, 3) + 2 * tk));
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float raw;
+            if constexpr (RB == 8) {
+              const int Z = C1[nn][c] * 256 + (C2[nn][c] + C1[nn][2 + c]);
+              const int Y = C2[nn][2 + c] + C3[nn][c];
+              raw = fmaf((float)Y, 1.0f / 256.0f, (float)Z);
+            } else {
+              // lanes g < 4: d2.kh, d0.kh (row g + 8), d2.kl; lanes g >= 4: d1.kh, d1.kl
+              const bool top = g < 4;
+              const int hi = top ? C1[nn][c] * 256 + C2[nn][c] : C1[nn][c];
+              const int lo = top ? C1[nn][2 + c] : C2[nn][c];
+              const float part = fmaf((float)lo, 1.0f / 256.0f, (float)hi);
+              raw = part + __shfl_xor_sync(kFull, part, 16);
+            }
+            sv[n][c] = raw * ((c ? nk2.y : nk2.x) * kf);
           }
-          sv[n][c] = raw * ((c ? nk2.y : nk2.x) * kf);
         }
       }
 
@@ -513,7 +579,7 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
 #pragma unroll
   for (int o = 1; o < 4; o <<= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
   __syncthreads();  // all warps done with their rings
-  float* mb = reinterpret_cast<float*>(smem);  // [kWarps][8 rows][D + 4]
+  float* mb = reinterpret_cast<float*>(smem);  // [NW][8 rows][D + 4]
   {
     // acc_true = acc * sigma / ALPHA (times 1 / exp2(m2) in the log2 frame).  Lane (g, t):
     // m-tile mt = 8 up + 4 p + b, rows g / g + 8 = dims 8u + 2b / + 1 with u = 2 (g + 8 up)
@@ -547,11 +613,11 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
     const int h = i / (D + 1), c = i - h * (D + 1);
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mb[(w * 8 + h) * PS + D]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mb[(w * 8 + h) * PS + D]);
     float v = 0.f;
     if (M != -CUDART_INF_F) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
+      for (int w = 0; w < NW; ++w) {
         const float mw = mb[(w * 8 + h) * PS + D];
         if (mw == -CUDART_INF_F) continue;
         const float sc = ex2(mw - M);
@@ -567,27 +633,41 @@ __global__ void __launch_bounds__(kWarps * 32, i8_min_blocks<D>())
   }
 }
 
-template <int D, int NST, int RB, typename TQ, bool MQ>
+template <int D, int NST, int RB, typename TQ, bool MQ, int NW>
 cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream) {
-  using SM = I8Smem<D, NST, RB>;
+  using SM = I8Smem<D, NST, RB, NW>;
   // the dynamic shared-memory opt-in is per function and per device
   static unsigned long long attr_set = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !((attr_set >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(decode_i8_kernel<D, NST, RB, TQ, MQ>,
+    e = cudaFuncSetAttribute(decode_i8_kernel<D, NST, RB, TQ, MQ, NW>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
     if (e != cudaSuccess) return e;
     attr_set |= 1ull << dev;
   }
   const int G = a.n_q_heads / a.n_kv_heads;
   dim3 grid(a.n_splits, a.n_kv_heads * ((a.n_q * G + RB - 1) / RB), a.n_seqs);
-  decode_i8_kernel<D, NST, RB, TQ, MQ><<<grid, kWarps * 32, SM::kBytes, stream>>>(
+  decode_i8_kernel<D, NST, RB, TQ, MQ, NW><<<grid, NW * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
       a.n_splits, a.partials, a.status);
   return cudaGetLastError();
+}
+
+// Wide CTAs (more warps, one CTA per SM) when the whole grid fits in one CTA per SM: the
+// GPU would otherwise run a small decode with a few warps per SM, each walking its pages
+// one after another.
+template <int D, int NST, int RB, typename TQ, bool MQ>
+cudaError_t launch_i8_w(const DecodeArgs& a, cudaStream_t stream) {
+  constexpr int kWide = D == 128 ? 16 : 8;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  const long long ctas =
+      (long long)a.n_splits * a.n_kv_heads * ((a.n_q * G + RB - 1) / RB) * a.n_seqs;
+  if (ctas <= (long long)decode_i8_sms())
+    return launch_i8_t<D, NST, RB, TQ, MQ, kWide>(a, stream);
+  return launch_i8_t<D, NST, RB, TQ, MQ, 4>(a, stream);
 }
 
 template <int D, int NST, int RB>
@@ -595,14 +675,14 @@ cudaError_t launch_i8_rb(const DecodeArgs& a, cudaStream_t stream) {
   const bool mq = a.n_q > 1;
   switch (a.q_dtype) {
     case ISOQ_F32:
-      return mq ? launch_i8_t<D, NST, RB, float, true>(a, stream)
-                : launch_i8_t<D, NST, RB, float, false>(a, stream);
+      return mq ? launch_i8_w<D, NST, RB, float, true>(a, stream)
+                : launch_i8_w<D, NST, RB, float, false>(a, stream);
     case ISOQ_BF16:
-      return mq ? launch_i8_t<D, NST, RB, __nv_bfloat16, true>(a, stream)
-                : launch_i8_t<D, NST, RB, __nv_bfloat16, false>(a, stream);
+      return mq ? launch_i8_w<D, NST, RB, __nv_bfloat16, true>(a, stream)
+                : launch_i8_w<D, NST, RB, __nv_bfloat16, false>(a, stream);
     case ISOQ_F16:
-      return mq ? launch_i8_t<D, NST, RB, __half, true>(a, stream)
-                : launch_i8_t<D, NST, RB, __half, false>(a, stream);
+      return mq ? launch_i8_w<D, NST, RB, __half, true>(a, stream)
+                : launch_i8_w<D, NST, RB, __half, false>(a, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -626,8 +706,8 @@ cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream) {
   return cudaErrorInvalidValue;
 }
 
-// Resident CTAs per SM of the decode kernel for head dimension d on the current device
-// (cached per device; 2 when it cannot be queried).
+// Resident 4-warp CTAs per SM of the decode kernel for head dimension d on the current
+// device (cached per device; 2 when it cannot be queried).
 int decode_i8_resident_ctas(int d) {
   static int cache[64][2] = {{0}};
   int dev = 0;
@@ -640,17 +720,17 @@ int decode_i8_resident_ctas(int d) {
     int n = 0;
     cudaError_t e;
     if (d == 256) {
-      using SM = I8Smem<256, ISOQ_I8_NST256, 4>;
-      auto k = decode_i8_kernel<256, ISOQ_I8_NST256, 4, __nv_bfloat16, false>;
+      using SM = I8Smem<256, ISOQ_I8_NST256, 4, 4>;
+      auto k = decode_i8_kernel<256, ISOQ_I8_NST256, 4, __nv_bfloat16, false, 4>;
       e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kWarps * 32, SM::kBytes);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, 4 * 32, SM::kBytes);
     } else {
-      using SM = I8Smem<128, ISOQ_I8_NST128, 8>;
-      auto k = decode_i8_kernel<128, ISOQ_I8_NST128, 8, __nv_bfloat16, false>;
+      using SM = I8Smem<128, ISOQ_I8_NST128, 8, 4>;
+      auto k = decode_i8_kernel<128, ISOQ_I8_NST128, 8, __nv_bfloat16, false, 4>;
       e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
       if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kWarps * 32, SM::kBytes);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, 4 * 32, SM::kBytes);
     }
     if (e != cudaSuccess || n < 1) {
       cudaGetLastError();
@@ -659,6 +739,17 @@ int decode_i8_resident_ctas(int d) {
     cache[dev][di] = n;
   }
   return cache[dev][di];
+}
+
+// SM count of the current device (148 when it cannot be queried).
+int decode_i8_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  return sms;
 }
 
 }  // namespace isoq

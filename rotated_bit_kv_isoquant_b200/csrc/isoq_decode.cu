@@ -24,8 +24,10 @@ namespace isoq {
 // a later merge with the states of other context slices.  Part j of (s, h) sits at
 // parts + (s * n_q_heads + h) * sh_stride + j * part_stride floats.  One CTA of 128
 // threads per (sequence, head): the parts are spread over 4 groups of 32 lanes (each lane
-// 4 or 8 dims, 16-byte loads, several parts in flight), so the merge costs a few memory
-// round trips however many parts there are; warp 0 then finishes.
+// 4 or 8 dims, 16-byte loads, several parts in flight), each group merging its parts in
+// one pass with a running maximum; the groups then merge in shared memory and warp 0
+// finishes.  Launched as a programmatic dependent of the split kernel: the rotation
+// parameters are read before griddepcontrol.wait, the partials after it.
 template <int D, bool FINAL>
 __global__ void __launch_bounds__(128)
     decode_combine_kernel(const float* __restrict__ params, int H, int n_q_heads,
@@ -43,61 +45,67 @@ __global__ void __launch_bounds__(128)
   const int G = n_q_heads / H;
   const float* base = partials + ((size_t)s * rows_per_seq + h) * sh_stride;
 
-  // global max of the splits' running maxima (empty splits report -inf)
-  float M = -CUDART_INF_F;
-  for (int j = tid; j < n_splits; j += 128) M = fmaxf(M, __ldg(base + (size_t)j * part_stride + D));
-  M = warp_max(M);
-  if (lane == 0) red_m[grp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+  // the inverse rotation's block matrices (independent of the split kernel)
+  float Mb[NB][16];
+  if (FINAL && grp == 0) {
+    const float* hp = params + (size_t)((h % n_q_heads) / G) * D * 4;
+#pragma unroll
+    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, Mb[k]);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials are complete
 
-  float acc[E], L = 0.f;
+  // this group's parts j = grp, grp + 4, ...: running maximum Mg, acc and L relative to it
+  float acc[E], L = 0.f, Mg = -CUDART_INF_F;
 #pragma unroll
   for (int i = 0; i < E; ++i) acc[i] = 0.f;
-  if (M != -CUDART_INF_F) {
-    int j = grp;
-    for (; j + 4 * (UNROLL - 1) < n_splits; j += 4 * UNROLL) {
-      float mj[UNROLL], lj[UNROLL];
-      float4 v[UNROLL][NB];
+  auto take = [&](float mj, float lj, const float4 (&v)[NB]) {
+    if (mj == -CUDART_INF_F) return;  // an empty chunk
+    if (mj > Mg) {                    // group-uniform
+      const float r = __expf(Mg - mj);  // 0 when Mg was -inf
+      L *= r;
 #pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        const float* p = base + (size_t)(j + 4 * u) * part_stride;
-        mj[u] = __ldg(p + D);
-        lj[u] = __ldg(p + D + 1);
-#pragma unroll
-        for (int k = 0; k < NB; ++k) v[u][k] = __ldg(reinterpret_cast<const float4*>(p + lane * E) + k);
-      }
-#pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        const float w = mj[u] == -CUDART_INF_F ? 0.f : __expf(mj[u] - M);
-        L = fmaf(w, lj[u], L);
-#pragma unroll
-        for (int k = 0; k < NB; ++k) {
-          acc[4 * k + 0] = fmaf(w, v[u][k].x, acc[4 * k + 0]);
-          acc[4 * k + 1] = fmaf(w, v[u][k].y, acc[4 * k + 1]);
-          acc[4 * k + 2] = fmaf(w, v[u][k].z, acc[4 * k + 2]);
-          acc[4 * k + 3] = fmaf(w, v[u][k].w, acc[4 * k + 3]);
-        }
-      }
+      for (int i = 0; i < E; ++i) acc[i] *= r;
+      Mg = mj;
     }
-    for (; j < n_splits; j += 4) {
-      const float* p = base + (size_t)j * part_stride;
-      const float mj = __ldg(p + D);
-      const float w = mj == -CUDART_INF_F ? 0.f : __expf(mj - M);
-      L = fmaf(w, __ldg(p + D + 1), L);
+    const float w = __expf(mj - Mg);
+    L = fmaf(w, lj, L);
 #pragma unroll
-      for (int k = 0; k < NB; ++k) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(p + lane * E) + k);
-        acc[4 * k + 0] = fmaf(w, x.x, acc[4 * k + 0]);
-        acc[4 * k + 1] = fmaf(w, x.y, acc[4 * k + 1]);
-        acc[4 * k + 2] = fmaf(w, x.z, acc[4 * k + 2]);
-        acc[4 * k + 3] = fmaf(w, x.w, acc[4 * k + 3]);
-      }
+    for (int k = 0; k < NB; ++k) {
+      acc[4 * k + 0] = fmaf(w, v[k].x, acc[4 * k + 0]);
+      acc[4 * k + 1] = fmaf(w, v[k].y, acc[4 * k + 1]);
+      acc[4 * k + 2] = fmaf(w, v[k].z, acc[4 * k + 2]);
+      acc[4 * k + 3] = fmaf(w, v[k].w, acc[4 * k + 3]);
     }
+  };
+  int j = grp;
+  for (; j + 4 * (UNROLL - 1) < n_splits; j += 4 * UNROLL) {
+    float mj[UNROLL], lj[UNROLL];
+    float4 v[UNROLL][NB];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const float* p = base + (size_t)(j + 4 * u) * part_stride;
+      mj[u] = __ldg(p + D);
+      lj[u] = __ldg(p + D + 1);
+#pragma unroll
+      for (int k = 0; k < NB; ++k) v[u][k] = __ldg(reinterpret_cast<const float4*>(p + lane * E) + k);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) take(mj[u], lj[u], v[u]);
   }
+  for (; j < n_splits; j += 4) {
+    const float* p = base + (size_t)j * part_stride;
+    float4 v[NB];
 #pragma unroll
-  for (int i = 0; i < E; ++i) red_acc[grp][lane * E + i] = acc[i];
-  if (lane == 0) red_l[grp] = L;
+    for (int k = 0; k < NB; ++k) v[k] = __ldg(reinterpret_cast<const float4*>(p + lane * E) + k);
+    take(__ldg(p + D), __ldg(p + D + 1), v);
+  }
+  if (lane == 0) red_m[grp] = Mg;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+  const float r = Mg == -CUDART_INF_F ? 0.f : __expf(Mg - M);  // this group's share
+#pragma unroll
+  for (int i = 0; i < E; ++i) red_acc[grp][lane * E + i] = acc[i] * r;
+  if (lane == 0) red_l[grp] = L * r;
   __syncthreads();
   if (grp != 0) return;
 
@@ -119,19 +127,35 @@ __global__ void __launch_bounds__(128)
     const int dd = lane * E + i;
     o[i] = (red_acc[0][dd] + red_acc[1][dd] + red_acc[2][dd] + red_acc[3][dd]) * inv;
   }
-  const float* hp = params + (size_t)((h % n_q_heads) / G) * D * 4;  // block matrices
   float y[E];
 #pragma unroll
-  for (int k = 0; k < NB; ++k) {
-    float M[16];
-    load_block_mat(hp, lane * NB + k, M);
-    mat_inv(M, o + 4 * k, y + 4 * k);
-  }
+  for (int k = 0; k < NB; ++k) mat_inv(Mb[k], o + 4 * k, y + 4 * k);
   wht_warp<E>(y, lane);
-  const float r = rsqrtf((float)D);
+  const float rs = rsqrtf((float)D);
   float* dst = out + ((size_t)s * rows_per_seq + h) * D + lane * E;
 #pragma unroll
-  for (int i = 0; i < E; ++i) dst[i] = y[i] * r;
+  for (int i = 0; i < E; ++i) dst[i] = y[i] * rs;
+}
+
+// The combine on `stream` as a programmatic dependent launch of the kernel before it (it
+// may start while that kernel drains; it waits in-kernel for its results).
+template <int D, bool FINAL>
+static cudaError_t launch_combine(dim3 grid, cudaStream_t stream, bool dependent,
+                                  const float* params, int H, int n_q_heads, int rows_per_seq,
+                                  int n_splits, const float* partials, size_t sh_stride,
+                                  size_t part_stride, float* out) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, FINAL>, params, H, n_q_heads,
+                            rows_per_seq, n_splits, partials, sh_stride, part_stride, out);
 }
 
 template <int D>
@@ -144,13 +168,12 @@ static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
   dim3 grid(rows, a.n_seqs);
   const size_t PS = partial_stride(D);
   if (a.state)
-    decode_combine_kernel<D, false><<<grid, 128, 0, stream>>>(
-        a.params, a.n_kv_heads, a.n_q_heads, rows, a.n_splits, a.partials, a.n_splits * PS, PS,
-        a.state);
+    e = launch_combine<D, false>(grid, stream, true, a.params, a.n_kv_heads, a.n_q_heads, rows,
+                                 a.n_splits, a.partials, a.n_splits * PS, PS, a.state);
   else
-    decode_combine_kernel<D, true><<<grid, 128, 0, stream>>>(
-        a.params, a.n_kv_heads, a.n_q_heads, rows, a.n_splits, a.partials, a.n_splits * PS, PS,
-        a.out);
+    e = launch_combine<D, true>(grid, stream, true, a.params, a.n_kv_heads, a.n_q_heads, rows,
+                                a.n_splits, a.partials, a.n_splits * PS, PS, a.out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -169,14 +192,16 @@ cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int 
   dim3 grid(n_q_heads, n_seqs);
   const size_t PS = partial_stride(d);
   const size_t slice = (size_t)n_seqs * n_q_heads * PS;
+  cudaError_t e;
   if (d == 128)
-    decode_combine_kernel<128, true><<<grid, 128, 0, stream>>>(
-        params, n_kv_heads, n_q_heads, n_q_heads, n_states, states, PS, slice, out);
+    e = launch_combine<128, true>(grid, stream, false, params, n_kv_heads, n_q_heads, n_q_heads,
+                                  n_states, states, PS, slice, out);
   else if (d == 256)
-    decode_combine_kernel<256, true><<<grid, 128, 0, stream>>>(
-        params, n_kv_heads, n_q_heads, n_q_heads, n_states, states, PS, slice, out);
+    e = launch_combine<256, true>(grid, stream, false, params, n_kv_heads, n_q_heads, n_q_heads,
+                                  n_states, states, PS, slice, out);
   else
     return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

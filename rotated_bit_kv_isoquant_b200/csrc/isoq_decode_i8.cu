@@ -574,7 +574,11 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
       if (!mbar_wait(mybar + (kk % NST), (kk / NST) & 1)) break;
   }
 
-  // ---- merge the 4 warps' states in shared memory, write the chunk's partials ---------
+  // the combine (launched as a programmatic dependent) may be scheduled from here on; it
+  // waits in-kernel until this grid has completed and its writes are visible
+  asm volatile("griddepcontrol.launch_dependents;");
+
+  // ---- merge the warps' states in shared memory, write the chunk's partials -----------
   // row rg's sum p over the lanes t (RB = 4: lanes g and g + 4 hold the same row)
 #pragma unroll
   for (int o = 1; o < 4; o <<= 1) lsum += __shfl_xor_sync(kFull, lsum, o);

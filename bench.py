@@ -38,7 +38,7 @@ SPEC_HBM_GBS = 8000.0    # B200 HBM3e specification (context for the measured co
 # the headline metric, printed identically by both arms
 METRIC = "packed-KV decode attention GB/s (% of B200 HBM peak); quantize Mvec/s"
 # what the decode's contraction computes in (operands and accumulator)
-DECODE_DTYPE = "f16 operands (query as an f16 high+low pair), f32 accumulate"
+DECODE_DTYPE = "s8xs8->s32 scores (integer codes, 3-digit query), f16xf16->f32 value sum"
 
 
 def _args():
@@ -112,9 +112,10 @@ def _tensor_peak():
 
 
 _KERNEL_SOURCES = {
-    "decode": ["isoq_decode_mma.cu", "isoq_decode.cu", "isoq_ptx.cuh", "isoq_common.cuh"],
+    "decode": ["isoq_decode_i8.cu", "isoq_decode.cu", "isoq_vtile.cuh", "isoq_ptx.cuh",
+               "isoq_common.cuh"],
     "quantize": ["isoq_quantize_tc.cu", "isoq_quantize.cu", "isoq_codes.cuh", "isoq_tc.cuh",
-                 "isoq_common.cuh"],
+                 "isoq_vtile.cuh", "isoq_common.cuh"],
 }
 
 

@@ -52,6 +52,8 @@ extern "C" {
 #define ISOQ_ST_NORM_SAT 0x8u   /* a norm >= 65520 was stored as 65504 (binary16 max) */
 #define ISOQ_ST_LEN_RANGE 0x10u /* decode: seq_len beyond the page table; clamped */
 #define ISOQ_ST_TIMEOUT 0x20u   /* decode: a bounded wait for a page copy gave up (no hang) */
+#define ISOQ_ST_BOUNDS 0x40u    /* bounds-checked build only: a kernel index fell outside its
+                                   extent; that access was skipped (see isoq_selftest_bounds) */
 
 /* ---- element types of K, V and Q ---------------------------------------------------- */
 #define ISOQ_F32 0
@@ -405,6 +407,17 @@ int isoq_last_cuda_error(void);
  * wait gave up, the completed wait succeeded), 1 for yes.  Asynchronous on `stream`.
  * Errors: ISOQ_E_ARG (null pointer, polls = 0), ISOQ_E_CUDA. */
 int isoq_selftest_bounded_wait(uint32_t* status, unsigned polls, uint32_t* result, void* stream);
+
+/* Self-test of the bounds-checked build (this build step has no counterpart in the paper;
+ * it stands in for a memory checker).  Every kernel of a library built with
+ * -DISOQ_CHECK_BOUNDS compares each computed global, shared-memory and tensor-memory index
+ * with its extent before the access; an index outside skips the access and ORs
+ * ISOQ_ST_BOUNDS into the status word.  This call launches one kernel that performs such a
+ * check on an index known to be outside (and accesses nothing), so a checked build sets
+ * ISOQ_ST_BOUNDS in *status and a normal build leaves it clear.
+ * status: device uint32.  Returns ISOQ_E_ARG for a null pointer, ISOQ_E_CUDA on a launch
+ * error, else ISOQ_OK (asynchronous on stream). */
+int isoq_selftest_bounds(uint32_t* status, void* stream);
 
 /* A static string describing an ISOQ_* return code. */
 const char* isoq_error_string(int code);

@@ -6,6 +6,11 @@ PyTorch supplies device memory and streams.  The functions carry the C names of
 ``include/isoq.h`` and raise :class:`IsoqError` on a negative return code.  Importing
 this package fails loudly if ``libisoq.so`` has not been built
 (``python rotated_bit_kv_isoquant_b200/build.py``); there is no fallback.
+
+With ``ISOQ_CHECK_BOUNDS=1`` in the environment at import, the package loads the
+bounds-checked build ``libisoq_checked.so`` (``build.py --checked``) instead: the same
+entry points, every kernel index compared with its extent, ISOQ_ST_BOUNDS set in the
+status word where one is not.
 """
 from __future__ import annotations
 
@@ -15,13 +20,14 @@ import os
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libisoq.so")
+CHECKED = os.environ.get("ISOQ_CHECK_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libisoq_checked.so" if CHECKED else "libisoq.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"libisoq.so is missing at {LIB_PATH}: build it with "
-        "`python rotated_bit_kv_isoquant_b200/build.py` (nvcc, sm_100a). "
-        "There is no CPU fallback.")
+        f"{os.path.basename(LIB_PATH)} is missing at {LIB_PATH}: build it with "
+        "`python rotated_bit_kv_isoquant_b200/build.py" + (" --checked" if CHECKED else "") +
+        "` (nvcc, sm_100a). There is no CPU fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -39,6 +45,7 @@ ISOQ_ST_PAGE_RANGE = 0x4
 ISOQ_ST_NORM_SAT = 0x8
 ISOQ_ST_LEN_RANGE = 0x10
 ISOQ_ST_TIMEOUT = 0x20
+ISOQ_ST_BOUNDS = 0x40
 
 ISOQ_F32, ISOQ_BF16, ISOQ_F16 = 0, 1, 2
 ISOQ_ROT_SO4, ISOQ_ROT_SO2 = 0, 1
@@ -95,6 +102,7 @@ _SIGS = {
     "isoq_reset_status": (_i, [_cp, _p]),
     "isoq_last_cuda_error": (_i, []),
     "isoq_selftest_bounded_wait": (_i, [_p, ctypes.c_uint, _p, _p]),
+    "isoq_selftest_bounds": (_i, [_p, _p]),
     "isoq_error_string": (ctypes.c_char_p, [_i]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -411,6 +419,17 @@ def isoq_selftest_bounded_wait(polls: int = 4096, stream=None):
     torch.cuda.synchronize()
     r = result.cpu().tolist()
     return int(status.item()) & 0xffffffff, bool(r[0]), bool(r[1])
+
+
+def isoq_selftest_bounds(stream=None) -> int:
+    """Runs the bounds-check self-test (one index equal to its extent); returns the status
+    word: ISOQ_ST_BOUNDS set by the checked build, clear in the normal one."""
+    import torch
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    _check(_lib.isoq_selftest_bounds(status.data_ptr(), _stream_ptr(stream)),
+           "isoq_selftest_bounds")
+    torch.cuda.synchronize()
+    return int(status.item()) & 0xffffffff
 
 
 def isoq_error_string(code: int) -> str:

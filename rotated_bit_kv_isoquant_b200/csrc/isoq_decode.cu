@@ -13,6 +13,7 @@
 // starts at -inf).
 #include <math_constants.h>
 
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 
@@ -32,7 +33,8 @@ template <int D, bool FINAL>
 __global__ void __launch_bounds__(128)
     decode_combine_kernel(const float* __restrict__ params, int H, int n_q_heads,
                           int rows_per_seq, int n_splits, const float* __restrict__ partials,
-                          size_t sh_stride, size_t part_stride, float* __restrict__ out) {
+                          size_t sh_stride, size_t part_stride, float* __restrict__ out,
+                          size_t parts_len, uint32_t* status) {
   constexpr int E = D / 32;   // dims per lane
   constexpr int NB = E / 4;
   constexpr int PS = D + 4;
@@ -77,6 +79,11 @@ __global__ void __launch_bounds__(128)
       acc[4 * k + 3] = fmaf(w, v[k].w, acc[4 * k + 3]);
     }
   };
+  // checked build: every part read lies inside the partials (parts_len floats)
+  [[maybe_unused]] const size_t base_off = base - partials;
+  if (!in_bounds(base_off + (size_t)(n_splits > 0 ? n_splits - 1 : 0) * part_stride + PS <= parts_len,
+                 status))
+    n_splits = 0;
   int j = grp;
   for (; j + 4 * (UNROLL - 1) < n_splits; j += 4 * UNROLL) {
     float mj[UNROLL], lj[UNROLL];
@@ -143,7 +150,8 @@ template <int D, bool FINAL>
 static cudaError_t launch_combine(dim3 grid, cudaStream_t stream, bool dependent,
                                   const float* params, int H, int n_q_heads, int rows_per_seq,
                                   int n_splits, const float* partials, size_t sh_stride,
-                                  size_t part_stride, float* out) {
+                                  size_t part_stride, float* out, size_t parts_len,
+                                  uint32_t* status) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(128);
@@ -155,7 +163,8 @@ static cudaError_t launch_combine(dim3 grid, cudaStream_t stream, bool dependent
   cfg.attrs = attr;
   cfg.numAttrs = dependent ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, FINAL>, params, H, n_q_heads,
-                            rows_per_seq, n_splits, partials, sh_stride, part_stride, out);
+                            rows_per_seq, n_splits, partials, sh_stride, part_stride, out,
+                            parts_len, status);
 }
 
 template <int D>
@@ -167,12 +176,15 @@ static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
   const int rows = a.n_q * a.n_q_heads;
   dim3 grid(rows, a.n_seqs);
   const size_t PS = partial_stride(D);
+  const size_t parts_len = (size_t)a.n_seqs * rows * a.n_splits * PS;
   if (a.state)
     e = launch_combine<D, false>(grid, stream, true, a.params, a.n_kv_heads, a.n_q_heads, rows,
-                                 a.n_splits, a.partials, a.n_splits * PS, PS, a.state);
+                                 a.n_splits, a.partials, a.n_splits * PS, PS, a.state, parts_len,
+                                 a.status);
   else
     e = launch_combine<D, true>(grid, stream, true, a.params, a.n_kv_heads, a.n_q_heads, rows,
-                                a.n_splits, a.partials, a.n_splits * PS, PS, a.out);
+                                a.n_splits, a.partials, a.n_splits * PS, PS, a.out, parts_len,
+                                a.status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -195,10 +207,10 @@ cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int 
   cudaError_t e;
   if (d == 128)
     e = launch_combine<128, true>(grid, stream, false, params, n_kv_heads, n_q_heads, n_q_heads,
-                                  n_states, states, PS, slice, out);
+                                  n_states, states, PS, slice, out, slice * n_states, nullptr);
   else if (d == 256)
     e = launch_combine<256, true>(grid, stream, false, params, n_kv_heads, n_q_heads, n_q_heads,
-                                  n_states, states, PS, slice, out);
+                                  n_states, states, PS, slice, out, slice * n_states, nullptr);
   else
     return cudaErrorInvalidValue;
   if (e != cudaSuccess) return e;

@@ -43,6 +43,7 @@
 
 #include <type_traits>
 
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
@@ -211,12 +212,18 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
   const int p_end = min((lim_hi + kPage - 1) / kPage, p_begin + pages_per_split);
 
   float* out_base = partials + ((size_t)s * n_q * n_q_heads) * n_splits * PS + (size_t)split * PS;
+  // extents of the checked build: partials / Q rows of the launch, the head's parameters
+  [[maybe_unused]] const size_t parts_len = (size_t)gridDim.z * n_q * n_q_heads * n_splits * PS;
+  [[maybe_unused]] const size_t q_rows = (size_t)gridDim.z * n_q * n_q_heads;
+  [[maybe_unused]] const size_t out_off0 = out_base - partials;
   if (tid < RB) row_off[tid] = tid < nh ? row_index(tid) : 0;
   __syncthreads();
   if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
     for (int i = tid; i < nh * PS; i += blockDim.x) {
       const int h = i / PS, c = i - h * PS;
-      out_base[(size_t)row_off[h] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+      const size_t o = (size_t)row_off[h] * n_splits * PS + c;
+      if (in_bounds(out_off0 + o < parts_len, status))
+        out_base[o] = (c == D) ? -CUDART_INF_F : 0.f;
     }
     return;
   }
@@ -235,8 +242,8 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
   auto issue = [&](int k) {  // lane 0 only
     const int pg = p_begin + warp + NW * k;
     const int st = k % NST;
-    const int phys = __ldg(pt_row + pg);
-    if (phys >= 0 && phys < n_pages) {
+    const int phys = in_bounds(pg < max_pages && st < NST, status) ? __ldg(pt_row + pg) : -1;
+    if (phys >= 0 && phys < n_pages && in_bounds(hk < H, status)) {
       mbar_expect_tx(mybar + st, BB);
       bulk_copy(myring + st * BB, blocks + ((size_t)phys * H + hk) * BB, BB, mybar + st);
     } else {
@@ -256,13 +263,16 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
     const float* hp = params + (size_t)hk * D * 4;  // this head's block matrices
     float pq[NB][16];
 #pragma unroll
-    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, pq[k]);
+    for (int k = 0; k < NB; ++k)
+      if (in_bounds(hk < H && lane * NB + k < D / 4, status)) load_block_mat(hp, lane * NB + k, pq[k]);
     for (int r = warp; r < RB; r += NW) {
       float v[E];
       if (r < nh) {
         const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[r]) * D + lane * E;
 #pragma unroll
-        for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
+        for (int i = 0; i < E; ++i)
+          v[i] = in_bounds((size_t)s * n_q * n_q_heads + row_off[r] < q_rows, status)
+                     ? to_f32<TQ>(qp[i]) : 0.f;
       } else {
 #pragma unroll
         for (int i = 0; i < E; ++i) v[i] = 0.f;
@@ -278,7 +288,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
       const float S = amax > 0.f ? kQMax / amax : 0.f;
       // log2 score per (integer score / 2^16 * nK): the unnormalised WHT makes z = sqrt(d)
       // q~ and K_hat = (nK / sqrt(d)) L, so q~.K_hat = nK (score / (S 10000)) / d
-      if (lane == 0)
+      if (lane == 0 && in_bounds(r < 8, status))
         kf_row[r] = S > 0.f ? scale * kLog2e * 65536.0f / (kLevelScale * (float)D * S) : 0.f;
       // this lane's E dims: lane * E .. + E-1 = E/4 runs of 4 dims (one A register each)
 #pragma unroll
@@ -294,6 +304,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
         // selects a0/a1 (dims +0..3) or a2/a3 (dims +4..7)
         const int q = base >> 5, u = (base >> 3) & 3, hf = (base >> 2) & 1;
         const int kb = 4 * (q >> 2) + u, tq = q & 3;
+        if (!in_bounds(kb < D / 32 && r < RB && tq < 4, status)) continue;
         if constexpr (RB == 8) {
           // lane (g' = r, t' = tq): A1 = (d2, d1, d2+4, d1+4), A2 = (d0, d0+4)
           uint32_t* f = afr + (kb * 32 + 4 * r + tq) * 4;
@@ -358,7 +369,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
     }
     const uint8_t* blk = myring + st * BB;
     const int pg = p_begin + warp + NW * k;
-    const int phys = __ldg(pt_row + pg);
+    const int phys = in_bounds(pg < max_pages && st < NST, status) ? __ldg(pt_row + pg) : -1;
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
 
@@ -378,17 +389,21 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
           uint32_t w[kI8NT][3];
 #pragma unroll
           for (int nn = 0; nn < kI8NT; ++nn) {
-            const uint32_t* p = reinterpret_cast<const uint32_t*>(
-                                    blk + (tb + 8 * (n0 + nn) + g) * CB) + 3 * (t + 4 * gq);
-            w[nn][0] = p[0];
-            w[nn][1] = p[1];
-            w[nn][2] = p[2];
+            const int ko = (tb + 8 * (n0 + nn) + g) * CB + 12 * (t + 4 * gq);
+            const uint32_t* p = reinterpret_cast<const uint32_t*>(blk + ko);
+            const bool kin = in_bounds(ko + 12 <= kPage * CB, status);
+            w[nn][0] = kin ? p[0] : 0u;
+            w[nn][1] = kin ? p[1] : 0u;
+            w[nn][2] = kin ? p[2] : 0u;
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int kb = 4 * gq + u;
-            const uint4 A1 = *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4);
-            const uint4 A2 = *reinterpret_cast<const uint4*>(afr2 + (kb * 32 + lane) * 4);
+            const bool ain = in_bounds(kb < D / 32, status);
+            const uint4 A1 = ain ? *reinterpret_cast<const uint4*>(afr + (kb * 32 + lane) * 4)
+                                 : make_uint4(0, 0, 0, 0);
+            const uint4 A2 = ain ? *reinterpret_cast<const uint4*>(afr2 + (kb * 32 + lane) * 4)
+                                 : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int nn = 0; nn < kI8NT; ++nn) {
               const uint32_t S = u == 0 ? (w[nn][0] & 0x77777777u)
@@ -419,8 +434,9 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
         for (int nn = 0; nn < kI8NT; ++nn) {
           const int n = n0 + nn;
           const int tk = tb + 8 * n + 2 * t;
-          const float2 nk2 = __half22float2(
-              *reinterpret_cast<const __half2*>(blk + k_norm_off(D, 3) + 2 * tk));
+          const float2 nk2 = in_bounds(tk + 2 <= kPage, status)
+              ? __half22float2(*reinterpret_cast<const __half2*>(blk + k_norm_off(D, 3) + 2 * tk))
+              : make_float2(0.f, 0.f);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             float raw;
@@ -447,8 +463,9 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
         const int tk = tb + 8 * n + 2 * t;
-        const float2 nv2 = __half22float2(
-            *reinterpret_cast<const __half2*>(blk + v_norm_off(D, 3) + 2 * tk));
+        const float2 nv2 = in_bounds(tk + 2 <= kPage, status)
+            ? __half22float2(*reinterpret_cast<const __half2*>(blk + v_norm_off(D, 3) + 2 * tk))
+            : make_float2(0.f, 0.f);
         nv[n][0] = nv2.x;
         nv[n][1] = nv2.y;
         if constexpr (!FULL) {
@@ -516,18 +533,18 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
       }
 
       // ---- a8: V accumulation, A = V_hat^T (rows = dims, k = the block's tokens) --------
-      const uint8_t* vbase = blk + v_codes_off(D, 3) + (tb >> 4) * 6 * D;
 #pragma unroll
       for (int up = 0; up < NU; ++up) {
 #pragma unroll
         for (int jb = 0; jb < 2; ++jb) {
           // this lane's 24 bytes of the 16-token block: units 2 (g + 8 up), +1 of quad t
           uint32_t W[6];
-          const uint2* src = reinterpret_cast<const uint2*>(
-              vbase + jb * 6 * D + vt_group_off(D, 0, t, 2 * (g + 8 * up)));
+          const int vo = ((tb >> 4) + jb) * 6 * D + vt_group_off(D, 0, t, 2 * (g + 8 * up));
+          const uint2* src = reinterpret_cast<const uint2*>(blk + v_codes_off(D, 3) + vo);
+          const bool vin = in_bounds(vo + 24 <= kPage * CB, status);
 #pragma unroll
           for (int i = 0; i < 3; ++i) {
-            const uint2 w = src[i];
+            const uint2 w = vin ? src[i] : make_uint2(0, 0);
             W[2 * i] = w.x;
             W[2 * i + 1] = w.y;
           }
@@ -598,6 +615,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
           for (int b = 0; b < 4; ++b) {
             const int mt = 8 * up + 4 * p + b;
             const int d0 = 8 * (2 * (g + 8 * up) + p) + 2 * b;
+            if (!in_bounds(d0 + 1 < D && 2 * t + 1 < 8, status)) continue;
             float* r0 = mb + (warp * 8 + 2 * t) * PS;
             float* r1 = mb + (warp * 8 + 2 * t + 1) * PS;
             r0[d0] = acc[mt][0] * f;
@@ -629,6 +647,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
       }
     }
     float* o = out_base + (size_t)row_off[h] * n_splits * PS;
+    if (!in_bounds(out_off0 + (size_t)row_off[h] * n_splits * PS + D + 1 < parts_len, status)) continue;
     if (c < D) o[c] = v;
     else {
       o[D] = M == -CUDART_INF_F ? -CUDART_INF_F : M / kLog2e;  // natural-log units

@@ -22,6 +22,7 @@
 // The partial results have the layout of the per-row kernel and go to the same combine.
 #include <math_constants.h>
 
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
@@ -116,7 +117,8 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
   if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
     for (int i = tid; i < nh * PS; i += blockDim.x) {
       const int r = i / PS, c = i - r * PS;
-      out_base[(size_t)row_off[r] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+      if (in_bounds(row_off[r] < n_q * n_q_heads, status))
+        out_base[(size_t)row_off[r] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
     }
     return;
   }
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
   const int n_my = p_end - p_begin;
   auto issue = [&](int k) {  // thread 0
     const int st = k & 1;
-    const int phys = __ldg(pt_row + p_begin + k);
+    const int phys = in_bounds(p_begin + k < max_pages, status) ? __ldg(pt_row + p_begin + k) : -1;
     uint64_t* bar = bars + st;
     if (phys >= 0 && phys < n_pages) {
       mbar_expect_tx(bar, BB);
@@ -156,7 +158,10 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
     for (int r = warp; r < 64; r += kMqWarps) {
       float v[E];
       if (r < nh) {
-        const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[r]) * D + lane * E;
+        const TQ* qp = Q + ((size_t)s * n_q * n_q_heads +
+                            (in_bounds(row_off[r] < n_q * n_q_heads, status) ? row_off[r] : 0)) *
+                               D +
+                       lane * E;
 #pragma unroll
         for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
       } else {
@@ -214,18 +219,23 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
           const int B = u >> 6, t4 = (u >> 4) & 3, un = u & 15;
           const uint32_t* wp = reinterpret_cast<const uint32_t*>(
               blk + v_codes_off(D, BITS) + vt_group_off(D, B, t4, un));
+          if (!in_bounds(vt_group_off(D, B, t4, un) + 12 <= kPage * CB, status)) continue;
           uint32_t o[4][4];
           vdeq_group(wp[0], wp[1], wp[2], tl0, tl1, th0, th1, o);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 4; ++j) {
+            if (!in_bounds(tile_off(vt_member_slot(B, t4, j), un) + 16 <= 64 * D * 2, status))
+              continue;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                              base + tile_off(vt_member_slot(B, t4, j), un)),
                          "r"(o[j][0]), "r"(o[j][1]), "r"(o[j][2]), "r"(o[j][3])
                          : "memory");
+          }
           continue;
         }
         const uint32_t* wp = reinterpret_cast<const uint32_t*>(blk + (kv ? v_codes_off(D, BITS) : 0) +
                                                              tk * CB) + W * q;
+        if (!in_bounds(tk * CB + 4 * W * (q + 1) <= kPage * CB, status)) continue;
         uint32_t w[W];
 #pragma unroll
         for (int i = 0; i < W; ++i) w[i] = wp[i];
@@ -233,6 +243,7 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
         for (int j = 0; j < 4; ++j) {
           uint32_t o[4];
           kdeq<BITS>(w, j, tl0, tl1, th0, th1, o);
+          if (!in_bounds(tile_off(tk, 4 * q + j) + 16 <= 64 * D * 2, status)) continue;
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + tile_off(tk, 4 * q + j)),
                        "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
                        : "memory");
@@ -276,7 +287,7 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
       dequant(k + 1);
     }
     const int pg = p_begin + k;
-    const int phys = __ldg(pt_row + pg);
+    const int phys = in_bounds(pg < max_pages, status) ? __ldg(pt_row + pg) : -1;
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
     const uint32_t sK = sTile + (k & 1) * SM::kTileBytes, sV = sK + 64 * D * 2;
@@ -447,7 +458,7 @@ __global__ void __launch_bounds__(kMqWarps * 32, 2)
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       const int r = 8 * (b ? rbB : rbA) + g;
-      if (r >= nh) continue;
+      if (r >= nh || !in_bounds(row_off[r] < n_q * n_q_heads, status)) continue;
       float* o = out_base + (size_t)row_off[r] * n_splits * PS;
 #pragma unroll
       for (int n = 0; n < 16; ++n) {

@@ -27,6 +27,7 @@
 
 #include <type_traits>
 
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
@@ -41,6 +42,8 @@ constexpr int kXD = 128;    // head dimension
 constexpr int kXRows = 128; // rows per CTA = threads per CTA
 constexpr uint32_t kXCols = 256;  // tensor-memory columns: S 64 | O 128 | P' 32
 constexpr uint32_t kColS = 0, kColO = 64, kColP = 192;
+static_assert(kColS + 64 <= kColO && kColO + 128 <= kColP && kColP + 32 <= kXCols,
+              "tensor-memory columns overlap or exceed the allocation");
 
 // Shared memory (bytes).  Operand tiles, no swizzle, core matrix = 8 rows x 16 bytes:
 //   Q~ hi / lo (A, K-major, 128 rows x 128 dims): (k/8) 2048 + (m/8) 128 + (m%8) 16 + (k%8) 2
@@ -123,7 +126,8 @@ __global__ void __launch_bounds__(kXRows, 2)
   if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
     for (int i = tid; i < nh * PS; i += blockDim.x) {
       const int r = i / PS, c = i - r * PS;
-      out_base[(size_t)row_off[r] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+      if (in_bounds(row_off[r] < n_q * n_q_heads, status))
+        out_base[(size_t)row_off[r] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
     }
     return;
   }
@@ -134,7 +138,7 @@ __global__ void __launch_bounds__(kXRows, 2)
   if (warp == 0) tc::alloc(tmem_slot, kXCols);
   auto issue = [&](int k) {  // thread 0
     const int st = k & 1;
-    const int phys = __ldg(pt_row + p_begin + k);
+    const int phys = in_bounds(p_begin + k < max_pages, status) ? __ldg(pt_row + p_begin + k) : -1;
     if (phys >= 0 && phys < n_pages) {
       mbar_expect_tx(bars + st, BB);
       bulk_copy(smem + SM::kOffRing + st * BB, blocks + ((size_t)phys * H + hk) * BB, BB, bars + st);
@@ -159,7 +163,7 @@ __global__ void __launch_bounds__(kXRows, 2)
     for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, M[k]);
     for (int r = warp; r < kXRows; r += 4) {
       float v[E];
-      if (r < nh) {
+      if (r < nh && in_bounds(row_off[r] < n_q * n_q_heads, status)) {
         const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[r]) * D + lane * E;
 #pragma unroll
         for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
@@ -174,6 +178,7 @@ __global__ void __launch_bounds__(kXRows, 2)
       // dims 4 lane .. 4 lane + 3: half of one 16-byte core-matrix row
       const int k0 = lane * E;
       const uint32_t off = (k0 >> 3) * 2048 + (r >> 3) * 128 + (r & 7) * 16 + (k0 & 7) * 2;
+      if (!in_bounds(off + 8 <= SM::kOffQl - SM::kOffQh, status)) continue;
       float hi[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) hi[e] = __half2float(__float2half_rn(z[e]));
@@ -213,11 +218,14 @@ __global__ void __launch_bounds__(kXRows, 2)
         const int B = u >> 6, t4 = (u >> 4) & 3, un = u & 15;
         const uint32_t* wp = reinterpret_cast<const uint32_t*>(
             blk + v_codes_off(D, BITS) + vt_group_off(D, B, t4, un));
+        if (!in_bounds(vt_group_off(D, B, t4, un) + 12 <= kPage * CB, status)) continue;
         uint32_t o[4][4];
         vdeq_group(wp[0], wp[1], wp[2], tl0, tl1, th0, th1, o);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int tkj = vt_member_slot(B, t4, j);
+          const int vo = (tkj >> 3) * 2048 + un * 128 + (tkj & 7) * 16;
+          if (!in_bounds(vo + 16 <= SM::kOffRing - SM::kOffV, status)) continue;
           st_v4(sV + (tkj >> 3) * 2048 + un * 128 + (tkj & 7) * 16, o[j]);
         }
         continue;
@@ -228,6 +236,7 @@ __global__ void __launch_bounds__(kXRows, 2)
       const int tk = 8 * (u >> 5) + (u & 7), q = (u >> 3) & 3;
       const uint32_t* wp = reinterpret_cast<const uint32_t*>(
                                blk + (kv ? v_codes_off(D, BITS) : 0) + tk * CB) + W * q;
+      if (!in_bounds(tk * CB + 4 * W * (q + 1) <= kPage * CB, status)) continue;
       uint32_t w[W];
 #pragma unroll
       for (int i = 0; i < W; ++i) w[i] = wp[i];
@@ -236,8 +245,11 @@ __global__ void __launch_bounds__(kXRows, 2)
         uint32_t o[4];
         kdeq<BITS>(w, j, tl0, tl1, th0, th1, o);  // dims 32q + 8j .. +7 of token tk
         const int c = 4 * q + j;
-        const uint32_t addr = kv ? sV + (tk >> 3) * 2048 + c * 128 + (tk & 7) * 16
-                                 : sK + c * 1024 + (tk >> 3) * 128 + (tk & 7) * 16;
+        const uint32_t to = kv ? (tk >> 3) * 2048 + c * 128 + (tk & 7) * 16
+                               : c * 1024 + (tk >> 3) * 128 + (tk & 7) * 16;
+        if (!in_bounds(to + 16 <= (kv ? SM::kOffRing - SM::kOffV : SM::kOffV - SM::kOffK), status))
+          continue;
+        const uint32_t addr = (kv ? sV : sK) + to;
         st_v4(addr, o);
       }
     }
@@ -451,12 +463,13 @@ __global__ void __launch_bounds__(kXRows, 2)
     } else {
       tc::fence_after();
       float* o = out_base + (size_t)row_off[tid] * n_splits * PS;
+      const bool w_ok = tid < nh && in_bounds(row_off[tid] < n_q * n_q_heads, status);
       const float f = sigma / ALPHA;  // O holds sum p |v| ALPHA L / sigma
       uint32_t ov[32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         tc::ld32(t_row + kColO + 32 * c, ov);  // warp-collective: every lane loads
-        if (tid < nh) {
+        if (w_ok) {
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(o + 32 * c + j) =
@@ -464,7 +477,7 @@ __global__ void __launch_bounds__(kXRows, 2)
                             __uint_as_float(ov[j + 2]) * f, __uint_as_float(ov[j + 3]) * f);
         }
       }
-      if (tid < nh) {
+      if (w_ok) {
         o[D] = m2 == -CUDART_INF_F ? -CUDART_INF_F : m2 / kLog2e;  // natural-log units
         o[D + 1] = lsum;
       }

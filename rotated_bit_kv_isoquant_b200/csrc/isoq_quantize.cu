@@ -16,6 +16,7 @@
 // stores.
 #include <math_constants.h>
 
+#include "isoq_check.cuh"
 #include "isoq_codes.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
@@ -70,6 +71,7 @@ __global__ void __launch_bounds__(256)
     }
     const int slot = pos & (kPage - 1);
 
+    if (!in_bounds(phys < n_pages && slot < kPage, status)) continue;
     for (int h = 0; h < H; ++h) {
       uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
       const size_t row = ((size_t)t * H + h) * D + lane * E;
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(256)
         }
         if (kv == 0) {
           uint8_t* dst = blk + slot * CB;
-          if (lane < CB / 16)
+          if (lane < CB / 16 && in_bounds(slot * CB + 16 * lane + 16 <= kPage * CB, status))
             *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
         } else {
           // V in the tile layout: the unit word of unit u (dims 8u..8u+7) is lane u's
@@ -217,10 +219,12 @@ __global__ void __launch_bounds__(256)
             uint32_t W[3], mask;
             vt_member_words(U, j, W, mask);
             uint32_t* g = reinterpret_cast<uint32_t*>(blk + v_codes_off(D) + vt_group_off(D, B, t, u));
+            if (in_bounds(vt_group_off(D, B, t, u) + 12 <= kPage * CB, status)) {
 #pragma unroll
-            for (int w = 0; w < 3; ++w) {
-              atomicAnd(g + w, ~mask);
-              atomicOr(g + w, W[w]);
+              for (int w = 0; w < 3; ++w) {
+                atomicAnd(g + w, ~mask);
+                atomicOr(g + w, W[w]);
+              }
             }
           }
         }
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
 #pragma unroll
         for (int j = 0; j < 3; ++j) rec[3 * g + j] = nib[4 * g + j] | ((N3 << (j + 1)) & 0x88888888u);
       }
-      if (kind == 1) {  // V: the unit words, for the V tile layout
+      if (kind == 1 && in_bounds(D / 8 <= kTpvStage, status)) {  // V: the unit words
 #pragma unroll
         for (int q = 0; q < D / 32; ++q)
           *reinterpret_cast<uint4*>(stage + 4 * q) =
@@ -472,6 +476,7 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
       set_status(status, ISOQ_ST_PAGE_RANGE);
       valid = false;
     }
+    if (valid && !in_bounds(h < H && (pos & (kPage - 1)) < kPage, status)) valid = false;
     if (!valid) phys = -1;
     if (valid) {
       uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
@@ -494,7 +499,8 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
     if constexpr (BITS == 3) {
       if (kind == 1) {  // warp-uniform: the task is the warp's
         __syncwarp();
-        vt_store_warp<D, kTpvStage>(stage - lane * kTpvStage, lane, sid, pos, phys, blocks, H, h);
+        vt_store_warp<D, kTpvStage>(stage - lane * kTpvStage, lane, sid, pos, phys, blocks, H, h,
+                                    status);
         __syncwarp();  // the stage is rewritten by the next task
       }
     }

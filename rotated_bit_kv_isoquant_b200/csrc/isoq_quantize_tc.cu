@@ -27,6 +27,7 @@
 
 #include <type_traits>
 
+#include "isoq_check.cuh"
 #include "isoq_codes.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(kQtThreads, 2)
   const uint32_t cp_dst = qt_off(cp_row, 8 * cp_j);
   const size_t row_bytes = (size_t)H * D * sizeof(T);
   auto prefetch = [&](Tile t, int li) {
-    if (t.chunk < n_chunks) {
+    if (t.chunk < n_chunks && in_bounds((t.rr >> 1) < H, status)) {
       const int h = t.rr >> 1;
       const int t0 = t.chunk * kQtRows;
       const uint8_t* src = ((t.rr & 1) ? Vb : Kb) + (size_t)(t0 + cp_row) * row_bytes +
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(kQtThreads, 2)
       float2 s01 = make_float2(0.f, 0.f), s23 = make_float2(0.f, 0.f);  // four partial sums
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
+        if (!in_bounds((li & 1) * 128 + 64 * hh + 64 <= (int)kQtCols, status)) break;
         tc::ld64(acc + 64 * hh, y);
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
@@ -325,7 +327,8 @@ __global__ void __launch_bounds__(kQtThreads, 2)
           for (int j = 0; j < 4; ++j) nib[j] = join_halves(half[8 * gg + 2 * j], half[8 * gg + 2 * j + 1]);
 #pragma unroll
           for (int j = 0; j < 3; ++j) rec[3 * gg + j] = nib[j] | ((nib[3] << (j + 1)) & 0x88888888u);
-          if (kind == 1)  // V: the unit words 8 hf + 4 gg .. +3, for the V tile layout
+          if (kind == 1 && in_bounds(8 * hf + 4 * gg + 4 <= kStageWords, status))
+            // V: the unit words 8 hf + 4 gg .. +3, for the V tile layout
             *reinterpret_cast<uint4*>(stage + 8 * hf + 4 * gg) =
                 make_uint4(nib[0], nib[1], nib[2], nib[3]);
         }
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kQtThreads, 2)
         for (int j = 0; j < NR; ++j) rec[j] = join_halves(half[2 * j], half[2 * j + 1]);
       }
 
-      if (phys >= 0) {
+      if (phys >= 0 && in_bounds(phys < n_pages && h < H && (CB / 2) * (hf + 1) <= CB, status)) {
         uint8_t* blk = blocks + ((size_t)phys * H + h) * BB;
         const int slot = pos & (kPage - 1);
         uint8_t* dst = blk + (kind == 0 ? 0 : v_codes_off(D, BITS)) + slot * CB + (CB / 2) * hf;
@@ -368,7 +371,8 @@ __global__ void __launch_bounds__(kQtThreads, 2)
     if constexpr (BITS == 3) {
       if (kind == 1) {  // CTA-uniform
         __syncwarp();
-        vt_store_warp<kQtD, kStageWords>(stage - lane * kStageWords, lane, sid, pos, phys, blocks, H, h);
+        vt_store_warp<kQtD, kStageWords>(stage - lane * kStageWords, lane, sid, pos, phys, blocks, H, h,
+                                         status);
       }
     }
     if (has_next) {

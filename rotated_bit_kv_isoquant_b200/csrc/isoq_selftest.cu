@@ -2,6 +2,7 @@
 // an mbarrier phase that nothing completes is awaited with a short poll limit, the wait
 // gives up, and the give-up is reported in the status word exactly as a kernel reports a
 // page copy that never lands; a phase that does complete is observed as completed.
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
@@ -23,6 +24,15 @@ __global__ void bounded_wait_selftest_kernel(uint32_t* status, unsigned polls, u
   result[1] = done ? 1u : 0u;
 }
 
+// An index check on an index outside its extent (index 8 of an 8-element buffer): nothing
+// is accessed; the checked build reports it.
+__global__ void bounds_selftest_kernel(uint32_t* status, int index, int extent) {
+  if (threadIdx.x != 0) return;
+  if (in_bounds(index < extent, status)) {
+    // an access at index would go here
+  }
+}
+
 }  // namespace
 }  // namespace isoq
 
@@ -31,6 +41,13 @@ extern "C" int isoq_selftest_bounded_wait(uint32_t* status, unsigned polls, uint
   if (!status || !result || polls == 0) return ISOQ_E_ARG;
   isoq::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       status, polls, result);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ISOQ_OK : isoq::record_cuda_error(e);
+}
+
+extern "C" int isoq_selftest_bounds(uint32_t* status, void* stream) {
+  if (!status) return ISOQ_E_ARG;
+  isoq::bounds_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status, 8, 8);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ISOQ_OK : isoq::record_cuda_error(e);
 }

@@ -15,6 +15,7 @@
 
 #include <stdint.h>
 
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 
 namespace isoq {
@@ -81,7 +82,8 @@ __device__ __forceinline__ void vt_member_words(uint32_t U, int j, uint32_t (&W)
 // this, after their unit words are in shared memory and a __syncwarp.
 template <int D, int SW>
 __device__ __forceinline__ void vt_store_warp(const uint32_t* warp_stage, int lane, int sid,
-                                              int pos, int phys, uint8_t* blocks, int H, int h) {
+                                              int pos, int phys, uint8_t* blocks, int H, int h,
+                                              uint32_t* status = nullptr) {
   constexpr int BB = block_bytes(D, 3);
   constexpr int NU = D / 8;  // units
   const int hb = lane & 16, hl = lane & 15;  // half-warp base lane, position in it
@@ -98,6 +100,9 @@ __device__ __forceinline__ void vt_store_warp(const uint32_t* warp_stage, int la
                   vt_group_off(D, (p0 & (kPage - 1)) >> 4, 0, 0);
 #pragma unroll
     for (int m = hl >> 2; m < NU / 4; m += 4) {
+      if (!in_bounds(4 * m + 4 <= SW && h < H && vt_group_off(D, 0, t, 4 * m + 3) + 12 <= 6 * D,
+                     status))
+        continue;
       uint4 U[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -127,6 +132,9 @@ __device__ __forceinline__ void vt_store_warp(const uint32_t* warp_stage, int la
       uint32_t W[3], mask;
       vt_member_words(mine[u], j, W, mask);
       uint32_t* g = reinterpret_cast<uint32_t*>(vb + vt_group_off(D, B, t, u));
+      if (!in_bounds(u < SW && h < H && vt_group_off(D, B, t, u) + 12 <= kPage * code_bytes(D, 3),
+                     status))
+        continue;
 #pragma unroll
       for (int w = 0; w < 3; ++w) {
         atomicAnd(g + w, ~mask);

@@ -31,6 +31,16 @@ def test_exports_every_declared_symbol():
     assert not missing, missing
 
 
+def test_checked_build_exports_every_declared_symbol():
+    """The bounds-checked variant (build.py --checked) has the same entry points."""
+    path = os.path.join(ROOT, "rotated_bit_kv_isoquant_b200", "libisoq_checked.so")
+    if not os.path.exists(path):
+        pytest.skip("libisoq_checked.so not built")
+    lib = ctypes.CDLL(path)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
 @pytest.mark.parametrize("seed,d,h", [(0, 128, 2), (0, 128, 8), (0, 256, 8), (12345, 128, 3),
                                       (2**63 + 7, 256, 1)])
 def test_params_generator_matches_oracle_bitwise(oracle, seed, d, h):

@@ -27,7 +27,8 @@
 // through a private ring of shared-memory stages filled by 1-D bulk copies (one page
 // block per copy, completion on an mbarrier, every wait bounded).  Per 32-token tile:
 //   scores  C[16 x 8 tokens] = A[16 x 32 dims] . K_hat^T, m16n8k32 s8, 4 tiles of 8 tokens:
-//           RB = 8: A = [d2; d1] against kh and kl, [d0; 0] against kh (3 mma per k-step);
+//           RB = 8: A = [d2; d1] against kh and kl, [0; d0] against kh added to the kl
+//           product (3 mma per k-step, two accumulators);
 //           RB = 4: A = [d2; d1; d0; 0] against kh, [d2; d1; 0; 0] against kl (2 mma).
 //           Lane t of a quad owns 32-dim group t of every token (the k order inside a
 //           k-step is a permutation of the dims, the query digits follow it).
@@ -139,15 +140,20 @@ struct I8Smem {
 #define ISOQ_I8_MINB128 4
 #endif
 #ifndef ISOQ_I8_NT  // 8-token score tiles per load of the query fragments (1, 2 or 4)
-#define ISOQ_I8_NT 4
+#define ISOQ_I8_NT 2
 #endif
 constexpr int kI8NT = ISOQ_I8_NT;
 static_assert(4 % kI8NT == 0, "score tiles per fragment load");
 
 // CTAs per SM the register budget is set for: 4-warp CTAs as many as fit (d = 128: 4, d =
 // 256: 2); the wide CTAs of small grids (one per SM) get the same per-thread budget.
+#ifndef ISOQ_I8_MINB256
+#define ISOQ_I8_MINB256 2
+#endif
 template <int D>
-constexpr int i8_min_blocks(int nw) { return nw == 4 ? (D == 128 ? ISOQ_I8_MINB128 : 2) : 1; }
+constexpr int i8_min_blocks(int nw) {
+  return nw == 4 ? (D == 128 ? ISOQ_I8_MINB128 : ISOQ_I8_MINB256) : 1;
+}
 
 
 // MQ: chunks of several query tokens per sequence with causal limits; the decode (one
@@ -306,13 +312,13 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
         const int kb = 4 * (q >> 2) + u, tq = q & 3;
         if (!in_bounds(kb < D / 32 && r < RB && tq < 4, status)) continue;
         if constexpr (RB == 8) {
-          // lane (g' = r, t' = tq): A1 = (d2, d1, d2+4, d1+4), A2 = (d0, d0+4)
+          // lane (g' = r, t' = tq): A1 = (d2, d1, d2+4, d1+4), A2 = (0, d0, 0, d0+4)
           uint32_t* f = afr + (kb * 32 + 4 * r + tq) * 4;
           f[2 * hf] = w2;
           f[2 * hf + 1] = w1;
-          uint32_t* f2 = afr2 + (kb * 32 + 4 * r + tq) * 4;  // A2 = [d0; 0]
-          f2[2 * hf] = w0;
-          f2[2 * hf + 1] = 0u;
+          uint32_t* f2 = afr2 + (kb * 32 + 4 * r + tq) * 4;  // A2 = [0; d0]
+          f2[2 * hf] = 0u;
+          f2[2 * hf + 1] = w0;
         } else {
           // A1: rows 0-3: d2 of rows r, 4-7: d1, 8-11: d0 (12-15 zero); A2: the same
           // without d0.  Lanes g' = r and r + 4.
@@ -382,8 +388,8 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
       float sv[4][2];  // log2-domain scores of tokens tb + 8n + 2t + c (row rg)
 #pragma unroll
       for (int n0 = 0; n0 < 4; n0 += kI8NT) {
+        // RB = 8: C1 = [d2.kh; d1.kh], C2 = [d2.kl; d1.kl + d0.kh]
         int C1[kI8NT][4], C2[kI8NT][4];
-        [[maybe_unused]] int C3[kI8NT][4];
 #pragma unroll
         for (int gq = 0; gq < NG; ++gq) {
           uint32_t w[kI8NT][3];
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
                 mma_s8_acc<F>(C1[nn], A1, bh0, bh1);
                 if constexpr (RB == 8) {
                   mma_s8_acc<F>(C2[nn], A1, bl0, bl1);
-                  mma_s8_acc<F>(C3[nn], A2, bh0, bh1);
+                  mma_s8_acc<false>(C2[nn], A2, bh0, bh1);
                 } else {
                   mma_s8_acc<F>(C2[nn], A2, bl0, bl1);
                 }
@@ -442,8 +448,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
             float raw;
             if constexpr (RB == 8) {
               const int Z = C1[nn][c] * 256 + (C2[nn][c] + C1[nn][2 + c]);
-              const int Y = C2[nn][2 + c] + C3[nn][c];
-              raw = fmaf((float)Y, 1.0f / 256.0f, (float)Z);
+              raw = fmaf((float)C2[nn][2 + c], 1.0f / 256.0f, (float)Z);
             } else {
               // lanes g < 4: d2.kh, d0.kh (row g + 8), d2.kl; lanes g >= 4: d1.kh, d1.kl
               const bool top = g < 4;

@@ -214,19 +214,31 @@ __global__ void __launch_bounds__(kXRows, 2)
     for (int hf = 0; hf < 2; ++hf) {
       const int u = tid + 128 * hf;
       if (BITS == 3 && kv == 1) {
-        // V tile layout: u = (block, quad, 8-dim unit) group of four tokens
-        const int B = u >> 6, t4 = (u >> 4) & 3, un = u & 15;
+        // V tile layout: u = (block, quad, 8-dim unit) group of four tokens.  Lanes 4m ..
+        // 4m+3 take quads 0-3 of one unit, so a warp's 12-byte group loads hit 32 distinct
+        // banks.  A member's 16-byte tile row sits at chunk (2 quad + member bit 0) % 8 of
+        // a 128-byte line, the same line for every member of a unit; lanes with an odd unit
+        // store their members in the order 1 0 3 2 (nibbles swapped within each byte of
+        // the words), so each quarter-warp's stores cover the 8 chunks once.
+        const int t4 = u & 3, un = (u >> 2) & 15, B = u >> 6, jf = un & 1;
         const uint32_t* wp = reinterpret_cast<const uint32_t*>(
             blk + v_codes_off(D, BITS) + vt_group_off(D, B, t4, un));
         if (!in_bounds(vt_group_off(D, B, t4, un) + 12 <= kPage * CB, status)) continue;
+        const int sh = 4 * jf;
+        uint32_t w3[3];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const uint32_t x = wp[i];
+          w3[i] = ((x >> sh) & 0x0F0F0F0Fu) | ((x << sh) & 0xF0F0F0F0u);
+        }
         uint32_t o[4][4];
-        vdeq_group(wp[0], wp[1], wp[2], tl0, tl1, th0, th1, o);
+        vdeq_group(w3[0], w3[1], w3[2], tl0, tl1, th0, th1, o);  // o[j]: member j ^ jf
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int tkj = vt_member_slot(B, t4, j);
+          const int tkj = vt_member_slot(B, t4, j ^ jf);
           const int vo = (tkj >> 3) * 2048 + un * 128 + (tkj & 7) * 16;
           if (!in_bounds(vo + 16 <= SM::kOffRing - SM::kOffV, status)) continue;
-          st_v4(sV + (tkj >> 3) * 2048 + un * 128 + (tkj & 7) * 16, o[j]);
+          st_v4(sV + vo, o[j]);
         }
         continue;
       }
@@ -368,14 +380,18 @@ __global__ void __launch_bounds__(kXRows, 2)
         for (int j = 0; j < 64; ++j) x[j] = x[j] - m2;  // -inf - -inf = NaN: masked below
       } else {
         float am[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+        const float2 nm2 = make_float2(-m2, -m2);
 #pragma unroll
         for (int j4 = 0; j4 < 64; j4 += 4) {
           const float4 nk4 = *reinterpret_cast<const float4*>(nrm + j4);
-          const float nk[4] = {nk4.x, nk4.y, nk4.z, nk4.w};
+          // a_j = s_j nK_j - m2, two tokens per packed FMA
+          const float2 a01 = f2_fma(make_float2(x[j4], x[j4 + 1]), make_float2(nk4.x, nk4.y), nm2);
+          const float2 a23 = f2_fma(make_float2(x[j4 + 2], x[j4 + 3]), make_float2(nk4.z, nk4.w), nm2);
+          const float av[4] = {a01.x, a01.y, a23.x, a23.y};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = j4 + e;
-            float a = fmaf(x[j], nk[e], -m2);
+            float a = av[e];
             if constexpr (!FULL) a = page_ok && tok0 + j < my_lim ? a : -CUDART_INF_F;
             x[j] = a;
             am[e] = fmaxf(am[e], a);
@@ -405,24 +421,27 @@ __global__ void __launch_bounds__(kXRows, 2)
         }
       }
       uint32_t pw[32];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 ls01 = make_float2(0.f, 0.f), ls23 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int j4 = 0; j4 < 64; j4 += 4) {
         const float4 nv4 = *reinterpret_cast<const float4*>(nrm + 64 + j4);
-        const float nv[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
-        float p[4];
+        float pe[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float a = x[j4 + e];
-          float pe = ex2(a);  // a = -inf: 0
-          if constexpr (!FULL) pe = a == a ? pe : 0.f;  // NaN from a row with no score yet
-          ls[e] += pe;
-          p[e] = pe * nv[e];  // |v| / sigma'; masked tokens have p = 0
+          pe[e] = ex2(a);  // a = -inf: 0
+          if constexpr (!FULL) pe[e] = a == a ? pe[e] : 0.f;  // NaN from a row with no score yet
         }
-        pw[j4 / 2] = pack_f16x2(p[0], p[1]);
-        pw[j4 / 2 + 1] = pack_f16x2(p[2], p[3]);
+        // row sums and weights p |v| / sigma' (masked tokens have p = 0), two per instruction
+        const float2 p01 = make_float2(pe[0], pe[1]), p23 = make_float2(pe[2], pe[3]);
+        ls01 = f2_add(ls01, p01);
+        ls23 = f2_add(ls23, p23);
+        const float2 w01 = f2_mul(p01, make_float2(nv4.x, nv4.y));
+        const float2 w23 = f2_mul(p23, make_float2(nv4.z, nv4.w));
+        pw[j4 / 2] = pack_f16x2(w01.x, w01.y);
+        pw[j4 / 2 + 1] = pack_f16x2(w23.x, w23.y);
       }
-      lsum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      lsum += (ls01.x + ls01.y) + (ls23.x + ls23.y);
       tc::st32(t_row + kColP, pw);
     };
     if (full) softmax_page(std::true_type{});

@@ -31,6 +31,33 @@ __device__ __forceinline__ float ex2(float x) {
   return r;
 }
 
+// Packed pairs of binary32 operations (one instruction each, the same per-lane rounding
+// as the scalar forms): a * b + c, a * b, a + b.
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+  float2 o;
+  asm("{\n .reg .b64 pa, pb, pc, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n"
+      " mov.b64 pc, {%6, %7};\n fma.rn.f32x2 pd, pa, pb, pc;\n mov.b64 {%0, %1}, pd;\n}"
+      : "=f"(o.x), "=f"(o.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return o;
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+  float2 o;
+  asm("{\n .reg .b64 pa, pb, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n"
+      " mul.rn.f32x2 pd, pa, pb;\n mov.b64 {%0, %1}, pd;\n}"
+      : "=f"(o.x), "=f"(o.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return o;
+}
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+  float2 o;
+  asm("{\n .reg .b64 pa, pb, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n"
+      " add.rn.f32x2 pd, pa, pb;\n mov.b64 {%0, %1}, pd;\n}"
+      : "=f"(o.x), "=f"(o.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return o;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

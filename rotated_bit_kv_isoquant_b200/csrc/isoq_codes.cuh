@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "isoq_common.cuh"
+#include "isoq_ptx.cuh"
 
 namespace isoq {
 
@@ -61,6 +62,25 @@ __device__ __forceinline__ float add_code(float W, float z, float coef,
 }
 template <int BITS>
 constexpr float code_base() { return BITS == 4 ? 4.0f : (float)(1 << (BITS - 1)) - 0.5f; }
+
+// add_code<3> for two coordinates za, zb at once, into a pair of partial sums W2 of one
+// half-word (the half-word is W2.x + W2.y).  The six saturating decisions stay scalar; the
+// sums (s0 + s1) + (s2 + 0.5) and the accumulation run as packed f32x2 pairs with the same
+// per-lane rounding, and every value involved is a small exact half-integer, so the sum
+// equals the scalar add_code's bit for bit.
+__device__ __forceinline__ void add_code3_pair(float2& W2, float za, float zb, float coef_a,
+                                               float coef_b, const float (&TB)[3]) {
+  float sa[3], sb[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    sa[k] = __saturatef(fmaf(fabsf(za), 0x1p64f, -TB[k]));
+    sb[k] = __saturatef(fmaf(fabsf(zb), 0x1p64f, -TB[k]));
+  }
+  const float2 m = ptx::f2_add(ptx::f2_add(make_float2(sa[0], sb[0]), make_float2(sa[1], sb[1])),
+                               ptx::f2_add(make_float2(sa[2], sb[2]), make_float2(0.5f, 0.5f)));
+  W2 = ptx::f2_fma(make_float2(copysignf(coef_a, za), copysignf(coef_b, zb)), m, W2);
+}
+
 
 // Two half-word sums, each as the bits of W + 2^23 (0x4B000000 | W), joined into one word:
 // the high half's exponent bits leave the 32-bit product.

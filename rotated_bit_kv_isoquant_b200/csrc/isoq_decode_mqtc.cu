@@ -269,7 +269,12 @@ __global__ void __launch_bounds__(kXRows, 2)
 
   // Per page k: K_hat(k) -> tile; S(k) issued; V_hat(k) -> tile while S(k) runs; softmax;
   // O += P' V_hat issued, which runs while the next page's K_hat is dequantised.
+  // page-table entry of the next page, loaded one page ahead (off the per-page chain)
+  int phys_nx = n_my > 0 && in_bounds(p_begin < max_pages, status) ? __ldg(pt_row + p_begin) : -1;
   for (; k < n_my; ++k) {
+    const int phys = phys_nx;
+    if (k + 1 < n_my)
+      phys_nx = in_bounds(p_begin + k + 1 < max_pages, status) ? __ldg(pt_row + p_begin + k + 1) : -1;
     // Three CTA barriers per page; every other hand-off is a thread's own mbarrier wait.
     // The K tile is free: S(k-1) completed before this thread's softmax read it.
     bool ok = mbar_wait(bars + (k & 1), (k >> 1) & 1);
@@ -297,7 +302,6 @@ __global__ void __launch_bounds__(kXRows, 2)
     ok = k == 0 || mbar_wait(bar_pv, (k - 1) & 1);
     if (ok) dequant(k & 1, 1);
     const int pg = p_begin + k;
-    const int phys = __ldg(pt_row + pg);
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
     const bool full = page_ok && tok0 + kPage <= lim_lo;

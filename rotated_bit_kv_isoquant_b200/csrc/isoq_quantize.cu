@@ -432,21 +432,32 @@ __global__ void __launch_bounds__(kTpvThreads, ISOQ_TPV_MINB)
 #pragma unroll
     for (int hw = 0; hw < D / 4 / HPB; ++hw) {
       float W = code_base<BITS>() * (BITS == 2 ? 21845.0f : 4369.0f);  // sum coef * base
+      float2 W2 = make_float2(W, 0.f);  // 3 bits: the half-word as two partial sums
 #pragma unroll
       for (int hb = 0; hb < HPB; ++hb) {
         const int b = hw * HPB + hb;
+        float zr[4];
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           const float4 m = mh[4 * b + rr];
           // the chain starts from +0, so z is never -0 (which would code as negative)
-          const float z = fmaf(m.w, x[4 * b + 3],
-                               fmaf(m.z, x[4 * b + 2], fmaf(m.y, x[4 * b + 1], fmaf(m.x, x[4 * b], 0.0f))));
-          const int e = 4 * hb + rr;  // dim inside the half-word's dims
-          const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + e) & 7)))
-                                       : (float)(1 << (4 * e));
-          W = add_code<BITS>(W, z, coef, TB);
+          zr[rr] = fmaf(m.w, x[4 * b + 3],
+                        fmaf(m.z, x[4 * b + 2], fmaf(m.y, x[4 * b + 1], fmaf(m.x, x[4 * b], 0.0f))));
+        }
+        if constexpr (BITS == 3) {
+          add_code3_pair(W2, zr[0], zr[1], 1.0f, 16.0f, TB);
+          add_code3_pair(W2, zr[2], zr[3], 256.0f, 4096.0f, TB);
+        } else {
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            const int e = 4 * hb + rr;  // dim inside the half-word's dims
+            const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + e) & 7)))
+                                         : (float)(1 << (4 * e));
+            W = add_code<BITS>(W, zr[rr], coef, TB);
+          }
         }
       }
+      if constexpr (BITS == 3) W = W2.x + W2.y;
       half[hw] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W (W in [0, 65535])
     }
     uint32_t rec[CB / 4];

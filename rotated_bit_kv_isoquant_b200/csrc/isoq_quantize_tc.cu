@@ -294,9 +294,11 @@ __global__ void __launch_bounds__(kQtThreads, 2)
 #pragma unroll
       for (int hw = 0; hw < NHW; ++hw) {
         float W = code_base<BITS>() * (BITS == 2 ? 21845.0f : 4369.0f);  // sum coef * base
+        float2 W2 = make_float2(W, 0.f);  // 3 bits: the half-word as two partial sums
 #pragma unroll
         for (int hb = 0; hb < HPB; ++hb) {
           const int bl = hw * HPB + hb;  // block of the half
+          float zr[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float4 m = mh[4 * bl + e];
@@ -308,12 +310,21 @@ __global__ void __launch_bounds__(kQtThreads, 2)
                             make_float2(0.f, 0.f));
             p = fma2(make_float2(m.z, m.w),
                      make_float2(__uint_as_float(yb[2]), __uint_as_float(yb[3])), p);
-            const float z = p.x + p.y;
-            const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + 4 * hb + e) & 7)))
-                                         : (float)(1 << (4 * e));
-            W = add_code<BITS>(W, z, coef, TB);
+            zr[e] = p.x + p.y;
+          }
+          if constexpr (BITS == 3) {
+            add_code3_pair(W2, zr[0], zr[1], 1.0f, 16.0f, TB);
+            add_code3_pair(W2, zr[2], zr[3], 256.0f, 4096.0f, TB);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float coef = BITS == 2 ? (float)(1 << (2 * (slot2(8 * (hw & 1) + 4 * hb + e) & 7)))
+                                           : (float)(1 << (4 * e));
+              W = add_code<BITS>(W, zr[e], coef, TB);
+            }
           }
         }
+        if constexpr (BITS == 3) W = W2.x + W2.y;
         half[hw] = __float_as_uint(W + 8388608.0f);  // 0x4B000000 | W
       }
       constexpr int NR = CB / 8;  // words of half the record

@@ -347,13 +347,10 @@ __global__ void __launch_bounds__(kXRows, 2)
     tc::fence_after();
     float x[64];
     {
-      uint32_t sr[32];
+      uint32_t sr[64];
+      tc::ld64(t_row + kColS, sr);  // the row's 64 scores in one tensor-memory round trip
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        tc::ld32(t_row + kColS + 32 * hh, sr);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[32 * hh + j] = __uint_as_float(sr[j]);
-      }
+      for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sr[j]);
     }
     // FULL: every token of the page is valid for every row of the CTA (no masking).  The
     // exponents a_j = s_j - m2 come from one FMA each; the running maximum m2 moves only

@@ -272,6 +272,16 @@ int isoq_quantize_append_layers(const isoq_params* const* params,
  * contributing nothing (the -inf start of an empty chunk is never exponentiated: cf. the
  * same release's note on a NaN from a softmax chunk that starts at -inf).
  *
+ * Arithmetic (3 bits): the levels are given to four decimals, so each score is computed
+ * exactly in integers -- the levels as 10000 L[c] split into two signed bytes, the rotated
+ * query of a row scaled to 24 bits and split into three, products on the 8-bit tensor
+ * cores with 32-bit sums -- and the only rounding before the binary32 softmax is that of
+ * the query (relative ~1e-7).  The value sum uses binary16 operands (the levels times a
+ * scale at which they round by < 2e-5, the weights p |v| / sigma) with binary32
+ * accumulation.  Measured against a binary64 evaluation of the same codes: relative L2
+ * error per (sequence, head) <= 5e-4 on the five test workloads.  2 and 4 bits: binary16
+ * operands throughout, the query as a high and a low binary16 part.
+ *
  * Q: device [n_seqs][n_q_heads][d], element type q_dtype.  seq_lens: device int32
  * [n_seqs], the number of cached tokens each query attends (0 gives an all-zero output;
  * beyond the page table it is clamped and ISOQ_ST_LEN_RANGE set).  max_seq_len: a host

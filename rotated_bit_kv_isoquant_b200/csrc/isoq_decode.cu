@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(128)
   constexpr int E = D / 32;   // dims per lane
   constexpr int NB = E / 4;
   constexpr int PS = D + 4;
-  constexpr int UNROLL = 4;
+  constexpr int UNROLL = 8;  // one round of loads covers 32 chunks
   __shared__ float red_m[4];
   __shared__ float red_acc[4][D];
   __shared__ float red_l[4];

@@ -30,6 +30,7 @@
 
 #include <type_traits>
 
+#include "isoq_check.cuh"
 #include "isoq_common.cuh"
 #include "isoq_internal.h"
 #include "isoq_ptx.cuh"
@@ -116,12 +117,17 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   const int p_end = min((lim_hi + kPage - 1) / kPage, p_begin + pages_per_split);
 
   float* out_base = partials + ((size_t)s * n_q * n_q_heads) * n_splits * PS + (size_t)split * PS;
+  // extents of the checked build: partials / Q rows of the launch
+  [[maybe_unused]] const size_t parts_len = (size_t)gridDim.z * n_q * n_q_heads * n_splits * PS;
+  [[maybe_unused]] const size_t q_rows = (size_t)gridDim.z * n_q * n_q_heads;
+  [[maybe_unused]] const size_t out_off0 = out_base - partials;
   if (tid < 8) row_off[tid] = tid < nh ? row_index(tid) : 0;
   __syncthreads();
   if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
     for (int i = tid; i < nh * PS; i += blockDim.x) {
       const int h = i / PS, c = i - h * PS;
-      out_base[(size_t)row_off[h] * n_splits * PS + c] = (c == D) ? -CUDART_INF_F : 0.f;
+      const size_t o = (size_t)row_off[h] * n_splits * PS + c;
+      if (in_bounds(out_off0 + o < parts_len, status)) out_base[o] = (c == D) ? -CUDART_INF_F : 0.f;
     }
     return;
   }
@@ -140,8 +146,8 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
   auto issue = [&](int k) {  // lane 0 only
     const int pg = p_begin + warp + kWarps * k;
     const int st = k % NST;
-    const int phys = __ldg(pt_row + pg);
-    if (phys >= 0 && phys < n_pages) {
+    const int phys = in_bounds(pg < max_pages && st < NST, status) ? __ldg(pt_row + pg) : -1;
+    if (phys >= 0 && phys < n_pages && in_bounds(hk < H, status)) {
       mbar_expect_tx(mybar + st, BB);
       bulk_copy(myring + st * BB, blocks + ((size_t)phys * H + hk) * BB, BB, mybar + st);
     } else {
@@ -165,10 +171,11 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     const float* hp = params + (size_t)hk * D * 4;  // this head's block matrices
     float pq[NB][16];
 #pragma unroll
-    for (int k = 0; k < NB; ++k) load_block_mat(hp, lane * NB + k, pq[k]);
+    for (int k = 0; k < NB; ++k)
+      if (in_bounds(hk < H && lane * NB + k < D / 4, status)) load_block_mat(hp, lane * NB + k, pq[k]);
     for (int h = warp; h < 8; h += kWarps) {
       float v[E];
-      if (h < nh) {
+      if (h < nh && in_bounds((size_t)s * n_q * n_q_heads + row_off[h] < q_rows, status)) {
         const TQ* qp = Q + ((size_t)s * n_q * n_q_heads + row_off[h]) * D + lane * E;
 #pragma unroll
         for (int i = 0; i < E; ++i) v[i] = to_f32<TQ>(qp[i]);
@@ -191,6 +198,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
           hi[e] = __half2float(__float2half_rn(z[4 * k + e]));
           lo[e] = z[4 * k + e] - hi[e];
         }
+        if (!in_bounds(kb < D / 16 && h < 8, status)) continue;
         qa[kb * 32 + h * 4 + (q & 3)] =
             make_uint4(pack_f16x2(hi[0], hi[1]), pack_f16x2(lo[0], lo[1]),
                        pack_f16x2(hi[2], hi[3]), pack_f16x2(lo[2], lo[3]));
@@ -224,7 +232,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
     }
     const uint8_t* blk = myring + st * BB;
     const int pg = p_begin + warp + kWarps * k;
-    const int phys = __ldg(pt_row + pg);
+    const int phys = in_bounds(pg < max_pages && st < NST, status) ? __ldg(pt_row + pg) : -1;
     const bool page_ok = phys >= 0 && phys < n_pages;
     const int tok0 = pg * kPage;
 
@@ -241,15 +249,17 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
         uint32_t w[4][W];
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
-          const uint32_t* p =
-              reinterpret_cast<const uint32_t*>(blk + (tb + 8 * n + g) * CB) + W * (t + 4 * gq);
+          const int ko = (tb + 8 * n + g) * CB + 4 * W * (t + 4 * gq);
+          const uint32_t* p = reinterpret_cast<const uint32_t*>(blk + ko);
+          const bool kin = in_bounds(ko + 4 * W <= kPage * CB, status);
 #pragma unroll
-          for (int i = 0; i < W; ++i) w[n][i] = p[i];
+          for (int i = 0; i < W; ++i) w[n][i] = kin ? p[i] : 0u;
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint4 A0 = qa[(8 * gq + 2 * j) * 32 + lane];
-          const uint4 A1 = qa[(8 * gq + 2 * j + 1) * 32 + lane];
+          const bool ain = in_bounds(8 * gq + 2 * j + 1 < D / 16, status);
+          const uint4 A0 = ain ? qa[(8 * gq + 2 * j) * 32 + lane] : make_uint4(0, 0, 0, 0);
+          const uint4 A1 = ain ? qa[(8 * gq + 2 * j + 1) * 32 + lane] : make_uint4(0, 0, 0, 0);
           uint32_t f[4][4];
 #pragma unroll
           for (int n = 0; n < 4; ++n) kdeq<BITS>(w[n], j, tl0, tl1, th0, th1, f[n]);
@@ -267,10 +277,13 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
         const int tk = tb + 8 * n + 2 * t;
-        const float2 nk2 = __half22float2(
-            *reinterpret_cast<const __half2*>(blk + k_norm_off(D, BITS) + 2 * tk));
-        const float2 nv2 = __half22float2(
-            *reinterpret_cast<const __half2*>(blk + v_norm_off(D, BITS) + 2 * tk));
+        const bool nin = in_bounds(tk + 2 <= kPage, status);
+        const float2 nk2 = nin ? __half22float2(*reinterpret_cast<const __half2*>(
+                                     blk + k_norm_off(D, BITS) + 2 * tk))
+                               : make_float2(0.f, 0.f);
+        const float2 nv2 = nin ? __half22float2(*reinterpret_cast<const __half2*>(
+                                     blk + v_norm_off(D, BITS) + 2 * tk))
+                               : make_float2(0.f, 0.f);
         sv[n][0] = (C[n][0] + C[n][2]) * (nk2.x * kf);
         sv[n][1] = (C[n][1] + C[n][3]) * (nk2.y * kf);
         nv[n][0] = nv2.x;
@@ -348,7 +361,8 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
             const int tk = r + 2 * t + (x & 1) + 8 * (x >> 1);
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + tk * CB) + W * q;
+            const int vo = in_bounds(tk * CB + 4 * W * (q + 1) <= kPage * CB, status) ? tk * CB : 0;
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase + vo) + W * q;
             if constexpr (BITS == 3) {  // unit 3 = the spare bits of the three words
               const uint32_t w0 = w[0], w1 = w[1], w2 = w[2];
               S[x][0] = (odd ? w2 : w0) & 0x77777777u;
@@ -420,6 +434,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
         const int q = (g >> 1) + 4 * gq;
         const int j0 = 2 * (g & 1);
         const int d0 = 32 * q + 8 * j0 + 2 * mt;  // row g of m-tile; row g+8 is d0 + 1
+        if (!in_bounds(d0 + 1 < D && 2 * t + 1 < 8, status)) continue;
         float* r0 = mb + (warp * 8 + 2 * t) * PS;
         float* r1 = mb + (warp * 8 + 2 * t + 1) * PS;
         r0[d0] = acc[8 * gq + mt][0] * f;
@@ -451,6 +466,7 @@ __global__ void __launch_bounds__(kWarps * 32, dec_min_blocks<D>())
       }
     }
     float* o = out_base + (size_t)row_off[h] * n_splits * PS;
+    if (!in_bounds(out_off0 + (size_t)row_off[h] * n_splits * PS + D + 1 < parts_len, status)) continue;
     if (c < D) o[c] = v;
     else {
       o[D] = M == -CUDART_INF_F ? -CUDART_INF_F : M / kLog2e;  // natural-log units

@@ -7,8 +7,9 @@ library:
 
 Cases: the 1024-token GQA-4 workload (every code, every head), the 32k-token d = 256
 workload (sampled codes, every head), a ragged batch of the 64-sequence paged workload
-with single-token appends (every KV head of every sequence), and the two multi-token
-kernels.  Each case must leave the cache's status word at 0 (no index outside its extent,
+with single-token appends (every KV head of every sequence), the two multi-token kernels,
+the 2- and 4-bit formats (both rotation forms), and the RoPE-fused and layer-batched
+quantize-appends.  Each case must leave the cache's status word at 0 (no index outside its extent,
 no other condition) and stay within the parity tolerances.  One JSON line per case; exit
 status 0 when all pass.
 """
@@ -136,8 +137,63 @@ def case_multi_tc(oracle):
     return _multi_case(oracle, cfg, 32, edit)
 
 
+def case_formats(oracle):
+    # the 2- and 4-bit formats (the f16 decode kernel) with both rotation forms
+    recs = {}
+    for bits, rot in ((2, 0), (4, 1)):
+        cfg = wl.small_variant(wl.workload(2), length=1100)
+        run = Run(cfg, bits=bits, rot=rot)
+        run.prefill()
+        seqs, pos = _tokens(cfg, per_seq=256, seed=bits)
+        codes = codes_all(oracle, run, seqs, pos)
+        Q, out = run.decode()
+        att = check_attention(oracle, run, Q, out, cfg.decode_lens())
+        recs[f"b{bits}_r{rot}"] = {"codes": codes, "attention": att, "status": _status(run)}
+    return {"formats": recs, "status": max(r["status"] for r in recs.values())}
+
+
+def case_rope_layers(oracle):
+    # RoPE fused into the per-thread quantizer (a prefill and a decode step's appends), and
+    # the layer-batched append of the same step into three caches
+    from _gpu_util import check_codes, gather_records
+    cfg = wl.small_variant(wl.workload(4), n_seqs=4, len_range=(64, 700))
+    lay = wl.page_layout(cfg)
+    lens = cfg.prefill_lens()
+    tab = iq.isoq_rope_table(cfg.d, max(lens) + 1)
+    params = [iq.isoq_make_params(wl.PARAM_SEED + l, cfg.d, cfg.n_kv_heads) for l in range(3)]
+    caches = [iq.PagedCache(cfg.d, cfg.n_kv_heads, lay.n_pages, lay.page_table) for _ in range(3)]
+    for s, n in enumerate(lens):
+        K, V = wl.kv_tokens(cfg, s, 0, n, device="cuda", rope=False)
+        sid = torch.full((n,), s, dtype=torch.int32, device="cuda")
+        pos = torch.arange(n, dtype=torch.int32, device="cuda")
+        iq.isoq_quantize_append_rope(params[0], caches[0], K, V, sid, pos, tab)
+    sid = torch.arange(cfg.n_seqs, dtype=torch.int32, device="cuda")
+    pos = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(11)
+    Ks = [torch.randn((cfg.n_seqs, cfg.n_kv_heads, cfg.d), generator=g, device="cuda").bfloat16()
+          for _ in range(3)]
+    Vs = [torch.randn((cfg.n_seqs, cfg.n_kv_heads, cfg.d), generator=g, device="cuda").bfloat16()
+          for _ in range(3)]
+    iq.isoq_quantize_append_layers(params, caches, Ks, Vs, sid, pos, rope_table=tab)
+    torch.cuda.synchronize()
+    # the prefill codes of sequence 0 against the oracle's RoPE and quantiser
+    n0 = lens[0]
+    K0, V0 = wl.kv_tokens(cfg, 0, 0, n0, device="cuda", rope=False)
+    kc, kn, vc, vn = gather_records(caches[0], lay.page_table, np.zeros(n0, int), np.arange(n0),
+                                    cfg.d)
+    _, p32 = oracle.make_params_v(wl.PARAM_SEED, cfg.d, cfg.n_kv_heads, 0)
+    p64 = p32.astype(np.float64)
+    Kr = oracle.rope(K0.float().cpu().numpy().astype(np.float64),
+                     np.repeat(np.arange(n0), cfg.n_kv_heads), 10000.0)
+    sk = check_codes(oracle, p64, Kr, kc, kn, cfg.d)
+    sv = check_codes(oracle, p64, V0.float().cpu().numpy().astype(np.float64), vc, vn, cfg.d)
+    st = max(iq.isoq_get_status(c) for c in caches)
+    return {"codes": {k: sk[k] + sv[k] for k in sk}, "status": st}
+
+
 CASES = {"cfg1": case_cfg1, "cfg3": case_cfg3, "ragged": case_ragged,
-         "multi_mq": case_multi_mq, "multi_tc": case_multi_tc}
+         "multi_mq": case_multi_mq, "multi_tc": case_multi_tc, "formats": case_formats,
+         "rope_layers": case_rope_layers}
 
 
 def main(names):

@@ -2,8 +2,9 @@
 quantize and multi-token kernels compared with its extent (nvcc -DISOQ_CHECK_BOUNDS).
 
 A child process loads libisoq_checked.so (ISOQ_CHECK_BOUNDS=1) and runs the 1024-token
-workload, the 32k-token d = 256 workload, a ragged paged batch with appends and both
-multi-token kernels; every case must end with status 0 and parity green.  The self-test
+workload, the 32k-token d = 256 workload, a ragged paged batch with appends, both
+multi-token kernels, the 2- and 4-bit formats, and the RoPE-fused and layer-batched
+appends; every case must end with status 0 and parity green.  The self-test
 shows the check is live there (ISOQ_ST_BOUNDS set for an index equal to its extent) and
 compiled out of the normal library (status clear)."""
 import json
@@ -55,5 +56,5 @@ def test_checked_build_runs_clean():
             recs[r["case"]] = r
     assert p.returncode == 0, p.stdout[-4000:] + p.stderr[-4000:]
     assert recs["selftest"]["status"] == iq.ISOQ_ST_BOUNDS
-    for name in ("cfg1", "cfg3", "ragged", "multi_mq", "multi_tc"):
+    for name in ("cfg1", "cfg3", "ragged", "multi_mq", "multi_tc", "formats", "rope_layers"):
         assert recs[name]["ok"] and recs[name]["status"] == 0, recs[name]

@@ -112,8 +112,9 @@ def _tensor_peak():
 
 
 _KERNEL_SOURCES = {
-    "decode": ["isoq_decode_i8.cu", "isoq_decode.cu", "isoq_vtile.cuh", "isoq_ptx.cuh",
-               "isoq_common.cuh"],
+    # the 3-bit split kernel the decode profiles capture (the combine is < 3% of the call)
+    "decode": ["isoq_decode_i8.cu", "isoq_vtile.cuh", "isoq_ptx.cuh", "isoq_common.cuh",
+               "isoq_check.cuh", "isoq_internal.h"],
     "quantize": ["isoq_quantize_tc.cu", "isoq_quantize.cu", "isoq_codes.cuh", "isoq_tc.cuh",
                  "isoq_vtile.cuh", "isoq_common.cuh"],
 }

@@ -98,6 +98,9 @@ struct SplitPlan {
 #ifndef ISOQ_DEC_MIN_PAGES  // pages per decode CTA worth a launch
 #define ISOQ_DEC_MIN_PAGES 16
 #endif
+#ifndef ISOQ_DEC_MAX_CHUNK_PAGES  // longest decode chunk: a ragged batch sized by its
+#define ISOQ_DEC_MAX_CHUNK_PAGES 64  // longest sequence still gets chunks this short
+#endif
 #ifndef ISOQ_MQ_WAVES  // the same for the multi-token kernels
 #define ISOQ_MQ_WAVES 8
 #endif
@@ -125,6 +128,7 @@ SplitPlan plan_splits(int n_seqs, int n_q_heads, int n_kv_heads, int d, int max_
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   int pps = (int)((max_pages + want - 1) / want);
+  if (!shared_mq && pps > ISOQ_DEC_MAX_CHUNK_PAGES) pps = ISOQ_DEC_MAX_CHUNK_PAGES;
   if (pps < 1) pps = 1;
   if (pps > isoq::kMaxPagesPerSplit) pps = isoq::kMaxPagesPerSplit;
   int n_splits = (max_pages + pps - 1) / pps;

@@ -104,6 +104,19 @@ def test_split_plan_host_arithmetic():
     assert iq.raw_lib().isoq_decode_num_splits(1, 8, 4, 96, 100) == iq.ISOQ_E_DIM
 
 
+def test_split_plan_bounds_chunk_length():
+    # a decode chunk is at most 64 pages whatever the batch (a ragged batch is sized by its
+    # longest sequence), and at least 16 pages where the context has them
+    for (ns, hq, hkv, d, L) in [(64, 32, 8, 128, 65536), (2, 32, 8, 128, 1 << 20),
+                                (8, 64, 8, 128, 131072), (1, 32, 4, 128, 32768),
+                                (1, 16, 8, 256, 32768)]:
+        n = iq.isoq_decode_num_splits(ns, hq, hkv, d, L)
+        pages = -(-L // 64)
+        pps = -(-pages // n)
+        assert pps <= 64, (ns, L, n, pps)
+        assert pps >= min(16, pages) or n == 1, (ns, L, n, pps)
+
+
 def test_argument_validation_without_device():
     lib = iq.raw_lib()
     c = iq.isoq_cache(128, 2, 64, 4, 2, 1, None, None, None)

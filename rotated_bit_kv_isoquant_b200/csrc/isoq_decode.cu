@@ -169,10 +169,12 @@ static cudaError_t launch_combine(dim3 grid, cudaStream_t stream, bool dependent
 
 template <int D>
 static cudaError_t launch_dq(const DecodeArgs& a, cudaStream_t stream) {
+  bool combined = false;  // a single-chunk 3-bit decode writes the output itself
   cudaError_t e = use_shared_mq(a) ? launch_decode_split_mq(a, stream)
-                  : a.bits == 3    ? launch_decode_split_i8(a, stream)
+                  : a.bits == 3    ? launch_decode_split_i8(a, stream, &combined)
                                    : launch_decode_split_mma(a, stream);
   if (e != cudaSuccess) return e;
+  if (combined) return cudaSuccess;
   const int rows = a.n_q * a.n_q_heads;
   dim3 grid(rows, a.n_seqs);
   const size_t PS = partial_stride(D);

@@ -131,7 +131,8 @@ struct I8Smem {
   static constexpr int kKfOff = kA2Off + (D / 32) * 32 * 16;           // float [8]
   static constexpr int kRowOff = kKfOff + 8 * 4;                      // int [8]
   static constexpr int kBytes = kRowOff + 8 * 4;
-  static constexpr int kMergeBytes = NW * 8 * (D + 4) * 4;
+  // the warps' states [NW][8][D + 4] and, for a single chunk, the merged rows [8][D + 1]
+  static constexpr int kMergeBytes = NW * 8 * (D + 4) * 4 + 8 * (D + 1) * 4;
   static_assert(kMergeBytes <= kRing, "merge buffer must fit in the ring");
   static_assert(kAOff % 16 == 0 && kA2Off % 16 == 0, "A fragments must be aligned");
 };
@@ -162,13 +163,17 @@ constexpr int i8_min_blocks(int nw) {
 // GPU holds gives each CTA more warps (16 at d = 128, 8 at d = 256), so that the pages of
 // a chunk are in flight at once instead of one after another per warp, at the cost of one
 // query rotation and one merge per CTA as before.
+// out (decode with a single chunk only, else null): the CTA holds the whole context of its
+// rows, so it finishes the combine itself -- normalise, inverse rotation -- and writes the
+// output rows [n_seqs][n_q_heads][D] instead of partials.
 template <int D, int NST, int RB, typename TQ, bool MQ, int NW>
 __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
     decode_i8_kernel(const float* __restrict__ params, const uint8_t* __restrict__ blocks,
                      const int32_t* __restrict__ page_table, int n_pages, int max_pages, int H,
                      const TQ* __restrict__ Q, int n_q_heads, int n_q,
                      const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
-                     int n_splits, float* __restrict__ partials, uint32_t* status) {
+                     int n_splits, float* __restrict__ partials, uint32_t* status,
+                     float* __restrict__ out) {
   using SM = I8Smem<D, NST, RB, NW>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
@@ -224,7 +229,17 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
   [[maybe_unused]] const size_t out_off0 = out_base - partials;
   if (tid < RB) row_off[tid] = tid < nh ? row_index(tid) : 0;
   __syncthreads();
+  // extent of the direct output (single chunk): [gridDim.z][n_q_heads][D]
+  [[maybe_unused]] const size_t out_len = (size_t)gridDim.z * n_q_heads * D;
   if (p_begin >= p_end) {  // empty chunk: m = -inf, l = 0, acc = 0
+    if (out != nullptr) {  // the whole context is empty: zero output rows
+      for (int i = tid; i < nh * D; i += blockDim.x) {
+        const int h = i / D, c = i - h * D;
+        const size_t o = ((size_t)s * n_q_heads + row_off[h]) * D + c;
+        if (in_bounds(o < out_len, status)) out[o] = 0.f;
+      }
+      return;
+    }
     for (int i = tid; i < nh * PS; i += blockDim.x) {
       const int h = i / PS, c = i - h * PS;
       const size_t o = (size_t)row_off[h] * n_splits * PS + c;
@@ -651,6 +666,11 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
         v += sc * mb[(w * 8 + h) * PS + (c == D ? D + 1 : c)];
       }
     }
+    if (out != nullptr) {  // single chunk: the merged row goes on to the rotation below
+      if (in_bounds(NW * 8 * PS + h * (D + 1) + c < SM::kRing / 4, status))
+        mb[NW * 8 * PS + h * (D + 1) + c] = v;
+      continue;
+    }
     float* o = out_base + (size_t)row_off[h] * n_splits * PS;
     if (!in_bounds(out_off0 + (size_t)row_off[h] * n_splits * PS + D + 1 < parts_len, status)) continue;
     if (c < D) o[c] = v;
@@ -659,10 +679,36 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
       o[D + 1] = v;
     }
   }
+  if (out == nullptr) return;
+  // ---- a9 for a single chunk: o = acc / l, inverse SO(4) blocks, inverse WHT, as the
+  // combine computes it for one part (bitwise the same); a warp per row
+  __syncthreads();
+  const float* fin = mb + NW * 8 * PS;  // [nh][D + 1]: acc, l
+  const float* hp = params + (size_t)hk * D * 4;
+  float Mb[NB][16];
+#pragma unroll
+  for (int k = 0; k < NB; ++k)
+    if (in_bounds(hk < H && lane * NB + k < D / 4, status)) load_block_mat(hp, lane * NB + k, Mb[k]);
+  for (int h = warp; h < nh; h += NW) {
+    const float Ls = fin[h * (D + 1) + D];
+    const float inv = Ls > 0.f ? 1.f / (Ls * sqrtf((float)D)) : 0.f;
+    float o[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) o[i] = fin[h * (D + 1) + lane * E + i] * inv;
+    float y[E];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) mat_inv(Mb[k], o + 4 * k, y + 4 * k);
+    wht_warp<E>(y, lane);
+    const float rs = rsqrtf((float)D);
+    const size_t ob = ((size_t)s * n_q_heads + row_off[h]) * D + lane * E;
+    if (!in_bounds(ob + E <= out_len, status)) continue;
+#pragma unroll
+    for (int i = 0; i < E; ++i) out[ob + i] = y[i] * rs;
+  }
 }
 
 template <int D, int NST, int RB, typename TQ, bool MQ, int NW>
-cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream, float* direct_out) {
   using SM = I8Smem<D, NST, RB, NW>;
   // the dynamic shared-memory opt-in is per function and per device
   static unsigned long long attr_set = 0;
@@ -680,7 +726,7 @@ cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream) {
   decode_i8_kernel<D, NST, RB, TQ, MQ, NW><<<grid, NW * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
-      a.n_splits, a.partials, a.status);
+      a.n_splits, a.partials, a.status, direct_out);
   return cudaGetLastError();
 }
 
@@ -688,29 +734,29 @@ cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream) {
 // GPU would otherwise run a small decode with a few warps per SM, each walking its pages
 // one after another.
 template <int D, int NST, int RB, typename TQ, bool MQ>
-cudaError_t launch_i8_w(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t launch_i8_w(const DecodeArgs& a, cudaStream_t stream, float* direct_out) {
   constexpr int kWide = D == 128 ? 16 : 8;
   const int G = a.n_q_heads / a.n_kv_heads;
   const long long ctas =
       (long long)a.n_splits * a.n_kv_heads * ((a.n_q * G + RB - 1) / RB) * a.n_seqs;
   if (ctas <= (long long)decode_i8_sms())
-    return launch_i8_t<D, NST, RB, TQ, MQ, kWide>(a, stream);
-  return launch_i8_t<D, NST, RB, TQ, MQ, 4>(a, stream);
+    return launch_i8_t<D, NST, RB, TQ, MQ, kWide>(a, stream, direct_out);
+  return launch_i8_t<D, NST, RB, TQ, MQ, 4>(a, stream, direct_out);
 }
 
 template <int D, int NST, int RB>
-cudaError_t launch_i8_rb(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t launch_i8_rb(const DecodeArgs& a, cudaStream_t stream, float* direct_out) {
   const bool mq = a.n_q > 1;
   switch (a.q_dtype) {
     case ISOQ_F32:
-      return mq ? launch_i8_w<D, NST, RB, float, true>(a, stream)
-                : launch_i8_w<D, NST, RB, float, false>(a, stream);
+      return mq ? launch_i8_w<D, NST, RB, float, true>(a, stream, nullptr)
+                : launch_i8_w<D, NST, RB, float, false>(a, stream, direct_out);
     case ISOQ_BF16:
-      return mq ? launch_i8_w<D, NST, RB, __nv_bfloat16, true>(a, stream)
-                : launch_i8_w<D, NST, RB, __nv_bfloat16, false>(a, stream);
+      return mq ? launch_i8_w<D, NST, RB, __nv_bfloat16, true>(a, stream, nullptr)
+                : launch_i8_w<D, NST, RB, __nv_bfloat16, false>(a, stream, direct_out);
     case ISOQ_F16:
-      return mq ? launch_i8_w<D, NST, RB, __half, true>(a, stream)
-                : launch_i8_w<D, NST, RB, __half, false>(a, stream);
+      return mq ? launch_i8_w<D, NST, RB, __half, true>(a, stream, nullptr)
+                : launch_i8_w<D, NST, RB, __half, false>(a, stream, direct_out);
   }
   return cudaErrorInvalidValue;
 }
@@ -724,14 +770,25 @@ cudaError_t launch_i8_rb(const DecodeArgs& a, cudaStream_t stream) {
 #define ISOQ_I8_NST256 2
 #endif
 
-cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream) {
+#ifndef ISOQ_I8_DIRECT  // single-chunk decodes write their output without the combine
+#define ISOQ_I8_DIRECT 1
+#endif
+
+cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream, bool* combined) {
+  if (combined) *combined = false;
   if (a.bits != 3) return cudaErrorInvalidValue;
+  const bool direct = ISOQ_I8_DIRECT && combined && a.n_splits == 1 && a.n_q == 1 &&
+                      a.state == nullptr && a.out != nullptr;
+  float* out = direct ? a.out : nullptr;
   const int rb = decode_rows_per_block(a.d, a.n_q, a.n_q_heads / a.n_kv_heads);
+  cudaError_t e = cudaErrorInvalidValue;
   if (a.d == 128)
-    return rb == 8 ? launch_i8_rb<128, ISOQ_I8_NST128, 8>(a, stream)
-                   : launch_i8_rb<128, ISOQ_I8_NST128, 4>(a, stream);
-  if (a.d == 256) return launch_i8_rb<256, ISOQ_I8_NST256, 4>(a, stream);
-  return cudaErrorInvalidValue;
+    e = rb == 8 ? launch_i8_rb<128, ISOQ_I8_NST128, 8>(a, stream, out)
+                : launch_i8_rb<128, ISOQ_I8_NST128, 4>(a, stream, out);
+  else if (a.d == 256)
+    e = launch_i8_rb<256, ISOQ_I8_NST256, 4>(a, stream, out);
+  if (e == cudaSuccess && combined) *combined = direct;
+  return e;
 }
 
 // Resident 4-warp CTAs per SM of the decode kernel for head dimension d on the current

@@ -75,8 +75,11 @@ cudaError_t launch_merge_states(const float* params, int n_kv_heads, int d, int 
 cudaError_t launch_decode_split_mma(const DecodeArgs& a, cudaStream_t stream);
 // Resident CTAs per SM of that kernel for head dimension d on the current device.
 int decode_resident_ctas(int d);
-// The 3-bit split kernel on 8-bit integer tensor-core products (partials only).
-cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream);
+// The 3-bit split kernel on 8-bit integer tensor-core products.  With `combined` non-null,
+// a decode with a single context chunk writes its output directly (no combine needed:
+// *combined is set); otherwise partials only.
+cudaError_t launch_decode_split_i8(const DecodeArgs& a, cudaStream_t stream,
+                                   bool* combined = nullptr);
 int decode_i8_resident_ctas(int d);
 // Rows ((query token, head) pairs of one KV head) per CTA of the 3-bit split kernel: 4
 // when a KV head has at most 4 rows (the query digits of all of them then fit the 16 rows

@@ -77,6 +77,32 @@ __device__ __forceinline__ void mma_s8_first(int (&c)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The decode is bound by the logic pipe (byte permutes, shifts, masks) and by the latency of
+// its dependent chains.  A code word's selector (its nibbles with the top bit clear) is
+// formed as w - top_bits(w) on the multiply-add pipe, which has room to spare; the -1 is a
+// kernel argument so that the compiler keeps the multiply-add instead of folding it back
+// into a logic operation.  (Right shifts as high words of products lengthen the chains more
+// than they relieve the logic pipe, so the spare unit and the upper halves stay shifts.)
+struct I8Mul {
+  uint32_t neg1;
+};
+__device__ __forceinline__ uint32_t mad_lo_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+// Top bits of the nibbles of a code word (the spare unit's bits)
+__device__ __forceinline__ uint32_t top_bits(uint32_t w) { return w & 0x88888888u; }
+// Selector word of a code word: its nibbles with the top bit clear
+__device__ __forceinline__ uint32_t sel_word(uint32_t w, uint32_t top, const I8Mul& mk) {
+  return mad_lo_u32(top, mk.neg1, w);
+}
+// The spare unit's selector from the three top-bit words: nibble k = bits 4k+3 of w0, w1,
+// w2 as bits 2, 1, 0
+__device__ __forceinline__ uint32_t sel_spare(uint32_t t0, uint32_t t1, uint32_t t2) {
+  return (t2 >> 3) | (t1 >> 2) | (t0 >> 1);
+}
+
 template <bool FIRST>
 __device__ __forceinline__ void mma_s8_acc(int (&c)[4], uint4 a, uint32_t b0, uint32_t b1) {
   if constexpr (FIRST) mma_s8_first(c, a.x, a.y, a.z, a.w, b0, b1);
@@ -173,7 +199,7 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
                      const TQ* __restrict__ Q, int n_q_heads, int n_q,
                      const int32_t* __restrict__ seq_lens, float scale, int pages_per_split,
                      int n_splits, float* __restrict__ partials, uint32_t* status,
-                     float* __restrict__ out) {
+                     float* __restrict__ out, const I8Mul mk) {
   using SM = I8Smem<D, NST, RB, NW>;
   constexpr int E = D / 32;           // elements per lane in the warp WHT layout
   constexpr int NB = E / 4;
@@ -407,15 +433,17 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
         int C1[kI8NT][4], C2[kI8NT][4];
 #pragma unroll
         for (int gq = 0; gq < NG; ++gq) {
-          uint32_t w[kI8NT][3];
+          uint32_t w[kI8NT][3], wt[kI8NT][3];
 #pragma unroll
           for (int nn = 0; nn < kI8NT; ++nn) {
             const int ko = (tb + 8 * (n0 + nn) + g) * CB + 12 * (t + 4 * gq);
             const uint32_t* p = reinterpret_cast<const uint32_t*>(blk + ko);
             const bool kin = in_bounds(ko + 12 <= kPage * CB, status);
-            w[nn][0] = kin ? p[0] : 0u;
-            w[nn][1] = kin ? p[1] : 0u;
-            w[nn][2] = kin ? p[2] : 0u;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+              w[nn][j] = kin ? p[j] : 0u;
+              wt[nn][j] = top_bits(w[nn][j]);
+            }
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -427,10 +455,8 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
                                  : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int nn = 0; nn < kI8NT; ++nn) {
-              const uint32_t S = u == 0 ? (w[nn][0] & 0x77777777u)
-                               : u == 1 ? (w[nn][1] & 0x77777777u)
-                               : u == 2 ? (w[nn][2] & 0x77777777u)
-                                        : spare_codes(w[nn][0], w[nn][1], w[nn][2]);
+              const uint32_t S = u < 3 ? sel_word(w[nn][u], wt[nn][u], mk)
+                                       : sel_spare(wt[nn][0], wt[nn][1], wt[nn][2]);
               const uint32_t S2 = S >> 16;
               const uint32_t bh0 = prmt(kh0, kh1, S), bh1 = prmt(kh0, kh1, S2);
               const uint32_t bl0 = prmt(kl0, kl1, S), bl1 = prmt(kl0, kl1, S2);
@@ -571,11 +597,14 @@ __global__ void __launch_bounds__(NW * 32, i8_min_blocks<D>(NW))
 #pragma unroll
           for (int p = 0; p < 2; ++p) {      // unit 2 (g + 8 up) + p
             const uint32_t* w = W + 3 * p;
-            const uint32_t Sp = spare_codes(w[0], w[1], w[2]);
+            const uint32_t wt0 = top_bits(w[0]), wt1 = top_bits(w[1]), wt2 = top_bits(w[2]);
+            const uint32_t Sp = sel_spare(wt0, wt1, wt2);
 #pragma unroll
             for (int b = 0; b < 4; ++b) {    // words 0..2, then the spare unit
               const int mt = 8 * up + 4 * p + b;
-              const uint32_t S = b < 3 ? (w[b] & 0x77777777u) : Sp;
+              const uint32_t S = b == 0 ? sel_word(w[0], wt0, mk)
+                               : b == 1 ? sel_word(w[1], wt1, mk)
+                               : b == 2 ? sel_word(w[2], wt2, mk) : Sp;
               // low half: dim 8u + 2b of members 0-3 (row g); high half: dim + 1 (row g+8)
               const uint32_t Sh = S >> 16;
               const uint32_t le = prmt(tl0, tl1, S), he = prmt(th0, th1, S);
@@ -726,7 +755,8 @@ cudaError_t launch_i8_t(const DecodeArgs& a, cudaStream_t stream, float* direct_
   decode_i8_kernel<D, NST, RB, TQ, MQ, NW><<<grid, NW * 32, SM::kBytes, stream>>>(
       a.params, a.blocks, a.page_table, a.n_pages, a.max_pages, a.n_kv_heads,
       static_cast<const TQ*>(a.Q), a.n_q_heads, a.n_q, a.seq_lens, a.scale, a.pages_per_split,
-      a.n_splits, a.partials, a.status, direct_out);
+      a.n_splits, a.partials, a.status, direct_out,
+      I8Mul{0xFFFFFFFFu});
   return cudaGetLastError();
 }
 

@@ -176,6 +176,7 @@ def _len_run(cfg, lens):
 @pytest.mark.parametrize("d,G,lens,hint", [
     (128, 4, (1, 63, 64, 65), None),
     (128, 8, (0, 5, 200, 1000), 4096),        # empty sequence + many empty splits
+    (128, 4, (0, 17, 900), None),             # empty sequence, one chunk: no combine
     (128, 1, (129, 3000), None),
     (128, 16, (777,), None),
     (256, 2, (1, 64, 130), None),

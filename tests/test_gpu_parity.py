@@ -196,6 +196,28 @@ def test_edge_lengths(oracle, d, G, lens, hint):
     assert iq.isoq_get_status(run.cache) == 0
 
 
+@pytest.mark.parametrize("d,G,lens", [(128, 8, (0, 300, 900)), (128, 4, (1, 64, 1000)),
+                                      (256, 2, (5, 700))])
+def test_single_chunk_output_matches_combine(oracle, d, G, lens):
+    """A decode whose contexts fit one chunk writes its output rows from the split kernel
+    (normalisation and inverse rotation there, no combine launch).  The same decode planned
+    for a longer context (a larger length hint: several chunks, all but the first empty) goes
+    through the partials and the combine; the two outputs are bitwise equal."""
+    cfg, lens = _custom(d=d, G=G, lens=lens)
+    run = _len_run(cfg, lens)
+    run.prefill()
+    Q = wl.queries(cfg, device="cuda")
+    hq = cfg.n_kv_heads * G
+    assert iq.isoq_decode_num_splits(len(lens), hq, cfg.n_kv_heads, d, max(lens)) == 1
+    assert iq.isoq_decode_num_splits(len(lens), hq, cfg.n_kv_heads, d, 16384) > 1
+    Q, direct = run.decode(Q=Q, lens=lens)
+    Q, merged = run.decode(Q=Q, lens=lens, max_len=16384)
+    assert torch.equal(direct, merged)
+    _log(f"direct_d{d}_G{G}_{'-'.join(map(str, lens))}",
+         check_attention(oracle, run, Q, direct, lens))
+    assert iq.isoq_get_status(run.cache) == 0
+
+
 @pytest.mark.parametrize("kv_dtype,q_dtype", [(torch.float16, torch.float16),
                                               (torch.bfloat16, torch.float32),
                                               (torch.float32, torch.bfloat16)])
